@@ -1,0 +1,451 @@
+// fb_api.cu -- the extern "C" entry points of libflashblock.so: argument
+// checks, work decomposition (query-row tiles, key-range splits), TMA tensor
+// maps and kernel dispatch.  See include/flashblock.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "fb_internal.h"
+
+namespace fb {
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 4-D bf16 tensor map, innermost dimension first, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides_bytes[3],
+              const uint32_t box[4]) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t gs[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
+  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static int cache[64] = {0};
+  if (dev < 64 && cache[dev]) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int log2i(int x) {
+  int s = 0;
+  while ((1 << s) < x) ++s;
+  return s;
+}
+
+int64_t cache_rows(const fb_desc& d) {
+  return d.page_size > 0 ? (int64_t)d.max_pages * d.page_size : (int64_t)d.kv_capacity;
+}
+
+fb_status check_desc(const fb_desc* d) {
+  if (!d) return FB_ERR_INVALID_ARG;
+  if (d->batch <= 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->head_dim <= 0 ||
+      d->block_len <= 0)
+    return FB_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads) return FB_ERR_INVALID_ARG;
+  if (!(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale)) return FB_ERR_INVALID_ARG;
+  if (d->dtype == FB_BF16) {
+    if (d->head_dim != TC_D) return FB_ERR_UNSUPPORTED;
+    const int G = d->num_q_heads / d->num_kv_heads;
+    if (!pow2(G) || G > TC_BM) return FB_ERR_UNSUPPORTED;
+  } else if (d->dtype == FB_FP32) {
+    if (d->head_dim % 32 || d->head_dim > 128) return FB_ERR_UNSUPPORTED;
+  } else {
+    return FB_ERR_UNSUPPORTED;
+  }
+  return FB_OK;
+}
+
+fb_status check_cache(const fb_desc* d) {
+  if (!d->prefix_lens || (reinterpret_cast<uintptr_t>(d->prefix_lens) & 3u)) return FB_ERR_INVALID_ARG;
+  if (d->page_size > 0) {
+    if (!pow2(d->page_size) || d->page_size < 64) return FB_ERR_UNSUPPORTED;
+    if (!d->block_table || d->max_pages <= 0 || d->num_pages <= 0) return FB_ERR_INVALID_ARG;
+    if (cache_rows(*d) > (int64_t)1 << 30) return FB_ERR_UNSUPPORTED;
+  } else {
+    if (d->page_size < 0 || d->kv_capacity < 0) return FB_ERR_INVALID_ARG;
+  }
+  return FB_OK;
+}
+
+fb_status check_sparse(const fb_desc* d, const int32_t* chunk_idx) {
+  if (d->topk < 0) return FB_ERR_INVALID_ARG;
+  if (d->topk == 0) return FB_OK;
+  if (!chunk_idx) return FB_ERR_INVALID_ARG;
+  if (d->chunk_size <= 0 || d->chunk_size % TC_BN) return FB_ERR_UNSUPPORTED;
+  return FB_OK;
+}
+
+KeySource key_source(const fb_desc& d, bool prefix, bool block, const int32_t* chunk_idx) {
+  KeySource s;
+  std::memset(&s, 0, sizeof(s));
+  s.has_prefix = prefix;
+  s.has_block = block;
+  if (prefix) {
+    s.paged = d.page_size > 0;
+    s.page_shift = s.paged ? log2i(d.page_size) : 0;
+    s.max_pages = d.max_pages;
+    s.num_pages = d.num_pages;
+    s.cap = (int)cache_rows(d);
+    s.block_table = d.block_table;
+    s.prefix_lens = d.prefix_lens;
+    s.chunk_idx = (d.topk > 0) ? chunk_idx : nullptr;
+    s.topk = d.topk;
+    s.chunk_size = d.chunk_size;
+  }
+  return s;
+}
+
+AttnParams base_params(const fb_desc& d) {
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = d.batch;
+  p.Hq = d.num_q_heads;
+  p.Hkv = d.num_kv_heads;
+  p.G = d.num_q_heads / d.num_kv_heads;
+  p.S = d.block_len;
+  p.D = d.head_dim;
+  p.n_rt = (d.block_len * p.G + TC_BM - 1) / TC_BM;
+  p.nsplit = 1;
+  p.scale = d.softmax_scale;
+  p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  return p;
+}
+
+// Key-range splits of the prefix pass: enough CTAs to fill the GPU once, at
+// least 4 key tiles per split.
+int choose_splits(const fb_desc& d, long long est_tiles) {
+  if (d.dtype != FB_BF16) return 1;
+  const int G = d.num_q_heads / d.num_kv_heads;
+  const long long units = (long long)d.batch * d.num_kv_heads * ((d.block_len * G + TC_BM - 1) / TC_BM);
+  long long max_ns = est_tiles / 4;
+  if (max_ns < 1) max_ns = 1;
+  if (d.num_splits > 0) return (int)std::min<long long>(d.num_splits, std::max<long long>(est_tiles, 1));
+  const long long slots = device_sms();
+  if (units >= slots) {
+    int best = 1;
+    double best_eff = 0;
+    for (int ns = 1; ns <= 4 && ns <= max_ns; ++ns) {
+      const double w = (double)(units * ns) / (double)slots;
+      const double eff = w / std::ceil(w);
+      if (eff > best_eff + 0.05) {
+        best_eff = eff;
+        best = ns;
+      }
+    }
+    return best;
+  }
+  long long ns = slots / units;
+  if (ns > max_ns) ns = max_ns;
+  return (int)std::max<long long>(ns, 1);
+}
+
+long long prefix_tiles_estimate(const fb_desc& d) {
+  if (d.topk > 0) return (long long)d.topk * ((d.chunk_size + TC_BN - 1) / TC_BN);
+  return (cache_rows(d) + TC_BN - 1) / TC_BN;
+}
+
+size_t split_bytes(const fb_desc& d, int ns) {
+  if (ns <= 1) return 0;
+  const size_t rows = (size_t)d.batch * d.block_len * d.num_q_heads;
+  return (size_t)ns * rows * (size_t)(d.head_dim + 1) * sizeof(float);
+}
+
+fb_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FB_OK : FB_ERR_LAUNCH; }
+
+struct Maps {
+  CUtensorMap q, kp, vp, kb, vb;
+};
+
+bool q_map(CUtensorMap* m, const fb_desc& d, const void* Q) {
+  const int G = d.num_q_heads / d.num_kv_heads;
+  const uint64_t D = d.head_dim, Hq = d.num_q_heads, S = d.block_len, B = d.batch;
+  const uint64_t dims[4] = {D, Hq, S, B};
+  const uint64_t str[3] = {D * 2, Hq * D * 2, S * Hq * D * 2};
+  const uint32_t box[4] = {64, (uint32_t)G, (uint32_t)(TC_BM / G), 1};
+  return make_map(m, Q, dims, str, box);
+}
+
+bool block_map(CUtensorMap* m, const fb_desc& d, const void* X) {
+  const uint64_t D = d.head_dim, H = d.num_kv_heads, S = d.block_len, B = d.batch;
+  const uint64_t dims[4] = {D, H, S, B};
+  const uint64_t str[3] = {D * 2, H * D * 2, S * H * D * 2};
+  const uint32_t box[4] = {64, 1, TC_BN, 1};
+  return make_map(m, X, dims, str, box);
+}
+
+bool cache_map(CUtensorMap* m, const fb_desc& d, const void* X) {
+  const uint64_t D = d.head_dim, H = d.num_kv_heads;
+  if (d.page_size > 0) {
+    const uint64_t P = d.page_size, N = d.num_pages;
+    const uint64_t dims[4] = {D, H, P, N};
+    const uint64_t str[3] = {D * 2, H * D * 2, P * H * D * 2};
+    const uint32_t box[4] = {64, 1, (uint32_t)(d.page_size < TC_BN ? d.page_size : TC_BN), 1};
+    return make_map(m, X, dims, str, box);
+  }
+  const uint64_t cap = d.kv_capacity > 0 ? (uint64_t)d.kv_capacity : 1, B = d.batch;
+  const uint64_t dims[4] = {D, H, cap, B};
+  const uint64_t str[3] = {D * 2, H * D * 2, cap * H * D * 2};
+  const uint32_t box[4] = {64, 1, TC_BN, 1};
+  return make_map(m, X, dims, str, box);
+}
+
+}  // namespace
+}  // namespace fb
+
+using namespace fb;
+
+extern "C" {
+
+int64_t fb_cache_rows(const fb_desc* d) { return d ? cache_rows(*d) : -1; }
+
+size_t fb_workspace_bytes(const fb_desc* d) {
+  if (check_desc(d) != FB_OK) return 0;
+  const int ns_pre = choose_splits(*d, prefix_tiles_estimate(*d));
+  fb_desc dense = *d;
+  dense.topk = 0;
+  const int ns_full = choose_splits(dense, prefix_tiles_estimate(dense) + (d->block_len + TC_BN - 1) / TC_BN);
+  const size_t a = split_bytes(*d, ns_pre), b = split_bytes(*d, ns_full);
+  return a > b ? a : b;
+}
+
+fb_status fb_prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const void* Vc,
+                            const int32_t* chunk_idx, float* O_pre, float* LSE_pre, void* ws,
+                            size_t ws_bytes, int32_t* dev_status, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if ((st = check_cache(d)) != FB_OK) return st;
+  if ((st = check_sparse(d, chunk_idx)) != FB_OK) return st;
+  if (!Q || !Kc || !Vc || !O_pre || !LSE_pre) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O_pre) ||
+      (reinterpret_cast<uintptr_t>(LSE_pre) & 3u))
+    return FB_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  AttnParams p = base_params(*d);
+  p.src = key_source(*d, true, false, chunk_idx);
+  p.epi = EPI_PARTIAL;
+  p.dev_status = dev_status;
+  if (d->dtype == FB_FP32) {
+    p.out_o32 = O_pre;
+    p.out_lse = LSE_pre;
+    return from_cuda(launch_attn_simt(p, static_cast<const float*>(Q), static_cast<const float*>(Kc),
+                                      static_cast<const float*>(Vc), nullptr, nullptr, s));
+  }
+  const int ns = choose_splits(*d, prefix_tiles_estimate(*d));
+  const size_t need = split_bytes(*d, ns);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return FB_ERR_WORKSPACE;
+  Maps m;
+  if (!q_map(&m.q, *d, Q) || !cache_map(&m.kp, *d, Kc) || !cache_map(&m.vp, *d, Vc))
+    return FB_ERR_LAUNCH;
+  p.nsplit = ns;
+  float* part_o = O_pre;
+  float* part_l = LSE_pre;
+  if (ns > 1) {
+    part_o = static_cast<float*>(ws);
+    part_l = part_o + (size_t)ns * d->batch * d->block_len * d->num_q_heads * d->head_dim;
+  }
+  p.out_o32 = part_o;
+  p.out_lse = part_l;
+  const long long grid = (long long)d->batch * d->num_kv_heads * p.n_rt * ns;
+  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kp, m.vp, (int)grid, s);
+  if (e != cudaSuccess || ns == 1) return from_cuda(e);
+  CombineParams c;
+  std::memset(&c, 0, sizeof(c));
+  c.B = d->batch;
+  c.Hq = d->num_q_heads;
+  c.S = d->block_len;
+  c.D = d->head_dim;
+  c.nsplit = ns;
+  c.part_o = part_o;
+  c.part_lse = part_l;
+  c.out_o32 = O_pre;
+  c.out_lse = LSE_pre;
+  return from_cuda(launch_combine(c, s));
+}
+
+fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const void* Vb,
+                        const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
+                        int32_t* dev_status, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!Q || !Kb || !Vb || !O_pre || !LSE_pre || !O) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(Kb) || !aligned16(Vb) || !aligned16(O_pre) || !aligned16(O) ||
+      (reinterpret_cast<uintptr_t>(LSE_pre) & 3u) || (reinterpret_cast<uintptr_t>(LSE_out) & 3u))
+    return FB_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  AttnParams p = base_params(*d);
+  p.src = key_source(*d, false, true, nullptr);
+  p.epi = EPI_MERGE;
+  p.pre_o = O_pre;
+  p.pre_lse = LSE_pre;
+  p.out_o = O;
+  p.out_lse = LSE_out;
+  p.dev_status = dev_status;
+  if (d->dtype == FB_FP32)
+    return from_cuda(launch_attn_simt(p, static_cast<const float*>(Q), nullptr, nullptr,
+                                      static_cast<const float*>(Kb), static_cast<const float*>(Vb), s));
+  Maps m;
+  if (!q_map(&m.q, *d, Q) || !block_map(&m.kb, *d, Kb) || !block_map(&m.vb, *d, Vb)) return FB_ERR_LAUNCH;
+  const long long grid = (long long)d->batch * d->num_kv_heads * p.n_rt;
+  return from_cuda(launch_attn_tc(p, m.q, m.kb, m.vb, m.kb, m.vb, (int)grid, s));
+}
+
+fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc, const void* Vc,
+                                const void* Kb, const void* Vb, void* O, float* LSE_out, void* ws,
+                                size_t ws_bytes, int32_t* dev_status, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if ((st = check_cache(d)) != FB_OK) return st;
+  if (!Q || !Kc || !Vc || !Kb || !Vb || !O) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(Kb) || !aligned16(Vb) ||
+      !aligned16(O) || (reinterpret_cast<uintptr_t>(LSE_out) & 3u))
+    return FB_ERR_ALIGNMENT;
+  fb_desc dense = *d;
+  dense.topk = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  AttnParams p = base_params(dense);
+  p.src = key_source(dense, true, true, nullptr);
+  p.dev_status = dev_status;
+  if (d->dtype == FB_FP32) {
+    p.epi = EPI_NORM;
+    p.out_o = O;
+    p.out_lse = LSE_out;
+    return from_cuda(launch_attn_simt(p, static_cast<const float*>(Q), static_cast<const float*>(Kc),
+                                      static_cast<const float*>(Vc), static_cast<const float*>(Kb),
+                                      static_cast<const float*>(Vb), s));
+  }
+  const int ns = choose_splits(dense, prefix_tiles_estimate(dense) + (d->block_len + TC_BN - 1) / TC_BN);
+  const size_t need = split_bytes(dense, ns);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return FB_ERR_WORKSPACE;
+  Maps m;
+  if (!q_map(&m.q, dense, Q) || !cache_map(&m.kp, dense, Kc) || !cache_map(&m.vp, dense, Vc) ||
+      !block_map(&m.kb, dense, Kb) || !block_map(&m.vb, dense, Vb))
+    return FB_ERR_LAUNCH;
+  const long long units = (long long)d->batch * d->num_kv_heads * p.n_rt;
+  if (ns == 1) {
+    p.epi = EPI_NORM;
+    p.out_o = O;
+    p.out_lse = LSE_out;
+    return from_cuda(launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, (int)units, s));
+  }
+  p.epi = EPI_PARTIAL;
+  p.nsplit = ns;
+  float* part_o = static_cast<float*>(ws);
+  float* part_l = part_o + (size_t)ns * d->batch * d->block_len * d->num_q_heads * d->head_dim;
+  p.out_o32 = part_o;
+  p.out_lse = part_l;
+  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, (int)(units * ns), s);
+  if (e != cudaSuccess) return from_cuda(e);
+  CombineParams c;
+  std::memset(&c, 0, sizeof(c));
+  c.B = d->batch;
+  c.Hq = d->num_q_heads;
+  c.S = d->block_len;
+  c.D = d->head_dim;
+  c.nsplit = ns;
+  c.part_o = part_o;
+  c.part_lse = part_l;
+  c.out_o = O;
+  c.out_bf16 = 1;
+  c.out_lse = LSE_out;
+  return from_cuda(launch_combine(c, s));
+}
+
+fb_status fb_chunk_means(const fb_desc* d, const void* Kc, int32_t c0, int32_t c1, float* Kmean,
+                         int32_t* dev_status, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if ((st = check_cache(d)) != FB_OK) return st;
+  if (!Kc || !Kmean) return FB_ERR_INVALID_ARG;
+  if (d->chunk_size <= 0) return FB_ERR_INVALID_ARG;
+  const int64_t nch = (cache_rows(*d) + d->chunk_size - 1) / d->chunk_size;
+  if (c0 < 0 || c1 < c0 || c1 > nch) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Kc) || !aligned16(Kmean)) return FB_ERR_ALIGNMENT;
+  return from_cuda(launch_chunk_means(*d, Kc, c0, c1, Kmean, dev_status,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fb_status fb_select_chunks(const fb_desc* d, const void* Q, const float* Kmean, int32_t* chunk_idx,
+                           int32_t* dev_status, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if ((st = check_cache(d)) != FB_OK) return st;
+  if (!Q || !Kmean || !chunk_idx) return FB_ERR_INVALID_ARG;
+  if (d->chunk_size <= 0 || d->topk <= 0) return FB_ERR_INVALID_ARG;
+  const int64_t nch = (cache_rows(*d) + d->chunk_size - 1) / d->chunk_size;
+  if (nch > 16384) return FB_ERR_UNSUPPORTED;  // scores + flags stay within shared memory
+  if (!aligned16(Q) || !aligned16(Kmean) || (reinterpret_cast<uintptr_t>(chunk_idx) & 3u))
+    return FB_ERR_ALIGNMENT;
+  return from_cuda(launch_select_chunks(*d, Q, Kmean, chunk_idx, dev_status,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fb_status fb_kv_append(const fb_desc* d, const void* Kb, const void* Vb, void* Kc, void* Vc,
+                       int32_t* lens_inout, int32_t* dev_status, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!d->prefix_lens && !lens_inout) return FB_ERR_INVALID_ARG;
+  if (d->page_size > 0) {
+    if (!pow2(d->page_size) || !d->block_table || d->max_pages <= 0 || d->num_pages <= 0)
+      return FB_ERR_INVALID_ARG;
+  } else if (d->kv_capacity <= 0) {
+    return FB_ERR_INVALID_ARG;
+  }
+  if (!Kb || !Vb || !Kc || !Vc) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Kb) || !aligned16(Vb) || !aligned16(Kc) || !aligned16(Vc)) return FB_ERR_ALIGNMENT;
+  return from_cuda(launch_kv_append(*d, Kb, Vb, Kc, Vc, lens_inout, dev_status,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char* fb_status_string(fb_status s) {
+  switch (s) {
+    case FB_OK: return "FB_OK";
+    case FB_ERR_INVALID_ARG: return "FB_ERR_INVALID_ARG";
+    case FB_ERR_UNSUPPORTED: return "FB_ERR_UNSUPPORTED";
+    case FB_ERR_ALIGNMENT: return "FB_ERR_ALIGNMENT";
+    case FB_ERR_WORKSPACE: return "FB_ERR_WORKSPACE";
+    case FB_ERR_LAUNCH: return "FB_ERR_LAUNCH";
+    case FB_ERR_DEVICE_TIMEOUT: return "FB_ERR_DEVICE_TIMEOUT";
+    case FB_ERR_BOUNDS: return "FB_ERR_BOUNDS";
+  }
+  return "FB_ERR_UNKNOWN";
+}
+
+uint64_t fb_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int32_t fb_abi_version(void) { return FB_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,252 @@
+// fb_aux.cu -- sparse-prefix chunk means and top-k selection, and the block
+// append that grows the KV cache.
+//
+// Sparse prefix ("FlashBlock: Attention Caching for Efficient Long-Context
+// Block Diffusion", Technical Summary §2, Adaptive Reuse Strategies,
+// Compatibility with Sparse Attention): the prefix keys of each (b, kv head)
+// are restricted to the top-k chunks by the score
+//     qbar . kbar_c,
+// qbar the mean query of the block over its tokens and the G heads of the
+// group, kbar_c the mean key of chunk c over its valid rows.
+// Append (Technical Summary §1: KV caching with block-wise causal inference):
+// a finalized block's K/V joins the prefix.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "fb_internal.h"
+
+namespace fb {
+
+namespace {
+
+struct CacheGeom {
+  int B, Hkv, D, cap, paged, page_shift, max_pages, num_pages;
+  const int32_t* block_table;
+};
+
+CacheGeom geom_of(const fb_desc& d) {
+  CacheGeom g;
+  g.B = d.batch;
+  g.Hkv = d.num_kv_heads;
+  g.D = d.head_dim;
+  g.paged = d.page_size > 0;
+  g.page_shift = 0;
+  if (g.paged)
+    while ((1 << g.page_shift) < d.page_size) ++g.page_shift;
+  g.max_pages = d.max_pages;
+  g.num_pages = d.num_pages;
+  g.cap = g.paged ? d.max_pages * d.page_size : d.kv_capacity;
+  g.block_table = d.block_table;
+  return g;
+}
+
+// Element offset of cache row `pos` of sequence b, kv head kvh; -1 if the row
+// has no valid page.
+__device__ __forceinline__ long long cache_offset(const CacheGeom& g, int b, int pos, int kvh) {
+  if (g.paged) {
+    const int pi = pos >> g.page_shift;
+    if (pi >= g.max_pages) return -1;
+    const int pg = g.block_table[(size_t)b * g.max_pages + pi];
+    if (pg < 0 || pg >= g.num_pages) return -1;
+    const int prow = pos & ((1 << g.page_shift) - 1);
+    return (((long long)pg << g.page_shift) + prow) * g.Hkv * g.D + (long long)kvh * g.D;
+  }
+  return ((long long)b * g.cap + pos) * g.Hkv * g.D + (long long)kvh * g.D;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f(T v);
+template <>
+__device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// grid (chunks, Hkv, B), block D threads: thread d averages column d.
+template <typename T>
+__global__ void chunk_means_kernel(const CacheGeom g, const int32_t* lens, int chunk_size,
+                                   int c0, int nch_total, const T* __restrict__ K,
+                                   float* __restrict__ Kmean, int32_t* status) {
+  const int c = c0 + blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int d = threadIdx.x;
+  int L = lens[b];
+  if (L < 0 || L > g.cap) {
+    if (d == 0) report(status, FB_ERR_BOUNDS);
+    L = max(0, min(L, g.cap));
+  }
+  const int lo = c * chunk_size;
+  const int hi = min(lo + chunk_size, L);
+  float acc = 0.f;
+  for (int pos = lo; pos < hi; ++pos) {
+    const long long off = cache_offset(g, b, pos, kvh);
+    if (off < 0) {
+      if (d == 0) report(status, FB_ERR_BOUNDS);
+      continue;
+    }
+    acc += to_f<T>(K[off + d]);
+  }
+  const float mean = hi > lo ? acc / (float)(hi - lo) : 0.f;
+  Kmean[(((size_t)b * g.Hkv + kvh) * nch_total + c) * g.D + d] = mean;
+}
+
+// grid (Hkv, B), block 256.  Dynamic shared memory: D + nch floats + nch flags.
+template <typename T>
+__global__ void select_chunks_kernel(const CacheGeom g, const int32_t* lens, int chunk_size,
+                                     int nch_total, int S, int Hq, int topk,
+                                     const T* __restrict__ Q, const float* __restrict__ Kmean,
+                                     int32_t* __restrict__ idx, int32_t* status) {
+  extern __shared__ float sm[];
+  const int kvh = blockIdx.x;
+  const int b = blockIdx.y;
+  const int G = Hq / g.Hkv;
+  float* qbar = sm;
+  float* score = sm + g.D;
+  int* sel = reinterpret_cast<int*>(score + nch_total);
+  int L = lens[b];
+  if (L < 0 || L > g.cap) {
+    if (threadIdx.x == 0) report(status, FB_ERR_BOUNDS);
+    L = max(0, min(L, g.cap));
+  }
+  const int nch = (L + chunk_size - 1) / chunk_size;
+  for (int d = threadIdx.x; d < g.D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int t = 0; t < S; ++t)
+      for (int gg = 0; gg < G; ++gg)
+        acc += to_f<T>(Q[(((size_t)b * S + t) * Hq + kvh * G + gg) * g.D + d]);
+    qbar[d] = acc / (float)(S * G);
+  }
+  __syncthreads();
+  const float* km = Kmean + ((size_t)b * g.Hkv + kvh) * nch_total * g.D;
+  for (int c = threadIdx.x; c < nch; c += blockDim.x) {
+    float acc = 0.f;
+    for (int d = 0; d < g.D; ++d) acc = fmaf(qbar[d], km[(size_t)c * g.D + d], acc);
+    score[c] = acc;
+  }
+  __syncthreads();
+  // rank = chunks that beat c (higher score, or equal score and lower index)
+  for (int c = threadIdx.x; c < nch; c += blockDim.x) {
+    const float sc = score[c];
+    int better = 0;
+    for (int c2 = 0; c2 < nch; ++c2) {
+      const float s2 = score[c2];
+      better += (s2 > sc) || (s2 == sc && c2 < c);
+    }
+    sel[c] = better < topk;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t* out = idx + ((size_t)b * g.Hkv + kvh) * topk;
+    int n = 0;
+    for (int c = 0; c < nch && n < topk; ++c)
+      if (sel[c]) out[n++] = c;
+    for (; n < topk; ++n) out[n] = -1;
+  }
+}
+
+// One thread per 16-byte vector of the block's K and V.
+template <typename T>
+__global__ void kv_append_kernel(const CacheGeom g, const int32_t* lens, int S,
+                                 const T* __restrict__ Kb, const T* __restrict__ Vb,
+                                 T* __restrict__ Kc, T* __restrict__ Vc, int32_t* status) {
+  constexpr int VEC = 16 / sizeof(T);
+  const long long nvec_row = g.D / VEC;
+  const long long total = (long long)g.B * S * g.Hkv * nvec_row;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int v = (int)(i % nvec_row);
+    long long r = i / nvec_row;
+    const int kvh = (int)(r % g.Hkv);
+    r /= g.Hkv;
+    const int t = (int)(r % S);
+    const int b = (int)(r / S);
+    const int L = lens[b];
+    if (L < 0 || L + S > g.cap) {
+      if (t == 0 && kvh == 0 && v == 0) report(status, FB_ERR_BOUNDS);
+      continue;
+    }
+    const long long dst = cache_offset(g, b, L + t, kvh);
+    if (dst < 0) {
+      report(status, FB_ERR_BOUNDS);
+      continue;
+    }
+    const size_t src = (((size_t)b * S + t) * g.Hkv + kvh) * g.D + (size_t)v * VEC;
+    *reinterpret_cast<uint4*>(Kc + dst + v * VEC) = *reinterpret_cast<const uint4*>(Kb + src);
+    *reinterpret_cast<uint4*>(Vc + dst + v * VEC) = *reinterpret_cast<const uint4*>(Vb + src);
+  }
+}
+
+// Runs after the copy: advance each length by S when the block fitted.
+__global__ void lens_advance_kernel(int32_t* lens, int B, int S, int cap) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) {
+    const int L = lens[b];
+    if (L >= 0 && L + S <= cap) lens[b] = L + S;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_means(const fb_desc& d, const void* K, int c0, int c1, float* Kmean,
+                               int32_t* status, cudaStream_t stream) {
+  const CacheGeom g = geom_of(d);
+  const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
+  if (c1 <= c0) return cudaSuccess;
+  dim3 grid(c1 - c0, g.Hkv, g.B);
+  if (d.dtype == FB_BF16)
+    chunk_means_kernel<__nv_bfloat16><<<grid, g.D, 0, stream>>>(
+        g, d.prefix_lens, d.chunk_size, c0, nch_total, static_cast<const __nv_bfloat16*>(K), Kmean, status);
+  else
+    chunk_means_kernel<float><<<grid, g.D, 0, stream>>>(g, d.prefix_lens, d.chunk_size, c0, nch_total,
+                                                        static_cast<const float*>(K), Kmean, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* Kmean, int32_t* idx,
+                                 int32_t* status, cudaStream_t stream) {
+  const CacheGeom g = geom_of(d);
+  const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
+  const size_t smem = (size_t)(g.D + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int);
+  dim3 grid(g.Hkv, g.B);
+  if (d.dtype == FB_BF16) {
+    auto k = select_chunks_kernel<__nv_bfloat16>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, 256, smem, stream>>>(g, d.prefix_lens, d.chunk_size, nch_total, d.block_len, d.num_q_heads,
+                                   d.topk, static_cast<const __nv_bfloat16*>(Q), Kmean, idx, status);
+  } else {
+    auto k = select_chunks_kernel<float>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, 256, smem, stream>>>(g, d.prefix_lens, d.chunk_size, nch_total, d.block_len, d.num_q_heads,
+                                   d.topk, static_cast<const float*>(Q), Kmean, idx, status);
+  }
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kv_append(const fb_desc& d, const void* Kb, const void* Vb, void* Kc, void* Vc,
+                             int32_t* lens_inout, int32_t* status, cudaStream_t stream) {
+  const CacheGeom g = geom_of(d);
+  const int32_t* lens = lens_inout ? lens_inout : d.prefix_lens;
+  const int esz = d.dtype == FB_BF16 ? 2 : 4;
+  const long long total = (long long)g.B * d.block_len * g.Hkv * (g.D * esz / 16);
+  const int threads = 256;
+  const long long want = (total + threads - 1) / threads;
+  const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
+  if (d.dtype == FB_BF16)
+    kv_append_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(
+        g, lens, d.block_len, static_cast<const __nv_bfloat16*>(Kb), static_cast<const __nv_bfloat16*>(Vb),
+        static_cast<__nv_bfloat16*>(Kc), static_cast<__nv_bfloat16*>(Vc), status);
+  else
+    kv_append_kernel<float><<<grid, threads, 0, stream>>>(
+        g, lens, d.block_len, static_cast<const float*>(Kb), static_cast<const float*>(Vb),
+        static_cast<float*>(Kc), static_cast<float*>(Vc), status);
+  note_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || !lens_inout) return e;
+  lens_advance_kernel<<<(g.B + 127) / 128, 128, 0, stream>>>(lens_inout, g.B, d.block_len, g.cap);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace fb

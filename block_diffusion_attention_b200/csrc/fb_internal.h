@@ -1,0 +1,97 @@
+// fb_internal.h -- kernel parameter blocks and launchers shared between the
+// C-ABI layer (fb_api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "flashblock.h"
+
+namespace fb {
+
+// Output stage of the attention kernels.
+enum Epilogue : int {
+  EPI_PARTIAL = 0,  // normalised O (f32) + LSE: the cached pair, or one split's part
+  EPI_MERGE = 1,    // merge with (O_pre, LSE_pre), write O in the input dtype + LSE
+  EPI_NORM = 2,     // normalise, write O in the input dtype + LSE
+};
+
+// Where the keys of one (batch, kv head) work unit come from.  Virtual tile
+// index j runs over the prefix tiles first, then the block tiles.
+struct KeySource {
+  int has_prefix;     // 1: prefix rows j < prefix_lens[b] take part
+  int has_block;      // 1: all S block rows take part (after the prefix)
+  int paged;          // prefix cache is a page pool
+  int page_shift;     // log2(page_size) when paged
+  int max_pages;      // columns of block_table
+  int num_pages;      // pool pages
+  int cap;            // rows per sequence (contiguous capacity or pages*page_size)
+  const int32_t* block_table;
+  const int32_t* prefix_lens;
+  const int32_t* chunk_idx;  // sparse prefix list [B, Hkv, topk] or null
+  int topk;
+  int chunk_size;
+};
+
+struct AttnParams {
+  int B, Hq, Hkv, G, S, D;
+  int n_rt;      // row tiles per work unit (tensor-core path)
+  int nsplit;    // key-range splits per unit (EPI_PARTIAL only)
+  float scale;   // softmax scale (natural units)
+  float scale_log2;  // scale * log2(e)
+  int epi;
+  KeySource src;
+  // outputs
+  float* out_o32;         // EPI_PARTIAL: [nsplit][B][S][Hq][D]
+  float* out_lse;         // EPI_PARTIAL: [nsplit][B][Hq][S]; others: [B][Hq][S] or null
+  void* out_o;            // EPI_MERGE / EPI_NORM: [B][S][Hq][D] in the input dtype
+  const float* pre_o;     // EPI_MERGE inputs
+  const float* pre_lse;
+  int32_t* dev_status;
+};
+
+struct CombineParams {
+  int B, Hq, S, D, nsplit;
+  const float* part_o;    // [nsplit][B][S][Hq][D]
+  const float* part_lse;  // [nsplit][B][Hq][S]
+  float* out_o32;         // f32 output (prefix pass) or null
+  void* out_o;            // dtype output (full attention) or null
+  int out_bf16;           // out_o element type: 1 bf16, 0 f32
+  float* out_lse;         // [B][Hq][S] or null
+};
+
+// Tensor-core (bf16) path.
+constexpr int TC_BM = 128;      // query rows per tile (TMEM lanes)
+constexpr int TC_BN = 128;      // keys per tile
+constexpr int TC_D = 128;       // head dim
+constexpr int TC_STAGES = 2;    // K/V ring depth
+constexpr int TC_THREADS = 192; // 4 softmax warps + TMA warp + MMA warp
+size_t tc_smem_bytes();
+cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
+                           const CUtensorMap& tmVp, const CUtensorMap& tmKb,
+                           const CUtensorMap& tmVb, int grid, cudaStream_t stream);
+cudaError_t launch_combine(const CombineParams& c, cudaStream_t stream);
+
+// CUDA-core (fp32) path.
+cudaError_t launch_attn_simt(const AttnParams& p, const float* Q, const float* Kp,
+                             const float* Vp, const float* Kb, const float* Vb,
+                             cudaStream_t stream);
+
+// Sparse prefix helpers and the cache append.
+cudaError_t launch_chunk_means(const fb_desc& d, const void* K, int chunk_begin, int chunk_end,
+                               float* Kmean, int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* Kmean,
+                                 int32_t* idx, int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_kv_append(const fb_desc& d, const void* Kb, const void* Vb, void* Kc, void* Vc,
+                             int32_t* lens_inout, int32_t* dev_status, cudaStream_t stream);
+
+// Count of kernels launched (process-wide).
+void note_launch(int n = 1);
+
+// First error wins; later ones are dropped.
+__device__ __forceinline__ void report(int32_t* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+}  // namespace fb

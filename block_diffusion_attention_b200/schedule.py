@@ -1,0 +1,139 @@
+"""One attention layer's FlashBlock state on one GPU, driven through the C ABI.
+
+``CachedBlockAttention`` owns the device buffers of a layer -- the KV cache
+(contiguous or paged), the prefix lengths, the cached block-external pair
+(O_pre, LSE_pre), the split workspace, the sparse-prefix chunk means and
+chunk list -- and exposes the calls of one block of denoising steps:
+
+    refresh(Q)            prefix partial with this step's queries (refresh step)
+    step(Q, Kblk, Vblk)   in-block partial merged with the cached pair -> O
+    full(Q, Kblk, Vblk)   uncached attention over [prefix ; block] -> O
+    append(Kblk, Vblk)    finalized block joins the cache
+
+Each call is one or two C-ABI calls on the current CUDA stream; PyTorch only
+allocates the buffers.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import flashblock as fbl
+
+
+class CachedBlockAttention:
+    def __init__(self, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, block_len: int,
+                 capacity: int, dtype: str = "bf16", softmax_scale: float = 1.0, page_size: int = 0,
+                 block_table: Optional[torch.Tensor] = None, num_pages: int = 0,
+                 chunk_size: int = 0, topk: int = 0, num_splits: int = 0, device="cuda"):
+        self.device = torch.device(device)
+        self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.B, self.Hq, self.Hkv, self.D, self.S = batch, num_q_heads, num_kv_heads, head_dim, block_len
+        self.page_size = page_size
+        self.chunk_size, self.topk = chunk_size, topk
+        dev = self.device
+        if page_size > 0:
+            assert block_table is not None and num_pages > 0
+            self.block_table = block_table.to(dev, torch.int32).contiguous()
+            self.max_pages = self.block_table.shape[1]
+            self.num_pages = num_pages
+            cache_shape = (num_pages, page_size, num_kv_heads, head_dim)
+            self.capacity = self.max_pages * page_size
+        else:
+            self.block_table = None
+            self.max_pages = self.num_pages = 0
+            cache_shape = (batch, capacity, num_kv_heads, head_dim)
+            self.capacity = capacity
+        self.K = torch.zeros(cache_shape, dtype=self.tdtype, device=dev)
+        self.V = torch.zeros(cache_shape, dtype=self.tdtype, device=dev)
+        self.lens = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.lens_host = [0] * batch
+        self.desc = fbl.make_desc(
+            batch, num_q_heads, num_kv_heads, head_dim, block_len,
+            dtype=fbl.FB_BF16 if dtype == "bf16" else fbl.FB_FP32, softmax_scale=softmax_scale,
+            kv_capacity=self.capacity if page_size == 0 else 0, page_size=page_size,
+            max_pages=self.max_pages, num_pages=self.num_pages, block_table=self.block_table,
+            prefix_lens=self.lens, chunk_size=chunk_size, topk=topk, num_splits=num_splits)
+        self.O_pre = torch.empty((batch, block_len, num_q_heads, head_dim), dtype=torch.float32, device=dev)
+        self.LSE_pre = torch.empty((batch, num_q_heads, block_len), dtype=torch.float32, device=dev)
+        self.LSE = torch.empty((batch, num_q_heads, block_len), dtype=torch.float32, device=dev)
+        ws = fbl.fb_workspace_bytes(self.desc)
+        self.workspace = torch.empty(max(ws, 16) // 4 + 4, dtype=torch.float32, device=dev) if ws else None
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        if topk > 0:
+            nch = -(-self.capacity // chunk_size)
+            self.Kmean = torch.zeros((batch, num_kv_heads, nch, head_dim), dtype=torch.float32, device=dev)
+            self.chunk_idx = torch.full((batch, num_kv_heads, topk), -1, dtype=torch.int32, device=dev)
+        else:
+            self.Kmean = self.chunk_idx = None
+
+    # ------------------------------------------------------------------ state
+    def load_prefix(self, K: torch.Tensor, V: torch.Tensor, lens) -> None:
+        """Place a contiguous prefix [B, rows, Hkv, D] into the cache (rows >= lens are ignored)."""
+        lens = [int(x) for x in lens]
+        if self.page_size == 0:
+            n = min(K.shape[1], self.capacity)
+            self.K[:, :n].copy_(K[:, :n])
+            self.V[:, :n].copy_(V[:, :n])
+        else:
+            ps = self.page_size
+            bt = self.block_table.cpu()
+            for b in range(self.B):
+                for p in range(-(-lens[b] // ps)):
+                    lo, hi = p * ps, min((p + 1) * ps, K.shape[1])
+                    pg = int(bt[b, p])
+                    self.K[pg, :hi - lo].copy_(K[b, lo:hi])
+                    self.V[pg, :hi - lo].copy_(V[b, lo:hi])
+        self.lens.copy_(torch.tensor(lens, dtype=torch.int32))
+        self.lens_host = lens
+        if self.topk > 0:
+            self.update_chunk_means(0, -(-self.capacity // self.chunk_size))
+
+    def update_chunk_means(self, c0: int, c1: int) -> None:
+        fbl.fb_chunk_means(self.desc, self.K, c0, c1, self.Kmean, self.status)
+
+    # ------------------------------------------------------------------ steps
+    def refresh(self, Q: torch.Tensor) -> None:
+        """Refresh step: recompute the cached block-external pair with Q."""
+        idx = None
+        if self.topk > 0:
+            fbl.fb_select_chunks(self.desc, Q, self.Kmean, self.chunk_idx, self.status)
+            idx = self.chunk_idx
+        fbl.fb_prefix_partial(self.desc, Q, self.K, self.V, idx, self.O_pre, self.LSE_pre,
+                              self.workspace, self.status)
+
+    def step(self, Q, Kblk, Vblk, out: Optional[torch.Tensor] = None, lse: bool = False):
+        """Cached denoising step: O = merge(cached pair, in-block partial)."""
+        if out is None:
+            out = torch.empty_like(Q)
+        fbl.fb_block_step(self.desc, Q, Kblk, Vblk, self.O_pre, self.LSE_pre, out,
+                          self.LSE if lse else None, self.status)
+        return out
+
+    def full(self, Q, Kblk, Vblk, out: Optional[torch.Tensor] = None, lse: bool = False):
+        """Uncached step: attention over [prefix ; block] in one pass."""
+        if out is None:
+            out = torch.empty_like(Q)
+        fbl.fb_full_reference_gpu(self.desc, Q, self.K, self.V, Kblk, Vblk, out,
+                                  self.LSE if lse else None, self.workspace, self.status)
+        return out
+
+    def append(self, Kblk, Vblk) -> None:
+        """Block end: write the finalized block's K/V after the prefix and grow it."""
+        fbl.fb_kv_append(self.desc, Kblk, Vblk, self.K, self.V, self.lens, self.status)
+        old = self.lens_host
+        self.lens_host = [min(L + self.S, self.capacity) if L + self.S <= self.capacity else L for L in old]
+        if self.topk > 0:
+            c0 = min(old) // self.chunk_size
+            c1 = -(-max(self.lens_host) // self.chunk_size)
+            if c1 > c0:
+                self.update_chunk_means(c0, c1)
+
+    def check(self) -> None:
+        """Synchronise and raise if a kernel recorded a device-side error."""
+        torch.cuda.current_stream().synchronize()
+        st = int(self.status.item())
+        if st != 0:
+            self.status.zero_()
+            raise fbl.FlashBlockError("device", st)

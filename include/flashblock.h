@@ -1,0 +1,175 @@
+/*
+ * flashblock.h -- C ABI of libflashblock.so: cached block-diffusion attention
+ * (FlashBlock) on NVIDIA B200 (sm_100a).
+ *
+ * The method ("FlashBlock: Attention Caching for Efficient Long-Context Block
+ * Diffusion", Technical Summary §2 Methodology, Core Mechanism): at every
+ * denoising step of the active block, softmax attention over
+ * [finalized prefix ; block] splits into a block-external partial over the
+ * prefix (A_out, L_out = log Z_out) and a block-internal partial over the block
+ * (A_in, L_in).  The external pair is computed at a refresh step and reused on
+ * later steps; each step merges it with a fresh internal partial by the
+ * log-space merge equation
+ *     A = (e^{L_out-m} A_out + e^{L_in-m} A_in) / (e^{L_out-m} + e^{L_in-m}),
+ *     m = max(L_out, L_in).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every tensor pointer is a DEVICE pointer, contiguous, 16-byte aligned,
+ *    owned by the caller.  The library allocates no memory; scratch memory is
+ *    the caller's `workspace` (size from fb_workspace_bytes()).
+ *  - Layouts (row-major, innermost last):
+ *      Q, O            [B, S, Hq, D]
+ *      K/V cache       contiguous [B, kv_capacity, Hkv, D], or a page pool
+ *                      [num_pages, page_size, Hkv, D] addressed through
+ *                      block_table [B, max_pages] (int32, device)
+ *      K/V block       [B, S, Hkv, D]
+ *      O_pre           [B, S, Hq, D] float32
+ *      LSE, LSE_pre    [B, Hq, S] float32, natural log of the unnormalised sum
+ *      Kmean           [B, Hkv, ceil(capacity / chunk_size), D] float32
+ *      chunk_idx       [B, Hkv, topk] int32, ascending, padded with -1
+ *    Query head h reads KV head h / (Hq / Hkv).
+ *  - dtype FB_BF16: Q, K, V, O are bfloat16 (tensor-core path, D = 128).
+ *    dtype FB_FP32: Q, K, V, O are float32 (CUDA-core path, D in {32,64,96,128}).
+ *    Accumulation is float32 in both.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and deterministic: fixed split order, no floating-point atomics.
+ *  - Errors: argument checks run on the host before anything is launched and
+ *    return a non-zero fb_status synchronously.  Faults found on the device
+ *    (an index out of range, a pipeline wait past its time limit) are written
+ *    to *dev_status (device int32, nullable; the first error sticks, the
+ *    caller zeroes it and reads it after synchronising).  The library never
+ *    traps.
+ *  - The library keeps no per-call state and is safe to call from several host
+ *    threads; concurrent calls must not share output or workspace buffers.
+ */
+#ifndef FLASHBLOCK_H
+#define FLASHBLOCK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FB_ABI_VERSION 1
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* fb_stream_t;
+
+typedef enum fb_status {
+  FB_OK = 0,
+  FB_ERR_INVALID_ARG = 1,    /* null pointer, non-positive or inconsistent size */
+  FB_ERR_UNSUPPORTED = 2,    /* valid but not implemented (head_dim, group size, dtype) */
+  FB_ERR_ALIGNMENT = 3,      /* a tensor pointer is not 16-byte aligned */
+  FB_ERR_WORKSPACE = 4,      /* workspace missing or smaller than fb_workspace_bytes() */
+  FB_ERR_LAUNCH = 5,         /* no CUDA device, or the runtime refused a launch */
+  FB_ERR_DEVICE_TIMEOUT = 6, /* device-side: a pipeline wait exceeded its time limit */
+  FB_ERR_BOUNDS = 7          /* device-side: page, chunk or cache row out of range */
+} fb_status;
+
+typedef enum fb_dtype { FB_BF16 = 0, FB_FP32 = 1 } fb_dtype;
+
+typedef struct fb_desc {
+  int32_t batch;          /* B >= 1 */
+  int32_t num_q_heads;    /* Hq >= 1 */
+  int32_t num_kv_heads;   /* Hkv >= 1, Hq % Hkv == 0; bf16 needs G = Hq/Hkv a power of two <= 128 */
+  int32_t head_dim;       /* D */
+  int32_t block_len;      /* S >= 1: tokens of the active block */
+  int32_t dtype;          /* fb_dtype */
+  float softmax_scale;    /* > 0: logits are softmax_scale * (q . k) */
+  int32_t kv_capacity;    /* contiguous cache: rows per sequence; paged: unused */
+  int32_t page_size;      /* 0 = contiguous cache; else a power of two >= 64 */
+  int32_t max_pages;      /* paged: columns of block_table */
+  int32_t num_pages;      /* paged: pages in the pool */
+  const int32_t* block_table; /* paged: device [B, max_pages]; else NULL */
+  const int32_t* prefix_lens; /* device [B]: valid prefix rows L_b (0 allowed) */
+  int32_t chunk_size;     /* sparse prefix: tokens per chunk, a multiple of 128; 0 if unused */
+  int32_t topk;           /* sparse prefix: chunks kept per (b, kv head); 0 = dense prefix */
+  int32_t num_splits;     /* prefix pass: key-range splits per work unit; 0 = library's choice */
+} fb_desc;
+
+/* Rows each sequence can hold: kv_capacity (contiguous) or max_pages*page_size (paged). */
+int64_t fb_cache_rows(const fb_desc* d);
+
+/* Bytes of device workspace that fb_prefix_partial and fb_full_reference_gpu
+ * need for this descriptor on the current device (split-key partials:
+ * splits x B x S x Hq x (D + 1) float32).  0 means no workspace is needed. */
+size_t fb_workspace_bytes(const fb_desc* d);
+
+/* Block-external partial over the finalized prefix (the cached pair).
+ * Core Mechanism: A_out and L_out = log Z_out over J_out, the tokens outside
+ * the current block, here the prefix rows j < prefix_lens[b].  With
+ * d->topk > 0 the key set of each (b, kv head) is the union of the chunks
+ * listed in chunk_idx (the sparse prefix; see fb_select_chunks).
+ * Q [B,S,Hq,D] (dtype); Kcache/Vcache (dtype; contiguous or paged);
+ * chunk_idx [B,Hkv,topk] int32 or NULL when topk == 0.
+ * Writes O_pre [B,S,Hq,D] float32 (normalised) and LSE_pre [B,Hq,S] float32;
+ * an empty key set gives O_pre = 0, LSE_pre = -inf. */
+fb_status fb_prefix_partial(const fb_desc* d, const void* Q, const void* Kcache,
+                            const void* Vcache, const int32_t* chunk_idx,
+                            float* O_pre, float* LSE_pre, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status,
+                            fb_stream_t stream);
+
+/* One cached denoising step.  Core Mechanism: the block-internal partial of
+ * Q over the block's own keys (bidirectional, no mask) merged in the same
+ * kernel with the cached (O_pre, LSE_pre) by the merge equation.
+ * Q [B,S,Hq,D], Kblk/Vblk [B,S,Hkv,D] (dtype).  Writes O [B,S,Hq,D] (dtype)
+ * and, when LSE_out is not NULL, the merged LSE [B,Hq,S] float32. */
+fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kblk,
+                        const void* Vblk, const float* O_pre, const float* LSE_pre,
+                        void* O, float* LSE_out, int32_t* dev_status,
+                        fb_stream_t stream);
+
+/* Uncached block diffusion (Technical Summary §1 Problem Statement): attention
+ * of Q over [prefix rows j < L_b ; all S block rows] in one pass, no cached
+ * partial.  The dense prefix is always used (topk is ignored).
+ * Writes O [B,S,Hq,D] (dtype) and, when LSE_out is not NULL, LSE [B,Hq,S]. */
+fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kcache,
+                                const void* Vcache, const void* Kblk, const void* Vblk,
+                                void* O, float* LSE_out, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status,
+                                fb_stream_t stream);
+
+/* Sparse prefix, step 1 (Adaptive Reuse Strategies, "Compatibility with
+ * Sparse Attention": the selected keys are attended, the rest form J_out).
+ * Mean key of chunks [chunk_begin, chunk_end) over their valid rows
+ * j < prefix_lens[b]; chunks without a valid row get 0.  Call once for the
+ * whole prefix and again for the chunks an append touched.
+ * Kmean [B, Hkv, ceil(rows / chunk_size), D] float32. */
+fb_status fb_chunk_means(const fb_desc* d, const void* Kcache, int32_t chunk_begin,
+                         int32_t chunk_end, float* Kmean, int32_t* dev_status,
+                         fb_stream_t stream);
+
+/* Sparse prefix, step 2: per (b, kv head) score every valid chunk c by
+ * qbar . Kmean[c], qbar the mean of Q over the S block tokens and the G query
+ * heads of the group, and keep the top d->topk (ties to the lower index).
+ * Writes chunk_idx [B,Hkv,topk] int32 in ascending chunk order, -1 padded. */
+fb_status fb_select_chunks(const fb_desc* d, const void* Q, const float* Kmean,
+                           int32_t* chunk_idx, int32_t* dev_status, fb_stream_t stream);
+
+/* Block end ("KV caching with block-wise causal inference", Technical Summary
+ * §1): copy the finalized block's K/V [B,S,Hkv,D] into cache rows
+ * [L_b, L_b + S) (contiguous or paged).  When lens_inout is not NULL
+ * (device [B]), it is read for L_b and then advanced by S.  A block that does
+ * not fit records FB_ERR_BOUNDS in dev_status and is not written. */
+fb_status fb_kv_append(const fb_desc* d, const void* Kblk, const void* Vblk,
+                       void* Kcache, void* Vcache, int32_t* lens_inout,
+                       int32_t* dev_status, fb_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* fb_status_string(fb_status s);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t fb_launch_count(void);
+
+/* FB_ABI_VERSION of the loaded library. */
+int32_t fb_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHBLOCK_H */

@@ -1,0 +1,81 @@
+"""The C-ABI library loads, exports every function its header declares, and
+rejects bad arguments on the host before launching anything (CPU only: no
+compute call reaches a device here)."""
+import ctypes
+
+import pytest
+
+from block_diffusion_attention_b200 import flashblock as fbl
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return fbl.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = fbl.header_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in flashblock.h but not exported"
+
+
+def test_version_and_status_strings(lib):
+    assert fbl.fb_abi_version() == 1
+    for code, name in fbl.STATUS.items():
+        assert fbl.fb_status_string(code) == name
+    assert fbl.fb_status_string(99) == "FB_ERR_UNKNOWN"
+    assert fbl.fb_launch_count() >= 0
+
+
+def _desc(**kw):
+    base = dict(batch=1, num_q_heads=32, num_kv_heads=8, head_dim=128, block_len=32,
+                dtype=fbl.FB_BF16, softmax_scale=1.0, kv_capacity=8192)
+    base.update(kw)
+    d = fbl.make_desc(**base)
+    d.prefix_lens = 0x10000  # a host-side stand-in; validation never dereferences it
+    return d
+
+
+FAKE = 0x7f0000000000  # 16-byte aligned, never dereferenced
+
+
+def _prefix(lib, d, q=FAKE, k=FAKE, v=FAKE, idx=None, o=FAKE, l=FAKE, ws=None, wsb=0):
+    return lib.fb_prefix_partial(ctypes.byref(d), q, k, v, idx, o, l, ws, wsb, None, None) \
+        if d is not None else lib.fb_prefix_partial(None, q, k, v, idx, o, l, ws, wsb, None, None)
+
+
+def test_host_validation_codes(lib):
+    assert _prefix(lib, None) == 1
+    assert _prefix(lib, _desc(batch=0)) == 1
+    assert _prefix(lib, _desc(num_q_heads=30)) == 1           # not a multiple of Hkv
+    assert _prefix(lib, _desc(softmax_scale=0.0)) == 1
+    assert _prefix(lib, _desc(softmax_scale=float("nan"))) == 1
+    assert _prefix(lib, _desc(head_dim=64)) == 2              # bf16 path is D = 128
+    assert _prefix(lib, _desc(num_q_heads=24, num_kv_heads=8)) == 2  # G = 3
+    assert _prefix(lib, _desc(dtype=7)) == 2
+    assert _prefix(lib, _desc(dtype=fbl.FB_FP32, head_dim=48)) == 2
+    assert _prefix(lib, _desc(), q=None) == 1
+    assert _prefix(lib, _desc(), q=FAKE + 8) == 3              # TMA needs 16-byte alignment
+    assert _prefix(lib, _desc(page_size=100, max_pages=4, num_pages=4, block_table=None)) == 2
+    d = _desc(page_size=128, max_pages=4, num_pages=4)
+    assert _prefix(lib, d) == 1                                # paged without a block table
+    assert _prefix(lib, _desc(topk=4, chunk_size=256)) == 1    # sparse without a chunk list
+    assert _prefix(lib, _desc(topk=4, chunk_size=200), idx=FAKE) == 2
+    # long prefix -> split-key workspace required
+    d = _desc(kv_capacity=131072)
+    assert fbl.fb_workspace_bytes(d) > 0
+    assert _prefix(lib, d) == 4
+    blk = lib.fb_block_step(ctypes.byref(_desc()), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, None)
+    assert blk == 1
+    assert lib.fb_chunk_means(ctypes.byref(_desc(chunk_size=256)), FAKE, 0, 999, FAKE, None, None) == 1
+    assert lib.fb_select_chunks(ctypes.byref(_desc(chunk_size=256, topk=0)), FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.fb_kv_append(ctypes.byref(_desc(kv_capacity=0)), FAKE, FAKE, FAKE, FAKE, None, None, None) == 1
+
+
+def test_workspace_bytes_formula(lib):
+    d = _desc(kv_capacity=131072, num_splits=5)
+    # splits x rows x (D + 1) floats
+    assert fbl.fb_workspace_bytes(d) == 5 * 32 * 32 * 129 * 4
+    assert fbl.fb_workspace_bytes(_desc(dtype=fbl.FB_FP32, head_dim=64)) == 0
+    assert fbl.fb_cache_rows(_desc(page_size=256, max_pages=3, num_pages=9)) == 768

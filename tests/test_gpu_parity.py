@@ -1,0 +1,118 @@
+"""GPU parity: the CUDA path against the float64 oracle, element by element, on
+scaled-down versions of the five workloads that still span several key and
+query tiles with ragged tails, plus the edge cases of the method.  Every call
+goes through the C ABI."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import gpu_cases
+from block_diffusion_attention_b200 import synth
+from block_diffusion_attention_b200 import flashblock as fbl
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+
+
+def test_tiny_fp32_full_config():
+    # the tiny workload is small enough to run at its full size
+    gpu_cases.run_workload(W["tiny_fp32"])
+
+
+def test_tiny_fp32_ragged_multiblock():
+    w = W["tiny_fp32"].scaled(prefix_len=301, block_len=13, blocks=2, steps=3, num_q_heads=4, num_kv_heads=2,
+                              head_dim=128)
+    gpu_cases.run_workload(w)
+
+
+def test_lm_gqa_scaled_two_blocks():
+    w = W["lm_gqa"].scaled(prefix_len=1000, blocks=2, steps=3)
+    gpu_cases.run_workload(w)
+
+
+@pytest.mark.parametrize("num_splits", [1, 3, 7])
+def test_lm_gqa_split_counts(num_splits):
+    w = W["lm_gqa"].scaled(prefix_len=1500, blocks=1, steps=2)
+    gpu_cases.run_workload(w, num_splits=num_splits)
+
+
+@pytest.mark.parametrize("page_size", [64, 128, 256])
+def test_paged_cache(page_size):
+    w = W["lm_gqa"].scaled(prefix_len=900, blocks=2, steps=2, num_q_heads=16, num_kv_heads=4)
+    gpu_cases.run_workload(w, page_size=page_size)
+
+
+def test_video_scaled_mha_ragged_rows():
+    # G = 1: each 128-row query tile is 128 tokens of one head; 300 = 2*128 + 44
+    w = W["video"].scaled(num_q_heads=2, num_kv_heads=2, block_len=300, prefix_len=700, steps=2)
+    gpu_cases.run_workload(w)
+
+
+def test_batched_sparse_scaled():
+    w = W["batched_sparse"].scaled(batch=3, num_q_heads=8, num_kv_heads=2, prefix_len=1500,
+                                   prefix_min=600, topk=3, steps=5)
+    gpu_cases.run_workload(w)
+
+
+def test_sparse_topk_covers_all_chunks_equals_dense():
+    w = W["batched_sparse"].scaled(batch=2, num_q_heads=8, num_kv_heads=2, prefix_len=700,
+                                   prefix_min=300, topk=8, steps=1)
+    gpu_cases.run_workload(w)
+
+
+@pytest.mark.parametrize("L,S,G", [(0, 32, 4), (1, 32, 4), (127, 1, 4), (129, 7, 4), (255, 33, 2),
+                                   (257, 16, 8), (130, 64, 1)])
+def test_edge_lengths(L, S, G):
+    w = W["lm_gqa"].scaled(prefix_len=L, block_len=S, num_q_heads=2 * G, num_kv_heads=2, blocks=2, steps=2)
+    gpu_cases.run_workload(w)
+
+
+def test_edge_lengths_fp32_empty_prefix():
+    w = W["tiny_fp32"].scaled(prefix_len=0, block_len=5, steps=2, blocks=2)
+    gpu_cases.run_workload(w)
+
+
+def test_other_softmax_scale():
+    # Q ~ N(0,1)/sqrt(D) with the 1/sqrt(D) scale as well: flatter logits
+    w = W["lm_gqa"].scaled(prefix_len=800, blocks=1, steps=2, softmax_scale=1.0 / math.sqrt(128))
+    gpu_cases.run_workload(w)
+
+
+def test_large_logits_rescale_path():
+    # Q ~ N(0, 4): logits with std ~ 22, so the running row max keeps growing
+    # and the lazy rescale of the accumulator fires.
+    w = W["lm_gqa"].scaled(prefix_len=1200, blocks=1, steps=2, q_std=2.0, softmax_scale=1.0)
+    gpu_cases.run_workload(w)
+
+
+def test_refresh_determinism_bitwise():
+    w = W["lm_gqa"].scaled(prefix_len=2000, blocks=1, steps=1)
+    K, V, lens = synth.prefix_kv(w)
+    Kt, _ = gpu_cases.tensors(w, K)
+    Vt, _ = gpu_cases.tensors(w, V)
+    layer = gpu_cases.make_layer(w)
+    layer.load_prefix(Kt, Vt, lens)
+    Q, _, _ = synth.step_inputs(w, 0, 0)
+    Qt, _ = gpu_cases.tensors(w, Q)
+    layer.refresh(Qt)
+    a = (layer.O_pre.clone(), layer.LSE_pre.clone())
+    layer.refresh(Qt)
+    layer.check()
+    assert torch.equal(a[0], layer.O_pre) and torch.equal(a[1], layer.LSE_pre)
+
+
+def test_device_bounds_status_reported():
+    # a prefix length past the capacity is reported on the device, not faulted
+    w = W["lm_gqa"].scaled(prefix_len=256, blocks=1, steps=1)
+    layer = gpu_cases.make_layer(w)
+    K, V, lens = synth.prefix_kv(w)
+    layer.load_prefix(gpu_cases.tensors(w, K)[0], gpu_cases.tensors(w, V)[0], lens)
+    layer.lens.fill_(w.capacity + 5)
+    Q, _, _ = synth.step_inputs(w, 0, 0)
+    layer.refresh(gpu_cases.tensors(w, Q)[0])
+    with pytest.raises(fbl.FlashBlockError) as e:
+        layer.check()
+    assert e.value.status == 7
