@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark: FlashBlock cached vs uncached block-diffusion attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One timed *step* is one block of denoising steps of one attention layer, the
+cached FlashBlock way: the prefix partial at the refresh step(s), the
+in-block partial fused with the merge on every denoising step, and the block's
+append to the KV cache.  The uncached baseline (full attention over
+[prefix ; block] on every denoising step, plus the same append) is timed the
+same way right after.  Inputs are resident in HBM before the timed region;
+the KV cache (537 MB at 128K context) is larger than the 126 MB L2, so no
+flush is needed between steps.  The append writes the block's rows after the
+prefix without advancing the prefix length, so every timed block sees exactly
+the configured prefix.
+
+``value`` is cached attention tokens/s over all ranks (B * S tokens finalized
+per block per rank).  Under torchrun each rank runs an independent replica
+(weak scaling; the path has no collective).  Rank 0 prints one JSON line.
+
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the
+same workload (rank 0 only) and prints the same kind of line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention µs/denoise-step and tokens/s, cached vs uncached; prefix-pass HBM GB/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long_ctx")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--phases", default="cached,uncached,e2e",
+                    help="comma list of timed phases (profiling runs may keep only 'cached')")
+    return ap.parse_args()
+
+
+def workload_config(w, extra=None):
+    cfg = {
+        "workload": (f"{w.name}: B{w.batch} Hq{w.num_q_heads}/Hkv{w.num_kv_heads} D{w.head_dim} "
+                     f"block {w.block_len} prefix {w.prefix_len}"
+                     + (f" (varlen from {w.prefix_min})" if w.prefix_min else "")
+                     + f", {w.steps} denoising steps per block, refresh at {list(w.refresh)}"
+                     + (f", top-{w.topk} of {w.chunk_size}-token chunks" if w.topk else "")),
+        "global_batch": w.batch,
+        "seq_len": w.prefix_len,
+        "block_len": w.block_len,
+        "denoise_steps": w.steps,
+        "parallelism": "replicas",
+        "l2": "KV cache larger than the 126 MB L2 at this workload; no flush" if
+              2 * w.batch * w.prefix_len * w.num_kv_heads * w.head_dim * 2 > 126e6 else
+              "KV cache fits in L2: prefix-pass GB/s is L2-warm",
+    }
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def prefix_bytes(w, lens):
+    """Algorithmic bytes of one prefix pass: K+V of the valid (or selected)
+    prefix rows, Q, and the written O_pre (f32) and LSE_pre (f32)."""
+    if w.topk:
+        eff = sum(min(int(L), w.topk * w.chunk_size) for L in lens)
+    else:
+        eff = sum(int(L) for L in lens)
+    kv = 2 * eff * w.num_kv_heads * w.head_dim * 2
+    rows = w.batch * w.block_len * w.num_q_heads
+    return kv + rows * w.head_dim * 2 + rows * w.head_dim * 4 + rows * 4
+
+
+def prefix_flops(w, lens):
+    eff = sum(min(int(L), w.topk * w.chunk_size) if w.topk else int(L) for L in lens)
+    return 4.0 * w.num_q_heads * w.block_len * eff * w.head_dim
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            j = json.load(f)
+        return j.get("hbm_gbs", 6650.0), j.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+# --------------------------------------------------------------------------
+# Oracle timing (CPU baseline and the reference arm)
+# --------------------------------------------------------------------------
+
+def oracle_block_sample(w, K, V, lens, heads=1):
+    """Time the oracle's cached block on the first `heads` kv heads of the
+    workload (one block: refresh + every denoising step's in-block partial and
+    merge); returns seconds scaled to all kv heads."""
+    import numpy as np
+    from block_diffusion_attention_b200 import synth
+    from oracle import flashblock_oracle as ora
+    G = w.group
+    hs = slice(0, heads)
+    qs = slice(0, heads * G)
+    Kc = synth.as_dtype(w, K[:, :, hs])[1]
+    Vc = synth.as_dtype(w, V[:, :, hs])[1]
+    base = synth.block_base(w, 0)
+    steps = []
+    for s in range(w.steps):
+        Q, Kb, Vb = synth.step_inputs(w, 0, s, base)
+        steps.append((synth.as_dtype(w, Q[:, :, qs])[1], synth.as_dtype(w, Kb[:, :, hs])[1],
+                      synth.as_dtype(w, Vb[:, :, hs])[1]))
+    lens64 = np.asarray(lens, dtype=np.int64)
+    chunk_fn = None
+    if w.topk:
+        Km, valid = ora.chunk_means(Kc, lens64, w.chunk_size)
+        chunk_fn = lambda Q: ora.select_chunks(Q, Km, valid, w.topk)  # noqa: E731
+    t0 = time.perf_counter()
+    ora.cached_block([x[0] for x in steps], [x[1] for x in steps], [x[2] for x in steps], Kc, Vc, lens64,
+                     w.softmax_scale, w.refresh, chunk_fn, w.chunk_size)
+    dt = time.perf_counter() - t0
+    return dt * (w.num_kv_heads / heads)
+
+
+def run_reference(args):
+    from block_diffusion_attention_b200 import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = synth.WORKLOADS[args.workload]
+    K, V, lens = synth.prefix_kv(w)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = oracle_block_sample(w, K, V, lens, heads=1)
+        if i >= args.warmup:
+            times.append(t)
+    per_block = sum(times) / len(times)
+    tok_s = w.batch * w.block_len / per_block
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_block * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cached_us_per_denoise_step": per_block / w.steps * 1e6,
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"each step: the oracle's cached block on 1 of {w.num_kv_heads} kv heads, "
+                                   f"time scaled x{w.num_kv_heads}"},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from block_diffusion_attention_b200 import flashblock as fbl
+    from block_diffusion_attention_b200 import synth
+    from block_diffusion_attention_b200.schedule import CachedBlockAttention
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    fbl.load()
+    phases = set(args.phases.split(","))
+
+    w0 = synth.WORKLOADS[args.workload]
+    # the append rows sit after the prefix; the prefix length stays fixed
+    w = w0.scaled(blocks=1)
+    K, V, lens = synth.prefix_kv(w)
+    Kt = synth.as_dtype(w, K)[0].cuda()
+    Vt = synth.as_dtype(w, V)[0].cuda()
+    del K, V
+    base = synth.block_base(w, 0)
+    step_in = []
+    for s in range(w.steps):
+        Q, Kb, Vb = synth.step_inputs(w, 0, s, base)
+        step_in.append(tuple(synth.as_dtype(w, x)[0] for x in (Q, Kb, Vb)))
+    dev_in = [tuple(x.cuda() for x in t) for t in step_in]
+    outs = [torch.empty_like(dev_in[0][0]) for _ in range(w.steps)]
+    stream = torch.cuda.current_stream()
+
+    def new_layer():
+        layer = CachedBlockAttention(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_len, w.capacity,
+                                     dtype=w.dtype, softmax_scale=w.softmax_scale,
+                                     chunk_size=w.chunk_size if w.topk else 0, topk=w.topk)
+        layer.load_prefix(Kt, Vt, lens)
+        return layer
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    res = {}
+
+    def timed(block_fn, layer):
+        """W untimed blocks, then K blocks between CUDA events; max over ranks."""
+        for _ in range(args.warmup):
+            block_fn(None)
+        layer.check()
+        barrier()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        n0 = fbl.fb_launch_count()
+        t0.record(stream)
+        for k in range(args.steps):
+            block_fn(k)
+        t1.record(stream)
+        n1 = fbl.fb_launch_count()
+        torch.cuda.synchronize()
+        layer.check()
+        res.setdefault("launch_counts", []).append(n1 - n0)
+        return max_over_ranks(t0.elapsed_time(t1))
+
+    # ---- cached (FlashBlock) path: the headline
+    cached = new_layer()
+    nref = len(w.refresh)
+    ev_pre = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps * nref)]
+    ev_blk = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps * w.steps)]
+
+    def cached_block(k):
+        pi = 0
+        for s in range(w.steps):
+            Q, Kb, Vb = dev_in[s]
+            if s in w.refresh:
+                if k is not None:
+                    ev_pre[k * nref + pi][0].record(stream)
+                cached.refresh(Q)
+                if k is not None:
+                    ev_pre[k * nref + pi][1].record(stream)
+                pi += 1
+            if k is not None:
+                ev_blk[k * w.steps + s][0].record(stream)
+            cached.step(Q, Kb, Vb, out=outs[s])
+            if k is not None:
+                ev_blk[k * w.steps + s][1].record(stream)
+        cached.append(dev_in[-1][1], dev_in[-1][2], advance=False)
+
+    res["lens0"] = [int(x) for x in cached.lens.cpu()]
+    # clocks are sampled from the first warm-up block to the end of the last timed phase
+    sampler = ClockSampler(local)
+    sampler.start()
+    res["ms_cached"] = timed(cached_block, cached)
+    res["launches"] = res["launch_counts"][0]
+    res["lens1"] = [int(x) for x in cached.lens.cpu()]
+    res["pre_ms"] = [a.elapsed_time(b) for a, b in ev_pre]
+    res["blk_ms"] = [a.elapsed_time(b) for a, b in ev_blk]
+    del cached
+
+    # ---- uncached baseline: full attention at every denoising step
+    if "uncached" in phases:
+        unc = new_layer()
+
+        def uncached_block(k):
+            for s in range(w.steps):
+                Q, Kb, Vb = dev_in[s]
+                unc.full(Q, Kb, Vb, out=outs[s])
+            unc.append(dev_in[-1][1], dev_in[-1][2], advance=False)
+
+        res["ms_unc"] = timed(uncached_block, unc)
+        del unc
+
+    # ---- end to end through the public API: pinned host inputs in, O out
+    if "e2e" in phases:
+        e2e_layer = new_layer()
+        host_in = [tuple(x.pin_memory() for x in t) for t in step_in]
+        host_out = [torch.empty(dev_in[0][0].shape, dtype=dev_in[0][0].dtype).pin_memory()
+                    for _ in range(w.steps)]
+        stage = [tuple(torch.empty_like(x) for x in t) for t in dev_in]
+
+        def e2e_block(k):
+            for s in range(w.steps):
+                for dst, src in zip(stage[s], host_in[s]):
+                    dst.copy_(src, non_blocking=True)
+                Q, Kb, Vb = stage[s]
+                if s in w.refresh:
+                    e2e_layer.refresh(Q)
+                o = e2e_layer.step(Q, Kb, Vb, out=outs[s])
+                host_out[s].copy_(o, non_blocking=True)
+            e2e_layer.append(stage[-1][1], stage[-1][2], advance=False)
+
+        res["ms_e2e"] = timed(e2e_block, e2e_layer)
+        res["h2d"] = sum(x.numel() * x.element_size() for t in host_in for x in t)
+        res["d2h"] = sum(x.numel() * x.element_size() for x in host_out)
+        del e2e_layer
+
+    res["clocks"] = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        report(args, w0, w, world, res)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def report(args, w0, w, world, res):
+    from block_diffusion_attention_b200 import synth
+    tokens = world * w.batch * w.block_len * args.steps
+
+    def tps(ms):
+        return tokens / (ms / 1e3) if ms and ms == ms else None
+
+    pre_avg = sum(res["pre_ms"]) / len(res["pre_ms"])
+    blk_avg = sum(res["blk_ms"]) / len(res["blk_ms"])
+    mid = [(a + b) / 2 for a, b in zip(res["lens0"], res["lens1"])]
+    abytes = prefix_bytes(w, mid)
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    achieved = abytes / (pre_avg / 1e3) / 1e9
+    tflops = prefix_flops(w, mid) / (pre_avg / 1e3) / 1e12
+    ms_c = res["ms_cached"]
+    ms_u = res.get("ms_unc")
+    line = {
+        "metric": METRIC, "value": tps(ms_c), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_c / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) K/V, scaled Q, per-step drift)",
+        "config": workload_config(w0, {"prefix_rows_during_timing": [min(res["lens0"]), max(res["lens1"])]}),
+        "cached_us_per_denoise_step": ms_c * 1e3 / (args.steps * w.steps),
+        "uncached_us_per_denoise_step": ms_u * 1e3 / (args.steps * w.steps) if ms_u else None,
+        "uncached_tokens_per_s": tps(ms_u),
+        "cached_over_uncached_speedup": (ms_u / ms_c) if ms_u else None,
+        "prefix_pass_us": pre_avg * 1e3,
+        "block_step_us": blk_avg * 1e3,
+        "prefix_gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None,
+                     "kernel": "prefix pass: attn_tc_kernel<EPI_PARTIAL> + combine_kernel",
+                     "peak_source": f"{peak_kind} hbm_gbs", "algorithmic_bytes_per_launch": abytes,
+                     "tensor_tflops": tflops, "tensor_frac": tflops / tc_peak},
+        "clocks": res["clocks"],
+        "e2e": ({"value": tps(res["ms_e2e"]), "unit": "tokens/s", "h2d_bytes_per_step": res["h2d"],
+                 "d2h_bytes_per_step": res["d2h"]} if "ms_e2e" in res else None),
+        "gpu_launches": res["launches"],
+        "gpu_launches_per_step": res["launches"] / args.steps,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        K, V, lens_np = synth.prefix_kv(w0)
+        t = oracle_block_sample(w0, K, V, lens_np, heads=1)
+        line["cpu_baseline"] = {
+            "value": w0.batch * w0.block_len / t, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"the oracle's cached block (refresh + {w0.steps} steps) on 1 of {w0.num_kv_heads} kv heads, "
+                      f"time scaled x{w0.num_kv_heads}"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

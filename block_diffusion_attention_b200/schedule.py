@@ -119,9 +119,14 @@ class CachedBlockAttention:
                                   self.LSE if lse else None, self.workspace, self.status)
         return out
 
-    def append(self, Kblk, Vblk) -> None:
-        """Block end: write the finalized block's K/V after the prefix and grow it."""
-        fbl.fb_kv_append(self.desc, Kblk, Vblk, self.K, self.V, self.lens, self.status)
+    def append(self, Kblk, Vblk, advance: bool = True) -> None:
+        """Block end: write the finalized block's K/V after the prefix and grow it.
+
+        ``advance=False`` writes the rows but keeps the prefix length (a
+        benchmark holds its workload fixed this way)."""
+        fbl.fb_kv_append(self.desc, Kblk, Vblk, self.K, self.V, self.lens if advance else None, self.status)
+        if not advance:
+            return
         old = self.lens_host
         self.lens_host = [min(L + self.S, self.capacity) if L + self.S <= self.capacity else L for L in old]
         if self.topk > 0:
