@@ -32,16 +32,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 4-D bf16 tensor map, innermost dimension first, 128-byte swizzle.
+// 4-D tensor map, innermost dimension first, 128-byte swizzle (bf16 unless
+// `f32` is set).
 bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const uint64_t strides_bytes[3],
-              const uint32_t box[4]) {
+              const uint32_t box[4], bool f32 = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
   cuuint64_t gs[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
   cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
   cuuint32_t es[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gd, gs, bx, es,
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                  const_cast<void*>(base), gd, gs, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -142,6 +144,7 @@ AttnParams base_params(const fb_desc& d) {
   p.nsplit = 1;
   p.scale = d.softmax_scale;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  p.kv_stream_once = (p.n_rt == 1);  // one query tile per unit: each K/V byte is read once
   return p;
 }
 
@@ -153,7 +156,9 @@ int choose_splits(const fb_desc& d, long long est_tiles) {
   const long long units = (long long)d.batch * d.num_kv_heads * ((d.block_len * G + TC_BM - 1) / TC_BM);
   long long max_ns = est_tiles / 4;
   if (max_ns < 1) max_ns = 1;
-  if (d.num_splits > 0) return (int)std::min<long long>(d.num_splits, std::max<long long>(est_tiles, 1));
+  if (max_ns > TC_MAX_SPLITS) max_ns = TC_MAX_SPLITS;
+  if (d.num_splits > 0)
+    return (int)std::min<long long>(std::min<long long>(d.num_splits, TC_MAX_SPLITS), std::max<long long>(est_tiles, 1));
   const long long slots = device_sms();
   if (units >= slots) {
     int best = 1;
@@ -197,6 +202,17 @@ bool q_map(CUtensorMap* m, const fb_desc& d, const void* Q) {
   const uint64_t str[3] = {D * 2, Hq * D * 2, S * Hq * D * 2};
   const uint32_t box[4] = {64, (uint32_t)G, (uint32_t)(TC_BM / G), 1};
   return make_map(m, Q, dims, str, box);
+}
+
+// Cached O_pre [B, S, Hq, D] f32 in the packed query-row order of a tile:
+// 32-float column blocks (128 B) of G heads x 128/G tokens.
+bool pre_map(CUtensorMap* m, const fb_desc& d, const float* O_pre) {
+  const int G = d.num_q_heads / d.num_kv_heads;
+  const uint64_t D = d.head_dim, Hq = d.num_q_heads, S = d.block_len, B = d.batch;
+  const uint64_t dims[4] = {D, Hq, S, B};
+  const uint64_t str[3] = {D * 4, Hq * D * 4, S * Hq * D * 4};
+  const uint32_t box[4] = {32, (uint32_t)G, (uint32_t)(TC_BM / G), 1};
+  return make_map(m, O_pre, dims, str, box, true);
 }
 
 bool block_map(CUtensorMap* m, const fb_desc& d, const void* X) {
@@ -280,7 +296,7 @@ fb_status fb_prefix_partial(const fb_desc* d, const void* Q, const void* Kc, con
   p.out_o32 = part_o;
   p.out_lse = part_l;
   const long long grid = (long long)d->batch * d->num_kv_heads * p.n_rt * ns;
-  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kp, m.vp, (int)grid, s);
+  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kp, m.vp, m.q, (int)grid, s);
   if (e != cudaSuccess || ns == 1) return from_cuda(e);
   CombineParams c;
   std::memset(&c, 0, sizeof(c));
@@ -318,9 +334,12 @@ fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const v
     return from_cuda(launch_attn_simt(p, static_cast<const float*>(Q), nullptr, nullptr,
                                       static_cast<const float*>(Kb), static_cast<const float*>(Vb), s));
   Maps m;
-  if (!q_map(&m.q, *d, Q) || !block_map(&m.kb, *d, Kb) || !block_map(&m.vb, *d, Vb)) return FB_ERR_LAUNCH;
+  CUtensorMap tm_pre;
+  if (!q_map(&m.q, *d, Q) || !block_map(&m.kb, *d, Kb) || !block_map(&m.vb, *d, Vb) ||
+      !pre_map(&tm_pre, *d, O_pre))
+    return FB_ERR_LAUNCH;
   const long long grid = (long long)d->batch * d->num_kv_heads * p.n_rt;
-  return from_cuda(launch_attn_tc(p, m.q, m.kb, m.vb, m.kb, m.vb, (int)grid, s));
+  return from_cuda(launch_attn_tc(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_pre, (int)grid, s));
 }
 
 fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc, const void* Vc,
@@ -359,7 +378,7 @@ fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc,
     p.epi = EPI_NORM;
     p.out_o = O;
     p.out_lse = LSE_out;
-    return from_cuda(launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, (int)units, s));
+    return from_cuda(launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, (int)units, s));
   }
   p.epi = EPI_PARTIAL;
   p.nsplit = ns;
@@ -367,7 +386,7 @@ fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc,
   float* part_l = part_o + (size_t)ns * d->batch * d->block_len * d->num_q_heads * d->head_dim;
   p.out_o32 = part_o;
   p.out_lse = part_l;
-  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, (int)(units * ns), s);
+  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, (int)(units * ns), s);
   if (e != cudaSuccess) return from_cuda(e);
   CombineParams c;
   std::memset(&c, 0, sizeof(c));

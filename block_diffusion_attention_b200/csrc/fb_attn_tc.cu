@@ -16,17 +16,21 @@
 //
 // Warp roles (192 threads):
 //   warps 0-3  softmax: thread r owns query row r (TMEM lane r); online softmax
-//              in fp32 with base-2 exponentials, P to shared memory as bf16,
-//              lazy rescaling of the TMEM accumulator, epilogue;
-//   warp 4     TMA producer: Q once, then K and V tiles into a 2-stage ring;
-//   warp 5     TMEM owner and MMA issuer: S = Q K^T and O += P V with
-//              tcgen05.mma (M = 128, N = 128, K = 16 per instruction).
+//              in fp32 with base-2 exponentials, P written back into tensor
+//              memory as bf16 pairs, lazy rescaling of the accumulator, epilogue;
+//   warp 4     TMA producer: Q once, then K and V tiles into a ring of six
+//              32 KB shared-memory slots (K and V of a tile take one slot each);
+//   warp 5     TMEM owner and MMA issuer: S = Q K^T (A and B from shared
+//              memory) and O += P V (A = P from tensor memory, B = V from
+//              shared memory) with tcgen05.mma, M = 128, N = 128, K = 16.
 //
-// TMEM: S at columns [0, 128), O at [128, 256).
+// TMEM (512 columns): S double-buffered at columns [0, 128) and [128, 256) --
+// tile j's P overwrites the first 64 columns of its own S buffer -- and the
+// O accumulator at [256, 384).  QK^T of tile j + 1 therefore overlaps the
+// softmax of tile j, and a K slot is released as soon as its QK^T is done.
 // Shared memory (1024-byte aligned, 128-byte swizzle everywhere):
-//   Q [2 halves of 64 dims][128 rows][128 B]                 32 KB
-//   per stage: K [2][128 keys][128 B], V [2][128 keys][128 B]  64 KB
-//   P [2 halves of 64 keys][128 rows][128 B]                 32 KB
+//   Q     [2 halves of 64 dims][128 rows][128 B]        32 KB
+//   ring  6 x [2 halves][128 keys][128 B]              192 KB
 //
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // FB_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
@@ -40,19 +44,20 @@ namespace fb {
 
 namespace {
 
-constexpr int BM = TC_BM, BN = TC_BN, HD = TC_D, NST = TC_STAGES;
+constexpr int BM = TC_BM, BN = TC_BN, HD = TC_D, NSLOT = TC_SLOTS;
+static_assert(BM == BN && BN == HD, "square 128 tiles");
 constexpr uint32_t Q_BYTES = BM * HD * 2;       // 32 KB
-constexpr uint32_t KV_TILE_BYTES = BN * HD * 2; // 32 KB (K or V)
+constexpr uint32_t SLOT_BYTES = BN * HD * 2;    // 32 KB: one K or one V tile
 constexpr uint32_t HALF_BYTES = BN * 128;       // one 64-column half of a tile
-constexpr uint32_t P_BYTES = BM * BN * 2;       // 32 KB
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_KV = OFF_Q + Q_BYTES;
-constexpr uint32_t OFF_P = OFF_KV + NST * 2 * KV_TILE_BYTES;
-constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
-constexpr int NUM_BARS = 1 + 3 * NST + 5;
+constexpr uint32_t OFF_RING = OFF_Q + Q_BYTES;
+constexpr uint32_t OFF_BAR = OFF_RING + NSLOT * SLOT_BYTES;
+constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 + 2 + 3;
+constexpr uint32_t PRE_BYTES = BM * HD * 4;      // 64 KB: O_pre rows of a tile (f32)
+constexpr int PRE_SLOT = NSLOT - 2;             // O_pre prefetch uses the last two ring slots
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t TMEM_S = 0, TMEM_O = 128;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_S0 = 0, TMEM_O = 256;           // S buffers at 0 and 128
 constexpr float RESCALE_LOG2 = 8.0f;   // rescale O only when the row max grows by > 2^8
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 constexpr float LN2 = 0.6931471805599453f;
@@ -62,14 +67,13 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 struct Shared {
   uint64_t* q_full;
-  uint64_t* k_full;
-  uint64_t* v_full;
-  uint64_t* empty;
-  uint64_t* s_full;
-  uint64_t* s_free;
-  uint64_t* p_full;
-  uint64_t* o_done;
+  uint64_t* full;    // [NSLOT] ring slot loaded
+  uint64_t* empty;   // [NSLOT] ring slot consumed
+  uint64_t* s_full;  // [2] S buffer written by QK^T
+  uint64_t* p_full;  // [2] P written into that S buffer (and O rescaled)
+  uint64_t* o_done;  // PV finished
   uint64_t* drain;
+  uint64_t* pre_full; // O_pre rows prefetched (merge epilogue of short units)
   uint32_t* tmem_slot;
   volatile int* abort_flag;
 };
@@ -168,7 +172,7 @@ __device__ __forceinline__ Tile tile_at(const AttnParams& p, const UnitTiles& u,
 __device__ __forceinline__ void load_kv_tile(uint8_t* dst, const CUtensorMap* prefix_map,
                                              const CUtensorMap* block_map, uint64_t* bar,
                                              const AttnParams& p, const UnitTiles& u,
-                                             const Tile& t, int b, int kvh) {
+                                             const Tile& t, int b, int kvh, uint64_t policy) {
   const KeySource& s = p.src;
   if (t.seg == 1) {
 #pragma unroll
@@ -177,7 +181,8 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* dst, const CUtensorMap* pr
   }
   if (!s.paged) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) tma_load_4d(dst + h * HALF_BYTES, prefix_map, bar, h * 64, kvh, t.row, b);
+    for (int h = 0; h < 2; ++h)
+      tma_load_4d_hint(dst + h * HALF_BYTES, prefix_map, bar, h * 64, kvh, t.row, b, policy);
     return;
   }
   const int page_size = 1 << s.page_shift;
@@ -195,33 +200,37 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* dst, const CUtensorMap* pr
     const int prow = r & (page_size - 1);
 #pragma unroll
     for (int h = 0; h < 2; ++h)
-      tma_load_4d(dst + h * HALF_BYTES + sub * box * 128, prefix_map, bar, h * 64, kvh, prow, pg);
+      tma_load_4d_hint(dst + h * HALF_BYTES + sub * box * 128, prefix_map, bar, h * 64, kvh, prow, pg,
+                       policy);
   }
 }
+
+// Ring slot sequence: tile j uses slot item 2j for K and 2j + 1 for V.
+__device__ __forceinline__ int slot_of(int item) { return item % NSLOT; }
+__device__ __forceinline__ uint32_t use_of(int item) { return (uint32_t)(item / NSLOT); }
 
 template <int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKp,
                    const __grid_constant__ CUtensorMap tmVp, const __grid_constant__ CUtensorMap tmKb,
-                   const __grid_constant__ CUtensorMap tmVb, const AttnParams p) {
+                   const __grid_constant__ CUtensorMap tmVb, const __grid_constant__ CUtensorMap tmPre,
+                   const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem + OFF_Q;
-  uint8_t* sKV = smem + OFF_KV;
-  uint8_t* sP = smem + OFF_P;
+  uint8_t* sRing = smem + OFF_RING;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   Shared sh;
   sh.q_full = bars;
-  sh.k_full = bars + 1;
-  sh.v_full = sh.k_full + NST;
-  sh.empty = sh.v_full + NST;
-  sh.s_full = sh.empty + NST;
-  sh.s_free = sh.s_full + 1;
-  sh.p_full = sh.s_free + 1;
-  sh.o_done = sh.p_full + 1;
+  sh.full = bars + 1;
+  sh.empty = sh.full + NSLOT;
+  sh.s_full = sh.empty + NSLOT;
+  sh.p_full = sh.s_full + 2;
+  sh.o_done = sh.p_full + 2;
   sh.drain = sh.o_done + 1;
-  sh.tmem_slot = reinterpret_cast<uint32_t*>(sh.drain + 1);
+  sh.pre_full = sh.drain + 1;
+  sh.tmem_slot = reinterpret_cast<uint32_t*>(sh.pre_full + 1);
   sh.abort_flag = reinterpret_cast<volatile int*>(sh.tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -237,16 +246,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(sh.q_full, 1);
-    for (int i = 0; i < NST; ++i) {
-      mbar_init(&sh.k_full[i], 1);
-      mbar_init(&sh.v_full[i], 1);
+    for (int i = 0; i < NSLOT; ++i) {
+      mbar_init(&sh.full[i], 1);
       mbar_init(&sh.empty[i], 1);
     }
-    mbar_init(sh.s_full, 1);
-    mbar_init(sh.s_free, 128);
-    mbar_init(sh.p_full, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.s_full[i], 1);
+      mbar_init(&sh.p_full[i], 4);
+    }
     mbar_init(sh.o_done, 1);
     mbar_init(sh.drain, 1);
+    mbar_init(sh.pre_full, 1);
     *sh.abort_flag = 0;
     fence_barrier_init();
   }
@@ -258,6 +268,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *sh.tmem_slot;
+  // Everything above touches no global memory; from here on inputs may come
+  // from the previous kernel in the stream.
+  pdl_wait();
+  pdl_launch_dependents();
 
   const UnitTiles u = unit_tiles(p, b, kvh, threadIdx.x == 0);
   const int ntot = u.n0 + u.n1;
@@ -265,6 +279,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int j1 = (int)(((long long)(split + 1) * ntot) / p.nsplit);
   const int nt = j1 - j0;
   int32_t* status = p.dev_status;
+  // The merge epilogue of a unit with at most two key tiles leaves the last
+  // two ring slots free: the cached O_pre rows are prefetched into them.
+  const bool pre_smem = (EPI == EPI_MERGE) && nt <= 2;
 
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
@@ -272,95 +289,105 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tma_prefetch_map(&tmQ);
       tma_prefetch_map(&tmKp);
       tma_prefetch_map(&tmVp);
+      const uint64_t policy = p.kv_stream_once ? l2_policy_evict_first() : l2_policy_evict_normal();
       mbar_arrive_expect_tx(sh.q_full, Q_BYTES);
       const int t0 = rt * (BM / p.G);
       tma_load_4d(sQ, &tmQ, sh.q_full, 0, kvh * p.G, t0, b);
       tma_load_4d(sQ + BM * 128, &tmQ, sh.q_full, 64, kvh * p.G, t0, b);
-      int issued = 0;
+      if (pre_smem) {
+        // [4 column blocks of 32 floats][128 rows][128 B], 128-byte swizzle
+        mbar_arrive_expect_tx(sh.pre_full, PRE_BYTES);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tma_load_4d(sRing + PRE_SLOT * SLOT_BYTES + c * (BM * 128), &tmPre, sh.pre_full, c * 32, kvh * p.G,
+                      t0, b);
+      }
+      int issued = 0;  // ring items issued
       for (int jj = 0; jj < nt; ++jj) {
-        const int st = jj % NST;
-        const uint32_t use = jj / NST;
-        if (!wait_bar(&sh.empty[st], (use & 1) ^ 1, sh, status)) break;
         const Tile t = tile_at(p, u, b, kvh, j0 + jj);
-        uint8_t* dK = sKV + st * 2 * KV_TILE_BYTES;
-        uint8_t* dV = dK + KV_TILE_BYTES;
-        mbar_arrive_expect_tx(&sh.k_full[st], KV_TILE_BYTES);
-        load_kv_tile(dK, &tmKp, &tmKb, &sh.k_full[st], p, u, t, b, kvh);
-        mbar_arrive_expect_tx(&sh.v_full[st], KV_TILE_BYTES);
-        load_kv_tile(dV, &tmVp, &tmVb, &sh.v_full[st], p, u, t, b, kvh);
-        issued = jj + 1;
+        bool ok = true;
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+          const int item = 2 * jj + kv;
+          const int sl = slot_of(item);
+          if (!(ok = wait_bar(&sh.empty[sl], (use_of(item) & 1) ^ 1, sh, status))) break;
+          mbar_arrive_expect_tx(&sh.full[sl], SLOT_BYTES);
+          load_kv_tile(sRing + sl * SLOT_BYTES, kv ? &tmVp : &tmKp, kv ? &tmVb : &tmKb, &sh.full[sl], p, u,
+                       t, b, kvh, policy);
+          issued = item + 1;
+        }
+        if (!ok) break;
       }
       // After an abort, let the copies in flight land before the CTA exits.
       if (*sh.abort_flag) {
         wait_bar(sh.q_full, 0, sh, nullptr, false);
-        for (int jj = max(0, issued - NST); jj < issued; ++jj) {
-          const int st = jj % NST;
-          const uint32_t use = jj / NST;
-          wait_bar(&sh.k_full[st], use & 1, sh, nullptr, false);
-          wait_bar(&sh.v_full[st], use & 1, sh, nullptr, false);
-        }
+        if (pre_smem) wait_bar(sh.pre_full, 0, sh, nullptr, false);
+        for (int item = max(0, issued - NSLOT); item < issued; ++item)
+          wait_bar(&sh.full[slot_of(item)], use_of(item) & 1, sh, nullptr, false);
       }
     }
   } else if (warp == 5) {
     // --------------------------------------------------------------- MMA issuer
-    constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
     constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
-    const uint32_t tS = tmem + TMEM_S;
     const uint32_t tO = tmem + TMEM_O;
     const uint32_t aQ = smem_u32(sQ);
-    const uint32_t aP = smem_u32(sP);
-    auto issue_qk = [&](int st) {
-      const uint32_t aK = smem_u32(sKV + st * 2 * KV_TILE_BYTES);
+    // A tile with fewer valid keys runs N = (valid keys rounded up to 16) for
+    // QK^T and as many 16-key steps of PV: no work on empty columns.
+    auto issue_qk = [&](int jj) {
+      const Tile t = tile_at(p, u, b, kvh, j0 + jj);
+      const int n16 = (t.nvalid + 15) & ~15;
+      const uint32_t idesc = idesc_bf16_f32(BM, n16, false, false);
+      const uint32_t aK = smem_u32(sRing + slot_of(2 * jj) * SLOT_BYTES);
+      const uint32_t tS = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN;
 #pragma unroll
       for (int kk = 0; kk < HD / 16; ++kk) {
         const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-        umma_bf16_ss(tS, sw128_desc(aQ + off, 16, 1024), sw128_desc(aK + off, 16, 1024), IDESC_QK,
-                     kk > 0);
+        umma_bf16_ss(tS, sw128_desc(aQ + off, 16, 1024), sw128_desc(aK + off, 16, 1024), idesc, kk > 0);
       }
     };
-    auto issue_pv = [&](int st, bool acc) {
-      const uint32_t aV = smem_u32(sKV + st * 2 * KV_TILE_BYTES + KV_TILE_BYTES);
+    auto issue_pv = [&](int jj, int nvalid) {
+      const uint32_t aV = smem_u32(sRing + slot_of(2 * jj + 1) * SLOT_BYTES);
+      const uint32_t tP = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN;  // P (bf16 pairs) over S
+      const int ksteps = (nvalid + 15) >> 4;
 #pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk) {
-        const uint32_t offp = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-        umma_bf16_ss(tO, sw128_desc(aP + offp, 16, 1024),
-                     sw128_desc(aV + kk * 16 * 128, HALF_BYTES, 1024), IDESC_PV,
-                     (acc || kk > 0) ? 1u : 0u);
-      }
+      for (int kk = 0; kk < BN / 16; ++kk)
+        if (kk < ksteps)
+          umma_bf16_ts(tO, tP + kk * 8, sw128_desc(aV + kk * 16 * 128, HALF_BYTES, 1024), IDESC_PV,
+                       (jj > 0 || kk > 0) ? 1u : 0u);
     };
     bool ok = wait_bar(sh.q_full, 0, sh, status);
     if (ok && nt > 0) {
-      ok = wait_bar(&sh.k_full[0], 0, sh, status);
+      ok = wait_bar(&sh.full[slot_of(0)], 0, sh, status);
       if (ok) {
         tc_fence_after_sync();
         if (lane == 0) {
           issue_qk(0);
-          tc_commit(sh.s_full);
+          tc_commit(&sh.s_full[0]);
+          tc_commit(&sh.empty[slot_of(0)]);
         }
         __syncwarp();
       }
       for (int jj = 0; ok && jj < nt; ++jj) {
-        const int st = jj % NST;
-        const uint32_t use = jj / NST;
         if (jj + 1 < nt) {
-          const int st1 = (jj + 1) % NST;
-          const uint32_t use1 = (jj + 1) / NST;
-          if (!(ok = wait_bar(&sh.k_full[st1], use1 & 1, sh, status))) break;
-          if (!(ok = wait_bar(sh.s_free, jj & 1, sh, status))) break;
+          const int ik = 2 * (jj + 1);
+          if (!(ok = wait_bar(&sh.full[slot_of(ik)], use_of(ik) & 1, sh, status))) break;
           tc_fence_after_sync();
           if (lane == 0) {
-            issue_qk(st1);
-            tc_commit(sh.s_full);
+            issue_qk(jj + 1);
+            tc_commit(&sh.s_full[(jj + 1) & 1]);
+            tc_commit(&sh.empty[slot_of(ik)]);
           }
           __syncwarp();
         }
-        if (!(ok = wait_bar(&sh.v_full[st], use & 1, sh, status))) break;
+        const int iv = 2 * jj + 1;
+        if (!(ok = wait_bar(&sh.full[slot_of(iv)], use_of(iv) & 1, sh, status))) break;
         const Tile t = tile_at(p, u, b, kvh, j0 + jj);
-        if (t.seg == 0 && t.nvalid < BN) {
+        if (t.seg == 0 && (t.nvalid & 15)) {
           // Cache rows past the prefix may hold anything (even NaN); P is 0
-          // there but 0 * NaN is not, so clear those V rows.
-          uint8_t* dV = sKV + st * 2 * KV_TILE_BYTES + KV_TILE_BYTES;
-          const int nrow = BN - t.nvalid;
+          // there but 0 * NaN is not, so clear the V rows up to the next
+          // 16-key step that PV reads.
+          uint8_t* dV = sRing + slot_of(iv) * SLOT_BYTES;
+          const int nrow = ((t.nvalid + 15) & ~15) - t.nvalid;
           for (int i = lane; i < nrow * 16; i += 32) {
             const int r = t.nvalid + (i >> 4);
             const int h = (i >> 3) & 1;
@@ -370,12 +397,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           fence_proxy_async_smem();
         }
         __syncwarp();
-        if (!(ok = wait_bar(sh.p_full, jj & 1, sh, status))) break;
+        if (!(ok = wait_bar(&sh.p_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
         tc_fence_after_sync();
         if (lane == 0) {
-          issue_pv(st, jj > 0);
+          issue_pv(jj, t.nvalid);
           tc_commit(sh.o_done);
-          tc_commit(&sh.empty[st]);
+          tc_commit(&sh.empty[slot_of(iv)]);
         }
         __syncwarp();
       }
@@ -388,33 +415,44 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // ------------------------------------------------------ softmax + epilogue
     const int r = warp * 32 + lane;  // query row of this thread = TMEM lane
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t tS = tmem + TMEM_S + lane_off;
     const uint32_t tO = tmem + TMEM_O + lane_off;
-    const uint32_t p_row = smem_u32(sP) + r * 128;
     const float c2 = p.scale_log2;
+    const int pr = rt * BM + r;
+    const int tok = pr / p.G;
+    const int h = kvh * p.G + (pr - tok * p.G);
+    // cached LSE of this row, read before the key loop so its latency hides
+    const float lp_nat = (EPI == EPI_MERGE && tok < p.S) ? p.pre_lse[((size_t)b * p.Hq + h) * p.S + tok]
+                                                          : -CUDART_INF_F;
     float m_run = -CUDART_INF_F;
     float l_run = 0.f;
     bool ok = true;
     for (int jj = 0; jj < nt; ++jj) {
-      if (!(ok = wait_bar(sh.s_full, jj & 1, sh, status))) break;
+      const uint32_t tS = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN + lane_off;
+      const Tile t = tile_at(p, u, b, kvh, j0 + jj);
+      if (!(ok = wait_bar(&sh.s_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
       tc_fence_after_sync();
+      // S row of this thread.  A tail tile (fewer than BN valid keys) sets
+      // the columns past its keys to -inf first; full tiles skip that block.
       uint32_t sv[BN];
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c)
         tmem_ld_32x32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[c * 32]));
       tmem_ld_wait();
-      tc_fence_before_sync();
-      mbar_arrive(sh.s_free);
-
-      const Tile t = tile_at(p, u, b, kvh, j0 + jj);
-      float s[BN];
-      float mx = -CUDART_INF_F;
+      if (t.nvalid < BN) {
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        s[c] = (c < t.nvalid) ? __uint_as_float(sv[c]) : -CUDART_INF_F;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < BN; ++c)
+          if (c >= t.nvalid) sv[c] = 0xff800000u;  // -inf
       }
-      const float mt = mx * c2;
+      float* s = reinterpret_cast<float*>(sv);  // S, then p in place
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+      for (int c = 4; c < BN; c += 4) {
+        mx0 = fmaxf(mx0, s[c]);
+        mx1 = fmaxf(mx1, s[c + 1]);
+        mx2 = fmaxf(mx2, s[c + 2]);
+        mx3 = fmaxf(mx3, s[c + 3]);
+      }
+      const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c2;
       const bool need = mt > m_run + RESCALE_LOG2;
       const float m_new = need ? mt : m_run;
       const float alpha = ex2_approx(m_run - m_new);  // 0 when m_run = -inf
@@ -435,8 +473,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       m_run = m_new;
 
       if (jj > 0) {
-        // PV of the previous tile must be done: P is single-buffered and O
-        // may be rescaled below.
+        // Wait for the previous tile's PV before publishing this tile's P:
+        // o_done then never runs more than one phase ahead of this wait, and
+        // the accumulator is stable if rows whose max moved need rescaling.
         if (!(ok = wait_bar(sh.o_done, (jj - 1) & 1, sh, status))) break;
         tc_fence_after_sync();
         if (__any_sync(0xffffffffu, need)) {
@@ -449,31 +488,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
             tmem_st_32x32(tO + c * 32, ov);
           }
-          tmem_st_wait();
         }
       }
-      // P (bf16) into the K-major, 128-byte-swizzled A-operand layout.
+      // P as bf16 pairs over the first 64 columns of this S buffer: the
+      // A operand of PV, read from tensor memory.
 #pragma unroll
-      for (int c = 0; c < BN; c += 8) {
-        const int half = c >> 6;
-        const int chunk = (c & 63) >> 3;
-        const uint32_t addr = p_row + half * (BM * 128) + ((chunk ^ (r & 7)) << 4);
-        st_shared_v4(addr, pack_bf16x2(s[c], s[c + 1]), pack_bf16x2(s[c + 2], s[c + 3]),
-                     pack_bf16x2(s[c + 4], s[c + 5]), pack_bf16x2(s[c + 6], s[c + 7]));
+      for (int c = 0; c < BN / 64; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[c * 64 + 2 * i], s[c * 64 + 2 * i + 1]);
+        tmem_st_32x32(tS + c * 32, pk);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sh.p_full);
+      if (lane == 0) mbar_arrive(&sh.p_full[jj & 1]);
     }
     if (ok && nt > 0) {
       ok = wait_bar(sh.o_done, (nt - 1) & 1, sh, status);
       tc_fence_after_sync();
     }
+    if (ok && pre_smem) ok = wait_bar(sh.pre_full, 0, sh, status);
     // ---------------------------------------------------------------- epilogue
-    const int pr = rt * BM + r;
-    const int tok = pr / p.G;
-    const int h = kvh * p.G + (pr - tok * p.G);
     const bool row_ok = ok && tok < p.S;
     const bool empty = (nt == 0) || !(l_run > 0.f);
     const float inv_l = empty ? 0.f : 1.f / l_run;
@@ -507,8 +543,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       float wp = 0.f, wo = inv_l, inv_den = 1.f, lse_out2 = lse2;
       if (EPI == EPI_MERGE) {
         // merge equation in base 2: weights e^{L - m} become 2^{L2 - M}
-        const float lp2 = row_ok ? p.pre_lse[((size_t)b * p.Hq + h) * p.S + tok] * 1.4426950408889634f
-                                 : -CUDART_INF_F;
+        const float lp2 = row_ok ? lp_nat * 1.4426950408889634f : -CUDART_INF_F;
         const float M = fmaxf(lp2, lse2);
         const float Ms = (M == -CUDART_INF_F) ? 0.f : M;
         wp = ex2_approx(lp2 - Ms);
@@ -530,9 +565,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(ov[i]) * wo;
           if (EPI == EPI_MERGE) {
+            const uint8_t* prow = sRing + PRE_SLOT * SLOT_BYTES + c * (BM * 128) + r * 128;
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
-              const float4 q = *reinterpret_cast<const float4*>(pre + c * 32 + i);
+              const float4 q = pre_smem ? *reinterpret_cast<const float4*>(prow + (((i >> 2) ^ (r & 7)) << 4))
+                                        : *reinterpret_cast<const float4*>(pre + c * 32 + i);
               o[i] = (o[i] + wp * q.x) * inv_den;
               o[i + 1] = (o[i + 1] + wp * q.y) * inv_den;
               o[i + 2] = (o[i + 2] + wp * q.z) * inv_den;
@@ -560,10 +597,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 }
 
 // Log-space merge of the split-key partials of one query row (the merge
-// equation applied across splits, in a fixed order).  One warp per row.
-__global__ void combine_kernel(const CombineParams c) {
-  const int warps = blockDim.x >> 5;
-  const long long row = (long long)blockIdx.x * warps + (threadIdx.x >> 5);
+// equation applied across splits, in a fixed order).  One warp per row: lanes
+// read the splits' LSEs in parallel, the split weights go to shared memory,
+// then each lane accumulates four output columns over the splits.
+constexpr int CMB_WARPS = 4;
+constexpr int CMB_INFLIGHT = 16;  // split loads in flight per lane
+
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombineParams c) {
+  __shared__ float wsm[CMB_WARPS][TC_MAX_SPLITS];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int wi = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * CMB_WARPS + wi;
   const int lane = threadIdx.x & 31;
   const long long nrows = (long long)c.B * c.S * c.Hq;
   if (row >= nrows) return;
@@ -571,33 +627,48 @@ __global__ void combine_kernel(const CombineParams c) {
   const long long bt = row / c.Hq;
   const int t = (int)(bt % c.S);
   const int b = (int)(bt / c.S);
-  const size_t split_stride_o = (size_t)nrows * c.D;
-  const size_t split_stride_l = (size_t)c.B * c.Hq * c.S;
+  const size_t so = (size_t)nrows * c.D;              // split stride of the partial O
+  const size_t sl = (size_t)c.B * c.Hq * c.S;         // split stride of the partial LSE
   const size_t lrow = ((size_t)b * c.Hq + h) * c.S + t;
   float M = -CUDART_INF_F;
-  for (int s = 0; s < c.nsplit; ++s) M = fmaxf(M, c.part_lse[s * split_stride_l + lrow]);
+  for (int s = lane; s < c.nsplit; s += 32) M = fmaxf(M, c.part_lse[s * sl + lrow]);
+  M = warp_max_f(M);
   const bool empty = (M == -CUDART_INF_F);
   float den = 0.f;
+  for (int s = lane; s < c.nsplit; s += 32) {
+    const float ls = c.part_lse[s * sl + lrow];
+    const float w = (empty || ls == -CUDART_INF_F) ? 0.f : expf(ls - M);
+    wsm[wi][s] = w;
+    den += w;
+  }
+  den = warp_sum_f(den);
+  __syncwarp();
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  const float* base = c.part_o + row * c.D;
   for (int d0 = lane * 4; d0 < c.D; d0 += 128) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    den = 0.f;
-    if (!empty) {
-      for (int s = 0; s < c.nsplit; ++s) {
-        const float ls = c.part_lse[s * split_stride_l + lrow];
-        const float w = (ls == -CUDART_INF_F) ? 0.f : expf(ls - M);
-        den += w;
-        const float4 v = *reinterpret_cast<const float4*>(c.part_o + s * split_stride_o + row * c.D + d0);
-        acc.x += w * v.x;
-        acc.y += w * v.y;
-        acc.z += w * v.z;
-        acc.w += w * v.w;
+    // CMB_INFLIGHT splits' loads in flight at once, then the weighted sum in
+    // split order
+    for (int s0 = 0; s0 < c.nsplit; s0 += CMB_INFLIGHT) {
+      float4 v[CMB_INFLIGHT];
+#pragma unroll
+      for (int i = 0; i < CMB_INFLIGHT; ++i)
+        if (s0 + i < c.nsplit) v[i] = __ldg(reinterpret_cast<const float4*>(base + (s0 + i) * so + d0));
+#pragma unroll
+      for (int i = 0; i < CMB_INFLIGHT; ++i) {
+        if (s0 + i < c.nsplit) {
+          const float w = wsm[wi][s0 + i];
+          acc.x = fmaf(w, v[i].x, acc.x);
+          acc.y = fmaf(w, v[i].y, acc.y);
+          acc.z = fmaf(w, v[i].z, acc.z);
+          acc.w = fmaf(w, v[i].w, acc.w);
+        }
       }
-      const float inv = 1.f / den;
-      acc.x *= inv;
-      acc.y *= inv;
-      acc.z *= inv;
-      acc.w *= inv;
     }
+    acc.x *= inv;
+    acc.y *= inv;
+    acc.z *= inv;
+    acc.w *= inv;
     if (c.out_o32) {
       *reinterpret_cast<float4*>(c.out_o32 + row * c.D + d0) = acc;
     } else if (c.out_bf16) {
@@ -607,18 +678,7 @@ __global__ void combine_kernel(const CombineParams c) {
       *reinterpret_cast<float4*>(reinterpret_cast<float*>(c.out_o) + row * c.D + d0) = acc;
     }
   }
-  if (lane == 0 && c.out_lse) {
-    if (empty) {
-      c.out_lse[lrow] = -CUDART_INF_F;
-    } else {
-      float dd = 0.f;
-      for (int s = 0; s < c.nsplit; ++s) {
-        const float ls = c.part_lse[s * split_stride_l + lrow];
-        dd += (ls == -CUDART_INF_F) ? 0.f : expf(ls - M);
-      }
-      c.out_lse[lrow] = M + logf(dd);
-    }
-  }
+  if (lane == 0 && c.out_lse) c.out_lse[lrow] = empty ? -CUDART_INF_F : M + logf(den);
 }
 
 }  // namespace
@@ -626,13 +686,13 @@ __global__ void combine_kernel(const CombineParams c) {
 size_t tc_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
-                           const CUtensorMap& tmVp, const CUtensorMap& tmKb,
-                           const CUtensorMap& tmVb, int grid, cudaStream_t stream) {
+                           const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
+                           const CUtensorMap& tmPre, int grid, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static bool configured[64][3] = {};
-  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, AttnParams);
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, AttnParams);
   switch (p.epi) {
     case EPI_PARTIAL: kern = attn_tc_kernel<EPI_PARTIAL>; break;
     case EPI_MERGE: kern = attn_tc_kernel<EPI_MERGE>; break;
@@ -643,18 +703,35 @@ cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CU
     if (e != cudaSuccess) return e;
     configured[dev][p.epi] = true;
   }
-  kern<<<grid, TC_THREADS, SMEM_BYTES, stream>>>(tmQ, tmKp, tmVp, tmKb, tmVb, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tmQ, tmKp, tmVp, tmKb, tmVb, tmPre, p);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_combine(const CombineParams& c, cudaStream_t stream) {
   const long long rows = (long long)c.B * c.S * c.Hq;
-  const int warps = 8;
-  const long long grid = (rows + warps - 1) / warps;
-  combine_kernel<<<(unsigned)grid, warps * 32, 0, stream>>>(c);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((rows + CMB_WARPS - 1) / CMB_WARPS));
+  cfg.blockDim = dim3(CMB_WARPS * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel, c);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace fb

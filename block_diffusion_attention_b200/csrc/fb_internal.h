@@ -41,6 +41,7 @@ struct AttnParams {
   float scale;   // softmax scale (natural units)
   float scale_log2;  // scale * log2(e)
   int epi;
+  int kv_stream_once;  // 1: prefix K/V is read once (evict-first L2 hint)
   KeySource src;
   // outputs
   float* out_o32;         // EPI_PARTIAL: [nsplit][B][S][Hq][D]
@@ -65,12 +66,13 @@ struct CombineParams {
 constexpr int TC_BM = 128;      // query rows per tile (TMEM lanes)
 constexpr int TC_BN = 128;      // keys per tile
 constexpr int TC_D = 128;       // head dim
-constexpr int TC_STAGES = 2;    // K/V ring depth
+constexpr int TC_SLOTS = 6;     // K/V ring: 32 KB slots (K and V of a tile take one each)
 constexpr int TC_THREADS = 192; // 4 softmax warps + TMA warp + MMA warp
+constexpr int TC_MAX_SPLITS = 128;  // key-range splits per work unit
 size_t tc_smem_bytes();
 cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
-                           const CUtensorMap& tmVp, const CUtensorMap& tmKb,
-                           const CUtensorMap& tmVb, int grid, cudaStream_t stream);
+                           const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
+                           const CUtensorMap& tmPre, int grid, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& c, cudaStream_t stream);
 
 // CUDA-core (fp32) path.
