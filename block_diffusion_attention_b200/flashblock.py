@@ -68,6 +68,7 @@ def load() -> ctypes.CDLL:
             "fb_cache_rows": (ctypes.c_int64, [D]),
             "fb_workspace_bytes": (SZ, [D]),
             "fb_prefix_partial": (I32, [D, P, P, P, P, P, P, P, SZ, P, P]),
+            "fb_prefix_partial_noalloc": (I32, [D, P, P, P, P, P, P, P, P]),
             "fb_block_step": (I32, [D, P, P, P, P, P, P, P, P, P]),
             "fb_full_reference_gpu": (I32, [D, P, P, P, P, P, P, P, P, SZ, P, P]),
             "fb_chunk_means": (I32, [D, P, I32, I32, P, P, P]),
@@ -141,6 +142,13 @@ def fb_prefix_partial(d, Q, Kcache, Vcache, chunk_idx, O_pre, LSE_pre, workspace
     _ok("fb_prefix_partial", load().fb_prefix_partial(
         ctypes.byref(d), _p(Q), _p(Kcache), _p(Vcache), _p(chunk_idx), _p(O_pre), _p(LSE_pre),
         _p(workspace), _nbytes(workspace), _p(dev_status), _s(stream)))
+
+
+def fb_prefix_partial_noalloc(d, Q, Kcache, Vcache, chunk_idx, O_pre, LSE_pre, dev_status, stream=None):
+    """fb_prefix_partial with the library's static scratch in place of a workspace."""
+    _ok("fb_prefix_partial_noalloc", load().fb_prefix_partial_noalloc(
+        ctypes.byref(d), _p(Q), _p(Kcache), _p(Vcache), _p(chunk_idx), _p(O_pre), _p(LSE_pre),
+        _p(dev_status), _s(stream)))
 
 
 def fb_block_step(d, Q, Kblk, Vblk, O_pre, LSE_pre, O, LSE_out, dev_status, stream=None):

@@ -159,6 +159,31 @@ fb_status fb_kv_append(const fb_desc* d, const void* Kblk, const void* Vblk,
                        void* Kcache, void* Vcache, int32_t* lens_inout,
                        int32_t* dev_status, fb_stream_t stream);
 
+/* Bytes of the static scratch array behind fb_prefix_partial_noalloc. */
+#define FB_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* fb_prefix_partial for callers that cannot allocate device memory (a graph
+ * being captured, a fixed device-memory arena, a serving loop that must not
+ * trigger allocator synchronisation).  No counterpart in the paper: it is a
+ * deployment variant of the prefix pass.  Same arguments and results as
+ * fb_prefix_partial without the workspace: the split-key partials go to a
+ * FB_NOALLOC_SCRATCH_BYTES array inside the library's device image, present
+ * on every GPU that loads the library until the process exits.
+ *  - Allocates nothing and calls no allocating routine.
+ *  - Returns FB_ERR_WORKSPACE (nothing launched) when this call's partials
+ *    need more than FB_NOALLOC_SCRATCH_BYTES (fb_workspace_bytes() says how
+ *    much a descriptor needs; long single sequences fit, e.g. 9.5 MB at
+ *    B = 1, S = 32, Hq = 32, 128K prefix).
+ *  - The first call on each device looks up the array's device address with
+ *    that device current; make that first call before any stream capture.
+ *  - All calls share the one array, which keeps the last call's contents
+ *    (nothing in it needs to start at zero).  Calls that can overlap on the
+ *    GPU (other streams, other host threads) race on it: serialise them. */
+fb_status fb_prefix_partial_noalloc(const fb_desc* d, const void* Q, const void* Kcache,
+                                    const void* Vcache, const int32_t* chunk_idx,
+                                    float* O_pre, float* LSE_pre, int32_t* dev_status,
+                                    fb_stream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* fb_status_string(fb_status s);
 
