@@ -14,6 +14,11 @@ flush is needed between steps.  The append writes the block's rows after the
 prefix without advancing the prefix length, so every timed block sees exactly
 the configured prefix.
 
+By default each block is recorded once as a CUDA graph and replayed (the
+library's calls are capturable); ``--no-graph`` issues every call from the
+host.  The eager cached block is always timed too: CUDA events around its
+prefix pass give the roofline figures of the dominant kernel.
+
 ``value`` is cached attention tokens/s over all ranks (B * S tokens finalized
 per block per rank).  Under torchrun each rank runs an independent replica
 (weak scaling; the path has no collective).  Rank 0 prints one JSON line.
@@ -45,6 +50,8 @@ def parse():
     ap.add_argument("--workload", default="long_ctx")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="issue every call from the host instead of replaying one CUDA graph per block")
     ap.add_argument("--phases", default="cached,uncached,e2e",
                     help="comma list of timed phases (profiling runs may keep only 'cached')")
     return ap.parse_args()
@@ -310,7 +317,8 @@ def run_ours(args):
         res.setdefault("launch_counts", []).append(n1 - n0)
         return max_over_ranks(t0.elapsed_time(t1))
 
-    # ---- cached (FlashBlock) path: the headline
+    # ---- cached (FlashBlock) path, eager: events around the prefix pass give
+    # the roofline of the dominant kernel
     cached = new_layer()
     nref = len(w.refresh)
     # events only around the prefix pass: an event between two kernels would
@@ -336,8 +344,8 @@ def run_ours(args):
     # clocks are sampled from the first warm-up block to the end of the last timed phase
     sampler = ClockSampler(local)
     sampler.start()
-    res["ms_cached"] = timed(cached_block, cached)
-    res["launches"] = res["launch_counts"][0]
+    res["ms_cached_eager"] = timed(cached_block, cached)
+    res["launches_per_block"] = res["launch_counts"][0] / args.steps
     res["lens1"] = [int(x) for x in cached.lens.cpu()]
     res["pre_ms"] = [a.elapsed_time(b) for a, b in ev_pre]
     # block-step latency on its own: back-to-back denoising steps
@@ -354,44 +362,81 @@ def run_ours(args):
     torch.cuda.synchronize()
     res["blk_ms"] = [e0.elapsed_time(e1) / reps]
     cached.check()
+
+    # ---- cached path as one CUDA graph per block: the headline
+    use_graph = not args.no_graph
+    if use_graph:
+        g_cached = cached.capture_block(dev_in, outs, w.refresh, append_kv=(dev_in[-1][1], dev_in[-1][2]))
+        res["ms_cached"] = timed(lambda k: g_cached.replay(), cached)
+        del g_cached
+    else:
+        res["ms_cached"] = res["ms_cached_eager"]
+    res["launches"] = int(res["launches_per_block"] * args.steps)
     del cached
 
     # ---- uncached baseline: full attention at every denoising step
     if "uncached" in phases:
         unc = new_layer()
-
-        def uncached_block(k):
-            for s in range(w.steps):
-                Q, Kb, Vb = dev_in[s]
-                unc.full(Q, Kb, Vb, out=outs[s])
-            unc.append(dev_in[-1][1], dev_in[-1][2], advance=False)
-
-        res["ms_unc"] = timed(uncached_block, unc)
+        if use_graph:
+            g_unc = unc.capture_block(dev_in, outs, w.refresh, append_kv=(dev_in[-1][1], dev_in[-1][2]),
+                                      cached=False)
+            res["ms_unc"] = timed(lambda k: g_unc.replay(), unc)
+            del g_unc
+        else:
+            def uncached_block(k):
+                unc.run_block(dev_in, outs, w.refresh, (dev_in[-1][1], dev_in[-1][2]), advance=False,
+                              cached=False)
+            res["ms_unc"] = timed(uncached_block, unc)
         del unc
 
-    # ---- end to end through the public API: pinned host inputs in, O out
+    # ---- end to end through the public API: the block's inputs copied in from
+    # pinned host memory (one copy) and its outputs read back (one copy),
+    # inside the timed region
     if "e2e" in phases:
         e2e_layer = new_layer()
-        host_in = [tuple(x.pin_memory() for x in t) for t in step_in]
-        host_out = [torch.empty(dev_in[0][0].shape, dtype=dev_in[0][0].dtype).pin_memory()
-                    for _ in range(w.steps)]
-        stage = [tuple(torch.empty_like(x) for x in t) for t in dev_in]
+        flat = [x.reshape(-1) for t in step_in for x in t]
+        sizes = [x.numel() for x in flat]
+        host_in = torch.cat(flat).pin_memory()
+        dev_flat = torch.empty_like(host_in, device="cuda")
+        stage, off = [], 0
+        for t in step_in:
+            views = []
+            for x in t:
+                views.append(dev_flat[off:off + x.numel()].view(x.shape))
+                off += x.numel()
+            stage.append(tuple(views))
+        outs_all = torch.empty((w.steps,) + tuple(dev_in[0][0].shape), dtype=dev_in[0][0].dtype, device="cuda")
+        e2e_outs = [outs_all[s] for s in range(w.steps)]
+        host_out = torch.empty(outs_all.shape, dtype=outs_all.dtype).pin_memory()
 
-        def e2e_block(k):
-            for s in range(w.steps):
-                for dst, src in zip(stage[s], host_in[s]):
-                    dst.copy_(src, non_blocking=True)
-                Q, Kb, Vb = stage[s]
-                if s in w.refresh:
-                    e2e_layer.refresh(Q)
-                o = e2e_layer.step(Q, Kb, Vb, out=outs[s])
-                host_out[s].copy_(o, non_blocking=True)
-            e2e_layer.append(stage[-1][1], stage[-1][2], advance=False)
+        def copy_in(s):
+            if s == 0:
+                dev_flat.copy_(host_in, non_blocking=True)
 
-        res["ms_e2e"] = timed(e2e_block, e2e_layer)
-        res["h2d"] = sum(x.numel() * x.element_size() for t in host_in for x in t)
-        res["d2h"] = sum(x.numel() * x.element_size() for x in host_out)
+        def copy_out(s):
+            if s == w.steps - 1:
+                host_out.copy_(outs_all, non_blocking=True)
+
+        if use_graph:
+            g_e2e = e2e_layer.capture_block(stage, e2e_outs, w.refresh, append_kv=(stage[-1][1], stage[-1][2]),
+                                            prologue=copy_in, epilogue=copy_out)
+            res["ms_e2e"] = timed(lambda k: g_e2e.replay(), e2e_layer)
+            del g_e2e
+        else:
+            def e2e_block(k):
+                for s in range(w.steps):
+                    copy_in(s)
+                    Q, Kb, Vb = stage[s]
+                    if s in w.refresh:
+                        e2e_layer.refresh(Q)
+                    e2e_layer.step(Q, Kb, Vb, out=e2e_outs[s])
+                    copy_out(s)
+                e2e_layer.append(stage[-1][1], stage[-1][2], advance=False)
+            res["ms_e2e"] = timed(e2e_block, e2e_layer)
+        res["h2d"] = host_in.numel() * host_in.element_size()
+        res["d2h"] = host_out.numel() * host_out.element_size()
         del e2e_layer
+    res["graph"] = use_graph
 
     res["clocks"] = sampler.stop()
     if world > 1:
@@ -426,6 +471,8 @@ def report(args, w0, w, world, res):
         "data": "synthetic (seeded N(0,1) K/V, scaled Q, per-step drift)",
         "config": workload_config(w0, {"prefix_rows_during_timing": [min(res["lens0"]), max(res["lens1"])]}),
         "cached_us_per_denoise_step": ms_c * 1e3 / (args.steps * w.steps),
+        "cached_eager_us_per_denoise_step": res["ms_cached_eager"] * 1e3 / (args.steps * w.steps),
+        "launch_mode": "one CUDA graph per block" if res["graph"] else "eager host launches",
         "uncached_us_per_denoise_step": ms_u * 1e3 / (args.steps * w.steps) if ms_u else None,
         "uncached_tokens_per_s": tps(ms_u),
         "cached_over_uncached_speedup": (ms_u / ms_c) if ms_u else None,

@@ -209,12 +209,15 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* dst, const CUtensorMap* pr
 __device__ __forceinline__ int slot_of(int item) { return item % NSLOT; }
 __device__ __forceinline__ uint32_t use_of(int item) { return (uint32_t)(item / NSLOT); }
 
-template <int EPI>
+// NC: key columns a tile can hold valid keys in (128, or 32/64 for the
+// in-block step of a short block, where every tile has at most NC keys).
+template <int EPI, int NC>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKp,
                    const __grid_constant__ CUtensorMap tmVp, const __grid_constant__ CUtensorMap tmKb,
                    const __grid_constant__ CUtensorMap tmVb, const __grid_constant__ CUtensorMap tmPre,
                    const AttnParams p) {
+  static_assert(NC == 32 || NC == 64 || NC == 128, "column count");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -335,7 +338,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // QK^T and as many 16-key steps of PV: no work on empty columns.
     auto issue_qk = [&](int jj) {
       const Tile t = tile_at(p, u, b, kvh, j0 + jj);
-      const int n16 = (t.nvalid + 15) & ~15;
+      const int n16 = min(NC, (t.nvalid + 15) & ~15);
       const uint32_t idesc = idesc_bf16_f32(BM, n16, false, false);
       const uint32_t aK = smem_u32(sRing + slot_of(2 * jj) * SLOT_BYTES);
       const uint32_t tS = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN;
@@ -350,7 +353,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t tP = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN;  // P (bf16 pairs) over S
       const int ksteps = (nvalid + 15) >> 4;
 #pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk)
+      for (int kk = 0; kk < NC / 16; ++kk)
         if (kk < ksteps)
           umma_bf16_ts(tO, tP + kk * 8, sw128_desc(aV + kk * 16 * 128, HALF_BYTES, 1024), IDESC_PV,
                        (jj > 0 || kk > 0) ? 1u : 0u);
@@ -433,20 +436,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after_sync();
       // S row of this thread.  A tail tile (fewer than BN valid keys) sets
       // the columns past its keys to -inf first; full tiles skip that block.
-      uint32_t sv[BN];
+      uint32_t sv[NC];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
+      for (int c = 0; c < NC / 32; ++c)
         tmem_ld_32x32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[c * 32]));
       tmem_ld_wait();
-      if (t.nvalid < BN) {
+      if (t.nvalid < NC) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c)
+        for (int c = 0; c < NC; ++c)
           if (c >= t.nvalid) sv[c] = 0xff800000u;  // -inf
       }
       float* s = reinterpret_cast<float*>(sv);  // S, then p in place
       float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-      for (int c = 4; c < BN; c += 4) {
+      for (int c = 4; c < NC; c += 4) {
         mx0 = fmaxf(mx0, s[c]);
         mx1 = fmaxf(mx1, s[c + 1]);
         mx2 = fmaxf(mx2, s[c + 2]);
@@ -459,7 +462,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const float m_use = (m_new == -CUDART_INF_F) ? 0.f : m_new;
       float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
 #pragma unroll
-      for (int c = 0; c < BN; c += 4) {
+      for (int c = 0; c < NC; c += 4) {
         s[c] = ex2_approx(fmaf(s[c], c2, -m_use));
         s[c + 1] = ex2_approx(fmaf(s[c + 1], c2, -m_use));
         s[c + 2] = ex2_approx(fmaf(s[c + 2], c2, -m_use));
@@ -492,12 +495,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       // P as bf16 pairs over the first 64 columns of this S buffer: the
       // A operand of PV, read from tensor memory.
+      if (NC >= 64) {
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) {
-        uint32_t pk[32];
+        for (int c = 0; c < NC / 64; ++c) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[c * 64 + 2 * i], s[c * 64 + 2 * i + 1]);
-        tmem_st_32x32(tS + c * 32, pk);
+          for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[c * 64 + 2 * i], s[c * 64 + 2 * i + 1]);
+          tmem_st_32x32(tS + c * 32, pk);
+        }
+      } else {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
+        tmem_st_32x16(tS, pk);
       }
       tmem_st_wait();
       tc_fence_before_sync();
@@ -514,30 +524,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const bool empty = (nt == 0) || !(l_run > 0.f);
     const float inv_l = empty ? 0.f : 1.f / l_run;
     const float lse2 = empty ? -CUDART_INF_F : m_run + log2f(l_run);  // log2 of Z
+    // the whole accumulator row in one batch of TMEM loads
+    uint32_t ov[HD];
+    if (nt > 0) {
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c)
+        tmem_ld_32x32(tO + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[c * 32]));
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int i = 0; i < HD; ++i) ov[i] = 0u;
+    }
     if (EPI == EPI_PARTIAL) {
       const size_t orow = (((size_t)split * p.B + b) * p.S + tok) * p.Hq + h;
       float* dst = p.out_o32 + orow * HD;
+      if (row_ok) {
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t ov[32];
-        if (nt > 0) {
-          tmem_ld_32x32(tO + c * 32, ov);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = 0u;
+        for (int i = 0; i < HD; i += 4) {
+          const float4 v = make_float4(__uint_as_float(ov[i]) * inv_l, __uint_as_float(ov[i + 1]) * inv_l,
+                                       __uint_as_float(ov[i + 2]) * inv_l, __uint_as_float(ov[i + 3]) * inv_l);
+          *reinterpret_cast<float4*>(dst + i) = v;
         }
-        if (row_ok) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            float4 v = make_float4(__uint_as_float(ov[i]) * inv_l, __uint_as_float(ov[i + 1]) * inv_l,
-                                   __uint_as_float(ov[i + 2]) * inv_l, __uint_as_float(ov[i + 3]) * inv_l);
-            *reinterpret_cast<float4*>(dst + c * 32 + i) = v;
-          }
-        }
-      }
-      if (row_ok)
         p.out_lse[(((size_t)split * p.B + b) * p.Hq + h) * p.S + tok] = lse2 * LN2;
+      }
     } else {
       const size_t orow = ((size_t)b * p.S + tok) * p.Hq + h;
       float wp = 0.f, wo = inv_l, inv_den = 1.f, lse_out2 = lse2;
@@ -555,15 +564,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out_o) + orow * HD;
       const float* pre = (EPI == EPI_MERGE) ? p.pre_o + orow * HD : nullptr;
+      if (row_ok) {
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld_32x32(tO + c * 32, ov);
-        tmem_ld_wait();
-        if (row_ok) {
+        for (int c = 0; c < HD / 32; ++c) {
           float o[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(ov[i]) * wo;
+          for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(ov[c * 32 + i]) * wo;
           if (EPI == EPI_MERGE) {
             const uint8_t* prow = sRing + PRE_SLOT * SLOT_BYTES + c * (BM * 128) + r * 128;
 #pragma unroll
@@ -583,8 +589,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             *reinterpret_cast<uint4*>(dst + c * 32 + i) = v;
           }
         }
+        if (p.out_lse) p.out_lse[((size_t)b * p.Hq + h) * p.S + tok] = lse_out2 * LN2;
       }
-      if (row_ok && p.out_lse) p.out_lse[((size_t)b * p.Hq + h) * p.S + tok] = lse_out2 * LN2;
     }
   }
 
@@ -601,7 +607,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 // read the splits' LSEs in parallel, the split weights go to shared memory,
 // then each lane accumulates four output columns over the splits.
 constexpr int CMB_WARPS = 4;
-constexpr int CMB_INFLIGHT = 16;  // split loads in flight per lane
+constexpr int CMB_INFLIGHT = 16;  // split loads in flight per lane (divides 32)
+static_assert(TC_MAX_SPLITS == 128, "combine holds four split weights per lane");
 
 __device__ __forceinline__ float warp_max_f(float v) {
 #pragma unroll
@@ -615,7 +622,6 @@ __device__ __forceinline__ float warp_sum_f(float v) {
 }
 
 __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombineParams c) {
-  __shared__ float wsm[CMB_WARPS][TC_MAX_SPLITS];
   pdl_wait();
   pdl_launch_dependents();
   const int wi = threadIdx.x >> 5;
@@ -630,19 +636,25 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombinePa
   const size_t so = (size_t)nrows * c.D;              // split stride of the partial O
   const size_t sl = (size_t)c.B * c.Hq * c.S;         // split stride of the partial LSE
   const size_t lrow = ((size_t)b * c.Hq + h) * c.S + t;
+  // lane l holds the LSE (then the weight) of splits l, l + 32, l + 64, l + 96
+  constexpr int PER_LANE = TC_MAX_SPLITS / 32;
+  float wreg[PER_LANE];
   float M = -CUDART_INF_F;
-  for (int s = lane; s < c.nsplit; s += 32) M = fmaxf(M, c.part_lse[s * sl + lrow]);
+#pragma unroll
+  for (int k = 0; k < PER_LANE; ++k) {
+    const int s = lane + 32 * k;
+    wreg[k] = s < c.nsplit ? c.part_lse[s * sl + lrow] : -CUDART_INF_F;
+    M = fmaxf(M, wreg[k]);
+  }
   M = warp_max_f(M);
   const bool empty = (M == -CUDART_INF_F);
   float den = 0.f;
-  for (int s = lane; s < c.nsplit; s += 32) {
-    const float ls = c.part_lse[s * sl + lrow];
-    const float w = (empty || ls == -CUDART_INF_F) ? 0.f : expf(ls - M);
-    wsm[wi][s] = w;
-    den += w;
+#pragma unroll
+  for (int k = 0; k < PER_LANE; ++k) {
+    wreg[k] = (empty || wreg[k] == -CUDART_INF_F) ? 0.f : expf(wreg[k] - M);
+    den += wreg[k];
   }
   den = warp_sum_f(den);
-  __syncwarp();
   const float inv = den > 0.f ? 1.f / den : 0.f;
   const float* base = c.part_o + row * c.D;
   for (int d0 = lane * 4; d0 < c.D; d0 += 128) {
@@ -654,10 +666,12 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombinePa
 #pragma unroll
       for (int i = 0; i < CMB_INFLIGHT; ++i)
         if (s0 + i < c.nsplit) v[i] = __ldg(reinterpret_cast<const float4*>(base + (s0 + i) * so + d0));
+      const int k = s0 >> 5;  // the same for the whole batch (CMB_INFLIGHT divides 32)
+      const float wk = k == 0 ? wreg[0] : k == 1 ? wreg[1] : k == 2 ? wreg[2] : wreg[3];
 #pragma unroll
       for (int i = 0; i < CMB_INFLIGHT; ++i) {
+        const float w = __shfl_sync(0xffffffffu, wk, (s0 + i) & 31);
         if (s0 + i < c.nsplit) {
-          const float w = wsm[wi][s0 + i];
           acc.x = fmaf(w, v[i].x, acc.x);
           acc.y = fmaf(w, v[i].y, acc.y);
           acc.z = fmaf(w, v[i].z, acc.z);
@@ -691,17 +705,27 @@ cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CU
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static bool configured[64][3] = {};
+  // short in-block steps run the 32- or 64-column instantiation
+  const bool short_block = (p.epi == EPI_MERGE) && !p.src.has_prefix;
+  const int nc = (short_block && p.S <= 32) ? 32 : (short_block && p.S <= 64) ? 64 : 128;
+  int which;
   void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, AttnParams);
-  switch (p.epi) {
-    case EPI_PARTIAL: kern = attn_tc_kernel<EPI_PARTIAL>; break;
-    case EPI_MERGE: kern = attn_tc_kernel<EPI_MERGE>; break;
-    default: kern = attn_tc_kernel<EPI_NORM>; break;
+  if (p.epi == EPI_PARTIAL) {
+    kern = attn_tc_kernel<EPI_PARTIAL, 128>;
+    which = 0;
+  } else if (p.epi == EPI_MERGE) {
+    kern = nc == 32 ? attn_tc_kernel<EPI_MERGE, 32> : nc == 64 ? attn_tc_kernel<EPI_MERGE, 64>
+                                                               : attn_tc_kernel<EPI_MERGE, 128>;
+    which = nc == 32 ? 1 : nc == 64 ? 2 : 3;
+  } else {
+    kern = attn_tc_kernel<EPI_NORM, 128>;
+    which = 4;
   }
-  if (dev < 64 && !configured[dev][p.epi]) {
+  static bool configured[64][5] = {};
+  if (dev < 64 && !configured[dev][which]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    configured[dev][p.epi] = true;
+    configured[dev][which] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);

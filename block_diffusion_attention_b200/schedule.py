@@ -135,6 +135,57 @@ class CachedBlockAttention:
             if c1 > c0:
                 self.update_chunk_means(c0, c1)
 
+    # ------------------------------------------------------------ graphs
+    def run_block(self, steps, outs, refresh_steps, append_kv=None, advance=True, cached=True):
+        """Issue one block of denoising steps: ``steps`` is a list of (Q, Kblk,
+        Vblk) device tensors, ``outs`` the per-step outputs.  Cached: refresh at
+        ``refresh_steps``, fused step everywhere; uncached: full attention at
+        every step.  Ends with the append of ``append_kv`` when given."""
+        for s, (Q, Kb, Vb) in enumerate(steps):
+            if cached:
+                if s in refresh_steps:
+                    self.refresh(Q)
+                self.step(Q, Kb, Vb, out=outs[s])
+            else:
+                self.full(Q, Kb, Vb, out=outs[s])
+        if append_kv is not None:
+            self.append(append_kv[0], append_kv[1], advance=advance)
+
+    def capture_block(self, steps, outs, refresh_steps, append_kv=None, cached=True, prologue=None,
+                      epilogue=None):
+        """Record one block of calls (see ``run_block``) into a CUDA graph.
+
+        The library's calls are capturable: they allocate nothing, never
+        synchronise, and pass their TMA descriptors by value.  The block runs
+        once eagerly first, so one-time kernel attribute settings happen outside
+        the capture.  The append is recorded without advancing the prefix
+        length (a replayed graph cannot update the host-side bookkeeping).
+        ``prologue``/``epilogue`` (callables) are recorded before/after each
+        step, e.g. host<->device copies.  Returns the ``torch.cuda.CUDAGraph``.
+        """
+        def body():
+            for s, (Q, Kb, Vb) in enumerate(steps):
+                if prologue is not None:
+                    prologue(s)
+                if cached:
+                    if s in refresh_steps:
+                        self.refresh(Q)
+                    self.step(Q, Kb, Vb, out=outs[s])
+                else:
+                    self.full(Q, Kb, Vb, out=outs[s])
+                if epilogue is not None:
+                    epilogue(s)
+            if append_kv is not None:
+                self.append(append_kv[0], append_kv[1], advance=False)
+
+        body()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            body()
+        torch.cuda.synchronize()
+        return g
+
     def check(self) -> None:
         """Synchronise and raise if a kernel recorded a device-side error."""
         torch.cuda.current_stream().synchronize()
