@@ -148,8 +148,10 @@ AttnParams base_params(const fb_desc& d) {
   return p;
 }
 
-// Key-range splits of the prefix pass: enough CTAs to fill the GPU once, at
-// least 4 key tiles per split.
+// Key-range splits of the prefix pass.  Cost model in key-tile times: every
+// wave of CTAs costs its longest split plus a fixed per-CTA overhead (set-up,
+// pipeline fill, epilogue ~ 3 tiles), and splitting adds a combine pass
+// (~ 2 tiles).  Splits keep at least 4 tiles each.
 int choose_splits(const fb_desc& d, long long est_tiles) {
   if (d.dtype != FB_BF16) return 1;
   const int G = d.num_q_heads / d.num_kv_heads;
@@ -160,22 +162,18 @@ int choose_splits(const fb_desc& d, long long est_tiles) {
   if (d.num_splits > 0)
     return (int)std::min<long long>(std::min<long long>(d.num_splits, TC_MAX_SPLITS), std::max<long long>(est_tiles, 1));
   const long long slots = device_sms();
-  if (units >= slots) {
-    int best = 1;
-    double best_eff = 0;
-    for (int ns = 1; ns <= 4 && ns <= max_ns; ++ns) {
-      const double w = (double)(units * ns) / (double)slots;
-      const double eff = w / std::ceil(w);
-      if (eff > best_eff + 0.05) {
-        best_eff = eff;
-        best = ns;
-      }
+  int best = 1;
+  double best_cost = 1e30;
+  for (long long ns = 1; ns <= max_ns; ++ns) {
+    const long long waves = (units * ns + slots - 1) / slots;
+    const double per_split = std::ceil((double)est_tiles / (double)ns);
+    const double cost = (double)waves * (per_split + 3.0) + (ns > 1 ? 2.0 : 0.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = (int)ns;
     }
-    return best;
   }
-  long long ns = slots / units;
-  if (ns > max_ns) ns = max_ns;
-  return (int)std::max<long long>(ns, 1);
+  return best;
 }
 
 long long prefix_tiles_estimate(const fb_desc& d) {

@@ -447,31 +447,39 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (c >= t.nvalid) sv[c] = 0xff800000u;  // -inf
       }
       float* s = reinterpret_cast<float*>(sv);  // S, then p in place
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+      float mx0 = fmax3(s[0], s[1], s[2]), mx1 = fmax3(s[3], s[4], s[5]);
 #pragma unroll
-      for (int c = 4; c < NC; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
+      for (int c = 6; c + 4 <= NC; c += 4) {
+        mx0 = fmax3(mx0, s[c], s[c + 1]);
+        mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
       }
-      const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c2;
+      // NC - 6 is a multiple of 4 plus 2: the last two columns
+      mx0 = fmax3(mx0, mx1, fmaxf(s[NC - 2], s[NC - 1]));
+      const float mt = mx0 * c2;
       const bool need = mt > m_run + RESCALE_LOG2;
       const float m_new = need ? mt : m_run;
       const float alpha = ex2_approx(m_run - m_new);  // 0 when m_run = -inf
       const float m_use = (m_new == -CUDART_INF_F) ? 0.f : m_new;
-      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+      // p = 2^(s * c2 - m): packed FMA for the argument; three of every four
+      // pairs through MUFU.EX2, one through the FMA-pipe polynomial
+      const float2 c2v = make_float2(c2, c2), mv = make_float2(-m_use, -m_use);
+      float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < NC; c += 4) {
-        s[c] = ex2_approx(fmaf(s[c], c2, -m_use));
-        s[c + 1] = ex2_approx(fmaf(s[c + 1], c2, -m_use));
-        s[c + 2] = ex2_approx(fmaf(s[c + 2], c2, -m_use));
-        s[c + 3] = ex2_approx(fmaf(s[c + 3], c2, -m_use));
-        l0 += s[c];
-        l1 += s[c + 1];
-        l2 += s[c + 2];
-        l3 += s[c + 3];
+      for (int c = 0; c < NC; c += 8) {
+        float2 x0 = ffma2(make_float2(s[c], s[c + 1]), c2v, mv);
+        float2 x1 = ffma2(make_float2(s[c + 2], s[c + 3]), c2v, mv);
+        float2 x2 = ffma2(make_float2(s[c + 4], s[c + 5]), c2v, mv);
+        float2 x3 = ffma2(make_float2(s[c + 6], s[c + 7]), c2v, mv);
+        x0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+        x1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+        x2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
+        x3 = exp2_poly2(x3);
+        s[c] = x0.x; s[c + 1] = x0.y; s[c + 2] = x1.x; s[c + 3] = x1.y;
+        s[c + 4] = x2.x; s[c + 5] = x2.y; s[c + 6] = x3.x; s[c + 7] = x3.y;
+        la = fadd2(la, fadd2(x0, x1));
+        lb = fadd2(lb, fadd2(x2, x3));
       }
+      const float l0 = la.x, l1 = la.y, l2 = lb.x, l3 = lb.y;
       l_run = l_run * alpha + ((l0 + l1) + (l2 + l3));
       m_run = m_new;
 

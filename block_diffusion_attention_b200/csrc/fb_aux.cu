@@ -90,18 +90,23 @@ __global__ void chunk_means_kernel(const CacheGeom g, const int32_t* lens, int c
   Kmean[(((size_t)b * g.Hkv + kvh) * nch_total + c) * g.D + d] = mean;
 }
 
-// grid (Hkv, B), block 256.  Dynamic shared memory: D + nch floats + nch flags.
+// grid (Hkv, B), block SEL_THREADS.  Dynamic shared memory:
+// (SEL_WARPS + 1) * D floats for the query mean, nch scores, nch flags.
+constexpr int SEL_WARPS = 8, SEL_THREADS = SEL_WARPS * 32;
+
 template <typename T>
-__global__ void select_chunks_kernel(const CacheGeom g, const int32_t* lens, int chunk_size,
-                                     int nch_total, int S, int Hq, int topk,
-                                     const T* __restrict__ Q, const float* __restrict__ Kmean,
-                                     int32_t* __restrict__ idx, int32_t* status) {
+__global__ void __launch_bounds__(SEL_THREADS)
+    select_chunks_kernel(const CacheGeom g, const int32_t* lens, int chunk_size, int nch_total, int S, int Hq,
+                         int topk, const T* __restrict__ Q, const float* __restrict__ Kmean,
+                         int32_t* __restrict__ idx, int32_t* status) {
   extern __shared__ float sm[];
   const int kvh = blockIdx.x;
   const int b = blockIdx.y;
   const int G = Hq / g.Hkv;
-  float* qbar = sm;
-  float* score = sm + g.D;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* part = sm;                       // [SEL_WARPS][D] per-warp row sums
+  float* qbar = sm + SEL_WARPS * g.D;     // [D]
+  float* score = qbar + g.D;              // [nch_total]
   int* sel = reinterpret_cast<int*>(score + nch_total);
   int L = lens[b];
   if (L < 0 || L > g.cap) {
@@ -109,23 +114,36 @@ __global__ void select_chunks_kernel(const CacheGeom g, const int32_t* lens, int
     L = max(0, min(L, g.cap));
   }
   const int nch = (L + chunk_size - 1) / chunk_size;
-  for (int d = threadIdx.x; d < g.D; d += blockDim.x) {
+  // query mean over the S block tokens and the G heads of the group: warp w
+  // sums rows w, w + SEL_WARPS, ...; lanes cover the D columns
+  const int rows = S * G;
+  for (int d = lane; d < g.D; d += 32) {
     float acc = 0.f;
-    for (int t = 0; t < S; ++t)
-      for (int gg = 0; gg < G; ++gg)
-        acc += to_f<T>(Q[(((size_t)b * S + t) * Hq + kvh * G + gg) * g.D + d]);
-    qbar[d] = acc / (float)(S * G);
+    for (int rr = warp; rr < rows; rr += SEL_WARPS) {
+      const int t = rr / G, gg = rr - (rr / G) * G;
+      acc += to_f<T>(Q[(((size_t)b * S + t) * Hq + kvh * G + gg) * g.D + d]);
+    }
+    part[warp * g.D + d] = acc;
   }
   __syncthreads();
-  const float* km = Kmean + ((size_t)b * g.Hkv + kvh) * nch_total * g.D;
-  for (int c = threadIdx.x; c < nch; c += blockDim.x) {
+  for (int d = threadIdx.x; d < g.D; d += SEL_THREADS) {
     float acc = 0.f;
-    for (int d = 0; d < g.D; ++d) acc = fmaf(qbar[d], km[(size_t)c * g.D + d], acc);
-    score[c] = acc;
+    for (int w2 = 0; w2 < SEL_WARPS; ++w2) acc += part[w2 * g.D + d];
+    qbar[d] = acc / (float)rows;
+  }
+  __syncthreads();
+  // score of chunk c: one warp per chunk, lanes over D, shuffle reduction
+  const float* km = Kmean + ((size_t)b * g.Hkv + kvh) * nch_total * g.D;
+  for (int c = warp; c < nch; c += SEL_WARPS) {
+    float acc = 0.f;
+    for (int d = lane; d < g.D; d += 32) acc = fmaf(qbar[d], km[(size_t)c * g.D + d], acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) score[c] = acc;
   }
   __syncthreads();
   // rank = chunks that beat c (higher score, or equal score and lower index)
-  for (int c = threadIdx.x; c < nch; c += blockDim.x) {
+  for (int c = threadIdx.x; c < nch; c += SEL_THREADS) {
     const float sc = score[c];
     int better = 0;
     for (int c2 = 0; c2 < nch; ++c2) {
@@ -135,13 +153,17 @@ __global__ void select_chunks_kernel(const CacheGeom g, const int32_t* lens, int
     sel[c] = better < topk;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int32_t* out = idx + ((size_t)b * g.Hkv + kvh) * topk;
-    int n = 0;
-    for (int c = 0; c < nch && n < topk; ++c)
-      if (sel[c]) out[n++] = c;
-    for (; n < topk; ++n) out[n] = -1;
+  // ascending chunk order: output slot = selected chunks before c
+  int32_t* out = idx + ((size_t)b * g.Hkv + kvh) * topk;
+  for (int c = threadIdx.x; c < nch; c += SEL_THREADS) {
+    if (sel[c]) {
+      int before = 0;
+      for (int c2 = 0; c2 < c; ++c2) before += sel[c2];
+      out[before] = c;
+    }
   }
+  const int nsel = min(topk, nch);
+  for (int i = nsel + threadIdx.x; i < topk; i += SEL_THREADS) out[i] = -1;
 }
 
 // One thread per 16-byte vector of the block's K and V.
@@ -207,18 +229,20 @@ cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* K
                                  int32_t* status, cudaStream_t stream) {
   const CacheGeom g = geom_of(d);
   const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
-  const size_t smem = (size_t)(g.D + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int);
+  const size_t smem = (size_t)((SEL_WARPS + 1) * g.D + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int);
   dim3 grid(g.Hkv, g.B);
   if (d.dtype == FB_BF16) {
     auto k = select_chunks_kernel<__nv_bfloat16>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, 256, smem, stream>>>(g, d.prefix_lens, d.chunk_size, nch_total, d.block_len, d.num_q_heads,
-                                   d.topk, static_cast<const __nv_bfloat16*>(Q), Kmean, idx, status);
+    k<<<grid, SEL_THREADS, smem, stream>>>(g, d.prefix_lens, d.chunk_size, nch_total, d.block_len,
+                                           d.num_q_heads, d.topk, static_cast<const __nv_bfloat16*>(Q), Kmean,
+                                           idx, status);
   } else {
     auto k = select_chunks_kernel<float>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, 256, smem, stream>>>(g, d.prefix_lens, d.chunk_size, nch_total, d.block_len, d.num_q_heads,
-                                   d.topk, static_cast<const float*>(Q), Kmean, idx, status);
+    k<<<grid, SEL_THREADS, smem, stream>>>(g, d.prefix_lens, d.chunk_size, nch_total, d.block_len,
+                                           d.num_q_heads, d.topk, static_cast<const float*>(Q), Kmean, idx,
+                                           status);
   }
   note_launch();
   return cudaGetLastError();
