@@ -52,12 +52,13 @@ constexpr uint32_t HALF_BYTES = BN * 128;       // one 64-column half of a tile
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_RING = OFF_Q + Q_BYTES;
 constexpr uint32_t OFF_BAR = OFF_RING + NSLOT * SLOT_BYTES;
-constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 + 2 + 3;
+constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 + 2 + 4;
 constexpr uint32_t PRE_BYTES = BM * HD * 4;      // 64 KB: O_pre rows of a tile (f32)
 constexpr int PRE_SLOT = NSLOT - 2;             // O_pre prefetch uses the last two ring slots
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_S0 = 0, TMEM_O = 256;           // S buffers at 0 and 128
+constexpr uint32_t TMEM_Q = 384;                        // Q (bf16 pairs), 64 columns
 constexpr float RESCALE_LOG2 = 8.0f;   // rescale O only when the row max grows by > 2^8
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 constexpr float LN2 = 0.6931471805599453f;
@@ -74,6 +75,7 @@ struct Shared {
   uint64_t* o_done;  // PV finished
   uint64_t* drain;
   uint64_t* pre_full; // O_pre rows prefetched (merge epilogue of short units)
+  uint64_t* q_tmem;   // Q copied into tensor memory by the softmax warps
   uint32_t* tmem_slot;
   volatile int* abort_flag;
 };
@@ -83,8 +85,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const S
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
+    // each try sleeps until the phase completes or 1 ms passes
     if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 63u) == 0) {
+    {
       if (honour_abort && *sh.abort_flag) return false;
       if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
         *sh.abort_flag = 1;
@@ -233,7 +236,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   sh.o_done = sh.p_full + 2;
   sh.drain = sh.o_done + 1;
   sh.pre_full = sh.drain + 1;
-  sh.tmem_slot = reinterpret_cast<uint32_t*>(sh.pre_full + 1);
+  sh.q_tmem = sh.pre_full + 1;
+  sh.tmem_slot = reinterpret_cast<uint32_t*>(sh.q_tmem + 1);
   sh.abort_flag = reinterpret_cast<volatile int*>(sh.tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -260,6 +264,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     mbar_init(sh.o_done, 1);
     mbar_init(sh.drain, 1);
     mbar_init(sh.pre_full, 1);
+    mbar_init(sh.q_tmem, 4);
     *sh.abort_flag = 0;
     fence_barrier_init();
   }
@@ -332,39 +337,43 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   } else if (warp == 5) {
     // --------------------------------------------------------------- MMA issuer
     constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, HD, false, true);
+    constexpr uint32_t IDESC_QK_FULL = idesc_bf16_f32(BM, NC, false, false);
     const uint32_t tO = tmem + TMEM_O;
-    const uint32_t aQ = smem_u32(sQ);
+    // Shared-memory descriptors: built once; an operand at byte offset `off`
+    // from its base is the base descriptor plus off >> 4 (start-address field).
+    const uint64_t dK = sw128_desc(smem_u32(sRing), 16, 1024);
+    const uint64_t dV = sw128_desc(smem_u32(sRing), HALF_BYTES, 1024);
     // A tile with fewer valid keys runs N = (valid keys rounded up to 16) for
     // QK^T and as many 16-key steps of PV: no work on empty columns.
-    auto issue_qk = [&](int jj) {
-      const Tile t = tile_at(p, u, b, kvh, j0 + jj);
-      const int n16 = min(NC, (t.nvalid + 15) & ~15);
-      const uint32_t idesc = idesc_bf16_f32(BM, n16, false, false);
-      const uint32_t aK = smem_u32(sRing + slot_of(2 * jj) * SLOT_BYTES);
+    auto issue_qk = [&](int jj, int nvalid) {
+      const uint32_t idesc =
+          nvalid >= NC ? IDESC_QK_FULL : idesc_bf16_f32(BM, min(NC, (nvalid + 15) & ~15), false, false);
+      const uint64_t dk = dK + ((slot_of(2 * jj) * SLOT_BYTES) >> 4);
       const uint32_t tS = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN;
+      // A = Q from tensor memory (16 dims = 8 packed columns per step), B = K
+      // from shared memory: only K crosses the shared-memory read port
 #pragma unroll
       for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-        umma_bf16_ss(tS, sw128_desc(aQ + off, 16, 1024), sw128_desc(aK + off, 16, 1024), idesc, kk > 0);
+        const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+        umma_bf16_ts(tS, tmem + TMEM_Q + kk * 8, dk + off, idesc, kk > 0);
       }
     };
     auto issue_pv = [&](int jj, int nvalid) {
-      const uint32_t aV = smem_u32(sRing + slot_of(2 * jj + 1) * SLOT_BYTES);
+      const uint64_t dv = dV + ((slot_of(2 * jj + 1) * SLOT_BYTES) >> 4);
       const uint32_t tP = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN;  // P (bf16 pairs) over S
       const int ksteps = (nvalid + 15) >> 4;
 #pragma unroll
       for (int kk = 0; kk < NC / 16; ++kk)
         if (kk < ksteps)
-          umma_bf16_ts(tO, tP + kk * 8, sw128_desc(aV + kk * 16 * 128, HALF_BYTES, 1024), IDESC_PV,
-                       (jj > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
     };
-    bool ok = wait_bar(sh.q_full, 0, sh, status);
+    bool ok = wait_bar(sh.q_tmem, 0, sh, status);
     if (ok && nt > 0) {
       ok = wait_bar(&sh.full[slot_of(0)], 0, sh, status);
       if (ok) {
         tc_fence_after_sync();
         if (lane == 0) {
-          issue_qk(0);
+          issue_qk(0, tile_at(p, u, b, kvh, j0).nvalid);
           tc_commit(&sh.s_full[0]);
           tc_commit(&sh.empty[slot_of(0)]);
         }
@@ -376,7 +385,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (!(ok = wait_bar(&sh.full[slot_of(ik)], use_of(ik) & 1, sh, status))) break;
           tc_fence_after_sync();
           if (lane == 0) {
-            issue_qk(jj + 1);
+            issue_qk(jj + 1, tile_at(p, u, b, kvh, j0 + jj + 1).nvalid);
             tc_commit(&sh.s_full[(jj + 1) & 1]);
             tc_commit(&sh.empty[slot_of(ik)]);
           }
@@ -428,8 +437,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                                           : -CUDART_INF_F;
     float m_run = -CUDART_INF_F;
     float l_run = 0.f;
-    bool ok = true;
-    for (int jj = 0; jj < nt; ++jj) {
+    bool ok = wait_bar(sh.q_full, 0, sh, status);
+    if (ok) {
+      // this thread's Q row (128 bf16, 128-byte swizzled in two 64-dim halves)
+      // into TMEM columns [TMEM_Q, TMEM_Q + 64): the A operand of QK^T
+      const uint32_t qrow = smem_u32(sQ) + r * 128;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t qv[32];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t addr = qrow + hf * (BM * 128) + ((ch ^ (r & 7)) << 4);
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(qv[ch * 4]), "=r"(qv[ch * 4 + 1]), "=r"(qv[ch * 4 + 2]), "=r"(qv[ch * 4 + 3])
+                       : "r"(addr));
+        }
+        tmem_st_32x32(tmem + TMEM_Q + lane_off + hf * 32, qv);
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sh.q_tmem);
+    }
+    for (int jj = 0; ok && jj < nt; ++jj) {
       const uint32_t tS = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN + lane_off;
       const Tile t = tile_at(p, u, b, kvh, j0 + jj);
       if (!(ok = wait_bar(&sh.s_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
