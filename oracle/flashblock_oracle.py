@@ -20,7 +20,9 @@ Efficient Long-Context Block Diffusion" (gist.science explainer of arXiv
   are recombined with the log-space merge equation (:func:`merge_partials`).
 * §2 Methodology, Adaptive Reuse Strategies, "Compatibility with Sparse
   Attention" -- unselected sparse keys play the role of J_out
-  (:func:`select_chunks`, :func:`chunk_token_positions`).
+  (:func:`select_chunks`, :func:`chunk_token_positions`); their cached
+  residual is merged with the freshly computed selected keys
+  (:func:`complement_chunks`, :func:`residual_block`).
 
 Readings where the page is silent (each listed in the design doc):
   L is the natural log of the unnormalised sum Z; J_out is the finalized
@@ -298,6 +300,48 @@ def cached_block(Qs, Kbs, Vbs, Kc, Vc, prefix_lens, scale, refresh_steps,
     return outs, pres
 
 
+def complement_chunks(chunk_idx, valid):
+    """The valid chunks a selection leaves out: [B, Hkv, nchunks] int32,
+    ascending, padded with -1 (Compatibility with Sparse Attention: the
+    unselected keys form the block-external set whose contribution is
+    cached)."""
+    B, Hkv, _ = chunk_idx.shape
+    nch = valid.shape[1]
+    comp = np.full((B, Hkv, nch), -1, dtype=np.int32)
+    for b in range(B):
+        for kvh in range(Hkv):
+            chosen = set(int(c) for c in chunk_idx[b, kvh] if c >= 0)
+            rest = [c for c in range(nch) if valid[b, c] and c not in chosen]
+            comp[b, kvh, :len(rest)] = rest
+    return comp
+
+
+def residual_block(Qs, Kbs, Vbs, Kc, Vc, prefix_lens, scale, refresh_steps, topk, chunk_size=256):
+    """One block with sparse attention and residual reuse (Adaptive Reuse
+    Strategies, Compatibility with Sparse Attention).
+
+    At a refresh step the top-k chunks are selected with that step's queries
+    and the partial over the *unselected* chunks (the residual) is computed
+    and cached.  Every step recomputes the partial over the selected chunks
+    with its own queries and merges three partials: residual, selected and
+    in-block.  Returns the list of O_s.
+    """
+    outs = []
+    res = idx = None
+    Km, valid = chunk_means(Kc, prefix_lens, chunk_size)
+    for s, Q in enumerate(Qs):
+        if s in refresh_steps or res is None:
+            idx = select_chunks(Q, Km, valid, topk)
+            comp = complement_chunks(idx, valid)
+            res = prefix_partial(Q, Kc, Vc, prefix_lens, scale, comp, chunk_size)
+        sel = prefix_partial(Q, Kc, Vc, prefix_lens, scale, idx, chunk_size)
+        o_pre, l_pre = merge_partials(res[0], np.transpose(res[1], (0, 2, 1)),
+                                      sel[0], np.transpose(sel[1], (0, 2, 1)))
+        o, _ = block_step(Q, Kbs[s], Vbs[s], o_pre, np.transpose(l_pre, (0, 2, 1)), scale)
+        outs.append(o)
+    return outs
+
+
 def attention_weights(q, k, scale):
     """Explicit softmax weight matrix e^{z - L} of one partial ([R, N])."""
     _, lse = attention_partial(q, k, np.zeros((k.shape[0], 1)), scale)
@@ -309,5 +353,5 @@ __all__ = [
     "NEG_INF", "attention_partial", "merge_partials", "chunk_token_positions",
     "prefix_partial", "inblock_partial", "block_step", "full_attention",
     "chunk_means", "chunk_scores", "select_chunks", "cached_block",
-    "attention_weights",
+    "complement_chunks", "residual_block", "attention_weights",
 ]

@@ -281,6 +281,47 @@ def pin_sparse(ora):
     _close(Lm.transpose(0, 2, 1), Ld, 1e-12, "selection + complement == dense LSE")
 
 
+def pin_residual_reuse(ora):
+    """Residual reuse with sparse attention: at a refresh step the residual +
+    selected + in-block merge equals full attention; with queries held fixed
+    every step does; with drifting queries the reuse steps differ."""
+    rng = np.random.default_rng(21)
+    B, S, Hq, Hkv, D, Lcap, chunk = 2, 3, 4, 2, 4, 45, 8
+    Kc, Vc = _rand(rng, B, Lcap, Hkv, D), _rand(rng, B, Lcap, Hkv, D)
+    lens = np.array([45, 30], dtype=np.int32)
+    Kbs = [_rand(rng, B, S, Hkv, D) for _ in range(3)]
+    Vbs = [_rand(rng, B, S, Hkv, D) for _ in range(3)]
+    Qfix = _rand(rng, B, S, Hq, D)
+    outs = ora.residual_block([Qfix] * 3, Kbs, Vbs, Kc, Vc, lens, 0.7, (0,), 2, chunk)
+    for s in range(3):
+        Of, _ = ora.full_attention(Qfix, Kc, Vc, lens, Kbs[s], Vbs[s], 0.7)
+        _close(outs[s], Of, 1e-12, f"residual reuse, fixed Q, step {s}")
+    Qs = [Qfix + 0.3 * _rand(rng, B, S, Hq, D) for _ in range(3)]
+    outs = ora.residual_block(Qs, Kbs, Vbs, Kc, Vc, lens, 0.7, (0,), 2, chunk)
+    Of, _ = ora.full_attention(Qs[0], Kc, Vc, lens, Kbs[0], Vbs[0], 0.7)
+    _close(outs[0], Of, 1e-12, "residual reuse, refresh step")
+    Of, _ = ora.full_attention(Qs[2], Kc, Vc, lens, Kbs[2], Vbs[2], 0.7)
+    assert np.max(np.abs(outs[2] - Of)) > 1e-6, "reuse steps use the stale residual"
+    # every chunk selected: no residual, so each step is exact even with drift
+    outs = ora.residual_block(Qs, Kbs, Vbs, Kc, Vc, lens, 0.7, (0,), 64, chunk)
+    for s in range(3):
+        Of, _ = ora.full_attention(Qs[s], Kc, Vc, lens, Kbs[s], Vbs[s], 0.7)
+        _close(outs[s], Of, 1e-12, f"residual reuse, all chunks selected, step {s}")
+    # nothing selected: everything is residual, i.e. the plain cached schedule
+    outs = ora.residual_block(Qs, Kbs, Vbs, Kc, Vc, lens, 0.7, (0,), 0, chunk)
+    cached, _ = ora.cached_block(Qs, Kbs, Vbs, Kc, Vc, lens, 0.7, (0,))
+    for s in range(3):
+        _close(outs[s], cached[s], 1e-12, f"residual reuse, no chunk selected, step {s}")
+    # the complement of a selection covers every other valid chunk exactly once
+    Km, valid = ora.chunk_means(Kc, lens, chunk)
+    idx = ora.select_chunks(Qfix, Km, valid, 2)
+    comp = ora.complement_chunks(idx, valid)
+    for b in range(B):
+        for kv in range(Hkv):
+            a = sorted([int(c) for c in idx[b, kv] if c >= 0] + [int(c) for c in comp[b, kv] if c >= 0])
+            assert a == [c for c in range(valid.shape[1]) if valid[b, c]], "selection + complement"
+
+
 def pin_selection_ties(ora):
     """Equal scores: the lower chunk index wins."""
     D = 2
@@ -298,7 +339,7 @@ def pin_selection_ties(ora):
 ALL_PINS = [pin_brute_partial, pin_brute_layer, pin_golden, pin_closed_forms,
             pin_merge_is_concat, pin_merge_algebra, pin_refresh_step_exact,
             pin_reuse_unchanged_queries, pin_refresh_recomputes, pin_rows_sum_to_one, pin_sparse,
-            pin_selection_ties]
+            pin_residual_reuse, pin_selection_ties]
 
 
 def failing_pins(ora):

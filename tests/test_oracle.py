@@ -39,6 +39,9 @@ MUTANTS = {
     "inblock_gqa": ("Vb[b, :, h // G, :], scale)", "Vb[b, :, h % Vb.shape[2], :], scale)"),
     "prefix_len_off_by_one": ("pos = np.arange(L)", "pos = np.arange(max(L - 1, 0))"),
     "reuse_never_refresh": ("if s in refresh_steps or pre is None:", "if pre is None:"),
+    "residual_stale_selected": ("sel = prefix_partial(Q, Kc, Vc, prefix_lens, scale, idx, chunk_size)",
+                                "sel = prefix_partial(Qs[0], Kc, Vc, prefix_lens, scale, idx, chunk_size)"),
+    "complement_drops_last": ("comp[b, kvh, :len(rest)] = rest", "comp[b, kvh, :len(rest) - 1] = rest[:-1]"),
 }
 
 
