@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--workload", default="long_ctx")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--residual", action="store_true",
+                    help="sparse workloads: residual reuse (cache the unselected chunks, recompute the selected ones)")
     ap.add_argument("--no-graph", action="store_true",
                     help="issue every call from the host instead of replaying one CUDA graph per block")
     ap.add_argument("--phases", default="cached,uncached,e2e",
@@ -78,10 +80,13 @@ def workload_config(w, extra=None):
     return cfg
 
 
-def prefix_bytes(w, lens):
-    """Algorithmic bytes of one prefix pass: K+V of the valid (or selected)
-    prefix rows, Q, and the written O_pre (f32) and LSE_pre (f32)."""
-    if w.topk:
+def prefix_bytes(w, lens, residual=False):
+    """Algorithmic bytes of one prefix pass: K+V of the valid (or selected,
+    or -- residual mode -- unselected) prefix rows, Q, and the written O_pre
+    (f32) and LSE_pre (f32)."""
+    if w.topk and residual:
+        eff = sum(int(L) - min(int(L), w.topk * w.chunk_size) for L in lens)
+    elif w.topk:
         eff = sum(min(int(L), w.topk * w.chunk_size) for L in lens)
     else:
         eff = sum(int(L) for L in lens)
@@ -90,8 +95,11 @@ def prefix_bytes(w, lens):
     return kv + rows * w.head_dim * 2 + rows * w.head_dim * 4 + rows * 4
 
 
-def prefix_flops(w, lens):
-    eff = sum(min(int(L), w.topk * w.chunk_size) if w.topk else int(L) for L in lens)
+def prefix_flops(w, lens, residual=False):
+    if w.topk and residual:
+        eff = sum(int(L) - min(int(L), w.topk * w.chunk_size) for L in lens)
+    else:
+        eff = sum(min(int(L), w.topk * w.chunk_size) if w.topk else int(L) for L in lens)
     return 4.0 * w.num_q_heads * w.block_len * eff * w.head_dim
 
 
@@ -288,7 +296,8 @@ def run_ours(args):
     def new_layer():
         layer = CachedBlockAttention(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_len, w.capacity,
                                      dtype=w.dtype, softmax_scale=w.softmax_scale,
-                                     chunk_size=w.chunk_size if w.topk else 0, topk=w.topk)
+                                     chunk_size=w.chunk_size if w.topk else 0, topk=w.topk,
+                                     residual=args.residual)
         layer.load_prefix(Kt, Vt, lens)
         return layer
 
@@ -485,10 +494,10 @@ def report(args, w0, w, world, res):
     pre_avg = sum(res["pre_ms"]) / len(res["pre_ms"])
     blk_avg = sum(res["blk_ms"]) / len(res["blk_ms"])
     mid = [(a + b) / 2 for a, b in zip(res["lens0"], res["lens1"])]
-    abytes = prefix_bytes(w, mid)
+    abytes = prefix_bytes(w, mid, args.residual)
     hbm_peak, tc_peak, tc_sustained, peak_kind = measured_peaks()
     achieved = abytes / (pre_avg / 1e3) / 1e9
-    pflops = prefix_flops(w, mid)
+    pflops = prefix_flops(w, mid, args.residual)
     tflops = pflops / (pre_avg / 1e3) / 1e12
     # the prefix pass is HBM-bound below the ridge point (measured bf16 peak /
     # measured copy bandwidth, ~258 flop/B) and tensor-bound above it
@@ -513,7 +522,10 @@ def report(args, w0, w, world, res):
         "warmup": args.warmup, "ms_per_step": ms_c / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded N(0,1) K/V, scaled Q, per-step drift)",
-        "config": workload_config(w0, {"prefix_rows_during_timing": [min(res["lens0"]), max(res["lens1"])]}),
+        "config": workload_config(w0, {"prefix_rows_during_timing": [min(res["lens0"]), max(res["lens1"])],
+                                       **({"sparse_mode": "residual reuse (refresh caches the unselected "
+                                                          "chunks; every step recomputes the selected ones)"}
+                                          if args.residual else {})}),
         "cached_us_per_denoise_step": ms_c * 1e3 / (args.steps * w.steps),
         "cached_eager_us_per_denoise_step": res["ms_cached_eager"] * 1e3 / (args.steps * w.steps),
         "launch_mode": "one CUDA graph per block" if res["graph"] else "eager host launches",

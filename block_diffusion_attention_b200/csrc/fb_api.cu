@@ -447,6 +447,33 @@ fb_status fb_kv_append(const fb_desc* d, const void* Kb, const void* Vb, void* K
                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
+fb_status fb_complement_chunks(const fb_desc* d, const int32_t* chunk_idx, int32_t* comp_idx,
+                               int32_t comp_cap, int32_t* dev_status, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if ((st = check_cache(d)) != FB_OK) return st;
+  if (!chunk_idx || !comp_idx || d->chunk_size <= 0 || d->topk <= 0 || comp_cap <= 0) return FB_ERR_INVALID_ARG;
+  const int64_t nch = (cache_rows(*d) + d->chunk_size - 1) / d->chunk_size;
+  if (nch > 16384) return FB_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(chunk_idx) & 3u) || (reinterpret_cast<uintptr_t>(comp_idx) & 3u))
+    return FB_ERR_ALIGNMENT;
+  return from_cuda(launch_complement_chunks(*d, chunk_idx, comp_idx, comp_cap, dev_status,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fb_status fb_merge_partials(const fb_desc* d, const float* O_a, const float* LSE_a, const float* O_b,
+                            const float* LSE_b, float* O_out, float* LSE_out, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!O_a || !LSE_a || !O_b || !LSE_b || !O_out || !LSE_out) return FB_ERR_INVALID_ARG;
+  if (d->head_dim % 4) return FB_ERR_UNSUPPORTED;
+  if (!aligned16(O_a) || !aligned16(O_b) || !aligned16(O_out) || (reinterpret_cast<uintptr_t>(LSE_a) & 3u) ||
+      (reinterpret_cast<uintptr_t>(LSE_b) & 3u) || (reinterpret_cast<uintptr_t>(LSE_out) & 3u))
+    return FB_ERR_ALIGNMENT;
+  return from_cuda(launch_merge_partials(*d, O_a, LSE_a, O_b, LSE_b, O_out, LSE_out,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char* fb_status_string(fb_status s) {
   switch (s) {
     case FB_OK: return "FB_OK";

@@ -198,6 +198,78 @@ __global__ void kv_append_kernel(const CacheGeom g, const int32_t* lens, int S,
   }
 }
 
+// grid (Hkv, B), block 32: the valid chunks that chunk_idx does not list, in
+// ascending order, padded with -1.  Shared memory: one flag per chunk.
+__global__ void complement_chunks_kernel(const CacheGeom g, const int32_t* lens, int chunk_size,
+                                         int nch_total, int topk, const int32_t* __restrict__ idx,
+                                         int32_t* __restrict__ comp, int comp_cap, int32_t* status) {
+  extern __shared__ int flag[];
+  const int kvh = blockIdx.x, b = blockIdx.y;
+  int L = lens[b];
+  if (L < 0 || L > g.cap) {
+    if (threadIdx.x == 0) report(status, FB_ERR_BOUNDS);
+    L = max(0, min(L, g.cap));
+  }
+  const int nch = (L + chunk_size - 1) / chunk_size;
+  for (int c = threadIdx.x; c < nch; c += blockDim.x) flag[c] = 0;
+  __syncwarp();
+  const int32_t* sel = idx + ((size_t)b * g.Hkv + kvh) * topk;
+  for (int i = threadIdx.x; i < topk; i += blockDim.x) {
+    const int c = sel[i];
+    if (c >= 0 && c < nch) flag[c] = 1;
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    int32_t* out = comp + ((size_t)b * g.Hkv + kvh) * comp_cap;
+    int n = 0;
+    for (int c = 0; c < nch; ++c) {
+      if (flag[c]) continue;
+      if (n < comp_cap) {
+        out[n] = c;
+      } else {
+        report(status, FB_ERR_BOUNDS);
+      }
+      ++n;
+    }
+    for (; n < comp_cap; ++n) out[n] = -1;
+  }
+}
+
+// One warp per query row: the merge equation of two partials (O, LSE) with
+// m = max(L_a, L_b); rows where both are empty stay (0, -inf).
+__global__ void merge_partials_kernel(int B, int S, int Hq, int D, const float* __restrict__ Oa,
+                                      const float* __restrict__ La, const float* __restrict__ Ob,
+                                      const float* __restrict__ Lb, float* Oo, float* Lo) {
+  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const long long nrows = (long long)B * S * Hq;
+  if (row >= nrows) return;
+  const int h = (int)(row % Hq);
+  const long long bt = row / Hq;
+  const int t = (int)(bt % S);
+  const int b = (int)(bt / S);
+  const size_t lrow = ((size_t)b * Hq + h) * S + t;
+  const float la = La[lrow], lb = Lb[lrow];
+  const float m = fmaxf(la, lb);
+  const bool empty = (m == -CUDART_INF_F);
+  const float wa = (empty || la == -CUDART_INF_F) ? 0.f : expf(la - m);
+  const float wb = (empty || lb == -CUDART_INF_F) ? 0.f : expf(lb - m);
+  const float den = wa + wb;
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  for (int d = lane * 4; d < D; d += 128) {
+    const float4 a = *reinterpret_cast<const float4*>(Oa + row * D + d);
+    const float4 c = *reinterpret_cast<const float4*>(Ob + row * D + d);
+    float4 o;
+    o.x = (wa * a.x + wb * c.x) * inv;
+    o.y = (wa * a.y + wb * c.y) * inv;
+    o.z = (wa * a.z + wb * c.z) * inv;
+    o.w = (wa * a.w + wb * c.w) * inv;
+    *reinterpret_cast<float4*>(Oo + row * D + d) = o;
+  }
+  __syncwarp();
+  if (lane == 0) Lo[lrow] = empty ? -CUDART_INF_F : m + logf(den);
+}
+
 // Runs after the copy: advance each length by S when the block fitted.
 __global__ void lens_advance_kernel(int32_t* lens, int B, int S, int cap) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
@@ -244,6 +316,30 @@ cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* K
                                            d.num_q_heads, d.topk, static_cast<const float*>(Q), Kmean, idx,
                                            status);
   }
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_complement_chunks(const fb_desc& d, const int32_t* idx, int32_t* comp, int comp_cap,
+                                     int32_t* status, cudaStream_t stream) {
+  const CacheGeom g = geom_of(d);
+  const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
+  dim3 grid(g.Hkv, g.B);
+  const size_t smem = (size_t)nch_total * sizeof(int);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(complement_chunks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  complement_chunks_kernel<<<grid, 32, smem, stream>>>(
+      g, d.prefix_lens, d.chunk_size, nch_total, d.topk, idx, comp, comp_cap, status);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge_partials(const fb_desc& d, const float* Oa, const float* La, const float* Ob,
+                                  const float* Lb, float* Oo, float* Lo, cudaStream_t stream) {
+  const long long rows = (long long)d.batch * d.block_len * d.num_q_heads;
+  const int warps = 8;
+  merge_partials_kernel<<<(unsigned)((rows + warps - 1) / warps), warps * 32, 0, stream>>>(
+      d.batch, d.block_len, d.num_q_heads, d.head_dim, Oa, La, Ob, Lb, Oo, Lo);
   note_launch();
   return cudaGetLastError();
 }

@@ -85,6 +85,10 @@ cudaError_t launch_chunk_means(const fb_desc& d, const void* K, int chunk_begin,
                                float* Kmean, int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* Kmean,
                                  int32_t* idx, int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_complement_chunks(const fb_desc& d, const int32_t* idx, int32_t* comp, int comp_cap,
+                                     int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_merge_partials(const fb_desc& d, const float* Oa, const float* La, const float* Ob,
+                                  const float* Lb, float* Oo, float* Lo, cudaStream_t stream);
 cudaError_t launch_kv_append(const fb_desc& d, const void* Kb, const void* Vb, void* Kc, void* Vc,
                              int32_t* lens_inout, int32_t* dev_status, cudaStream_t stream);
 

@@ -74,6 +74,8 @@ def load() -> ctypes.CDLL:
             "fb_chunk_means": (I32, [D, P, I32, I32, P, P, P]),
             "fb_select_chunks": (I32, [D, P, P, P, P, P]),
             "fb_kv_append": (I32, [D, P, P, P, P, P, P, P]),
+            "fb_complement_chunks": (I32, [D, P, P, I32, P, P]),
+            "fb_merge_partials": (I32, [D, P, P, P, P, P, P, P]),
             "fb_status_string": (ctypes.c_char_p, [I32]),
             "fb_launch_count": (ctypes.c_uint64, []),
             "fb_abi_version": (I32, []),
@@ -177,6 +179,16 @@ def fb_kv_append(d, Kblk, Vblk, Kcache, Vcache, lens_inout, dev_status, stream=N
     _ok("fb_kv_append", load().fb_kv_append(
         ctypes.byref(d), _p(Kblk), _p(Vblk), _p(Kcache), _p(Vcache), _p(lens_inout), _p(dev_status),
         _s(stream)))
+
+
+def fb_complement_chunks(d, chunk_idx, comp_idx, comp_cap, dev_status, stream=None):
+    _ok("fb_complement_chunks", load().fb_complement_chunks(
+        ctypes.byref(d), _p(chunk_idx), _p(comp_idx), int(comp_cap), _p(dev_status), _s(stream)))
+
+
+def fb_merge_partials(d, O_a, LSE_a, O_b, LSE_b, O_out, LSE_out, stream=None):
+    _ok("fb_merge_partials", load().fb_merge_partials(
+        ctypes.byref(d), _p(O_a), _p(LSE_a), _p(O_b), _p(LSE_b), _p(O_out), _p(LSE_out), _s(stream)))
 
 
 def fb_status_string(status: int) -> str:

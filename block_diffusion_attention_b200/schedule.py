@@ -26,7 +26,8 @@ class CachedBlockAttention:
     def __init__(self, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, block_len: int,
                  capacity: int, dtype: str = "bf16", softmax_scale: float = 1.0, page_size: int = 0,
                  block_table: Optional[torch.Tensor] = None, num_pages: int = 0,
-                 chunk_size: int = 0, topk: int = 0, num_splits: int = 0, device="cuda"):
+                 chunk_size: int = 0, topk: int = 0, num_splits: int = 0, residual: bool = False,
+                 device="cuda"):
         self.device = torch.device(device)
         self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
         self.B, self.Hq, self.Hkv, self.D, self.S = batch, num_q_heads, num_kv_heads, head_dim, block_len
@@ -55,10 +56,28 @@ class CachedBlockAttention:
             kv_capacity=self.capacity if page_size == 0 else 0, page_size=page_size,
             max_pages=self.max_pages, num_pages=self.num_pages, block_table=self.block_table,
             prefix_lens=self.lens, chunk_size=chunk_size, topk=topk, num_splits=num_splits)
+        self.residual = residual and topk > 0
         self.O_pre = torch.empty((batch, block_len, num_q_heads, head_dim), dtype=torch.float32, device=dev)
         self.LSE_pre = torch.empty((batch, num_q_heads, block_len), dtype=torch.float32, device=dev)
         self.LSE = torch.empty((batch, num_q_heads, block_len), dtype=torch.float32, device=dev)
         ws = fbl.fb_workspace_bytes(self.desc)
+        if self.residual:
+            # residual mode: the complement list is a chunk list of up to every chunk
+            nch = -(-self.capacity // chunk_size)
+            self.desc_res = fbl.make_desc(
+                batch, num_q_heads, num_kv_heads, head_dim, block_len,
+                dtype=self.desc.dtype, softmax_scale=softmax_scale,
+                kv_capacity=self.desc.kv_capacity, page_size=page_size, max_pages=self.max_pages,
+                num_pages=self.num_pages, block_table=self.block_table, prefix_lens=self.lens,
+                chunk_size=chunk_size, topk=nch, num_splits=num_splits)
+            ws = max(ws, fbl.fb_workspace_bytes(self.desc_res))
+            self.comp_idx = torch.full((batch, num_kv_heads, nch), -1, dtype=torch.int32, device=dev)
+            shape_o = (batch, block_len, num_q_heads, head_dim)
+            shape_l = (batch, num_q_heads, block_len)
+            self.O_res = torch.empty(shape_o, dtype=torch.float32, device=dev)
+            self.LSE_res = torch.empty(shape_l, dtype=torch.float32, device=dev)
+            self.O_sel = torch.empty(shape_o, dtype=torch.float32, device=dev)
+            self.LSE_sel = torch.empty(shape_l, dtype=torch.float32, device=dev)
         self.workspace = torch.empty(max(ws, 16) // 4 + 4, dtype=torch.float32, device=dev) if ws else None
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         if topk > 0:
@@ -95,18 +114,36 @@ class CachedBlockAttention:
 
     # ------------------------------------------------------------------ steps
     def refresh(self, Q: torch.Tensor) -> None:
-        """Refresh step: recompute the cached block-external pair with Q."""
+        """Refresh step: recompute the cached block-external pair with Q.
+
+        Residual mode: select the chunks, and cache the partial over the
+        chunks left out (the residual); the selected chunks are recomputed at
+        every step."""
         idx = None
         if self.topk > 0:
             fbl.fb_select_chunks(self.desc, Q, self.Kmean, self.chunk_idx, self.status)
             idx = self.chunk_idx
+        if self.residual:
+            cap = self.comp_idx.shape[2]
+            fbl.fb_complement_chunks(self.desc, self.chunk_idx, self.comp_idx, cap, self.status)
+            fbl.fb_prefix_partial(self.desc_res, Q, self.K, self.V, self.comp_idx, self.O_res, self.LSE_res,
+                                  self.workspace, self.status)
+            return
         fbl.fb_prefix_partial(self.desc, Q, self.K, self.V, idx, self.O_pre, self.LSE_pre,
                               self.workspace, self.status)
 
     def step(self, Q, Kblk, Vblk, out: Optional[torch.Tensor] = None, lse: bool = False):
-        """Cached denoising step: O = merge(cached pair, in-block partial)."""
+        """Cached denoising step: O = merge(cached pair, in-block partial).
+
+        Residual mode: the cached residual is first merged with a fresh
+        partial over the selected chunks (three partials in all)."""
         if out is None:
             out = torch.empty_like(Q)
+        if self.residual:
+            fbl.fb_prefix_partial(self.desc, Q, self.K, self.V, self.chunk_idx, self.O_sel, self.LSE_sel,
+                                  self.workspace, self.status)
+            fbl.fb_merge_partials(self.desc, self.O_res, self.LSE_res, self.O_sel, self.LSE_sel,
+                                  self.O_pre, self.LSE_pre)
         fbl.fb_block_step(self.desc, Q, Kblk, Vblk, self.O_pre, self.LSE_pre, out,
                           self.LSE if lse else None, self.status)
         return out

@@ -150,6 +150,26 @@ fb_status fb_chunk_means(const fb_desc* d, const void* Kcache, int32_t chunk_beg
 fb_status fb_select_chunks(const fb_desc* d, const void* Q, const float* Kmean,
                            int32_t* chunk_idx, int32_t* dev_status, fb_stream_t stream);
 
+/* Residual reuse with sparse attention (Adaptive Reuse Strategies,
+ * Compatibility with Sparse Attention: the unselected keys are the
+ * block-external set whose contribution is cached).  For each (b, kv head),
+ * the valid chunks (those holding a row j < prefix_lens[b]) that
+ * chunk_idx [B,Hkv,d->topk] does not list, ascending, padded with -1, into
+ * comp_idx [B,Hkv,comp_cap].  More than comp_cap of them records
+ * FB_ERR_BOUNDS.  Pass comp_idx to fb_prefix_partial with topk = comp_cap to
+ * get the residual partial. */
+fb_status fb_complement_chunks(const fb_desc* d, const int32_t* chunk_idx, int32_t* comp_idx,
+                               int32_t comp_cap, int32_t* dev_status, fb_stream_t stream);
+
+/* The merge equation on two partials (Core Mechanism): with m = max(L_a, L_b),
+ * O = (e^{L_a-m} O_a + e^{L_b-m} O_b) / (e^{L_a-m} + e^{L_b-m}) and
+ * L = m + log(e^{L_a-m} + e^{L_b-m}); two empty partials give (0, -inf).
+ * O_* [B,S,Hq,D] float32, LSE_* [B,Hq,S] float32; O_out/LSE_out may alias
+ * an input. */
+fb_status fb_merge_partials(const fb_desc* d, const float* O_a, const float* LSE_a,
+                            const float* O_b, const float* LSE_b, float* O_out,
+                            float* LSE_out, fb_stream_t stream);
+
 /* Block end ("KV caching with block-wise causal inference", Technical Summary
  * §1): copy the finalized block's K/V [B,S,Hkv,D] into cache rows
  * [L_b, L_b + S) (contiguous or paged).  When lens_inout is not NULL

@@ -39,7 +39,7 @@ def tensors(w, x):
     return t.cuda(), x64
 
 
-def make_layer(w, page_size=0, num_splits=0, topk=None):
+def make_layer(w, page_size=0, num_splits=0, topk=None, residual=False):
     topk = w.topk if topk is None else topk
     bt, npages = (None, 0)
     if page_size:
@@ -48,7 +48,7 @@ def make_layer(w, page_size=0, num_splits=0, topk=None):
     return CachedBlockAttention(
         w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_len, w.capacity, dtype=w.dtype,
         softmax_scale=w.softmax_scale, page_size=page_size, block_table=bt, num_pages=npages,
-        chunk_size=w.chunk_size if topk else 0, topk=topk, num_splits=num_splits)
+        chunk_size=w.chunk_size if topk else 0, topk=topk, num_splits=num_splits, residual=residual)
 
 
 def run_workload(w, page_size=0, num_splits=0, check_full=True, steps=None, blocks=None):
@@ -105,3 +105,30 @@ def run_workload(w, page_size=0, num_splits=0, check_full=True, steps=None, bloc
     layer.check()
     assert np.array_equal(layer.lens.cpu().numpy(), lens_o), "prefix lengths after append"
     return records
+
+
+def run_residual(w, steps=None):
+    """Residual reuse with sparse attention: GPU block vs the oracle's."""
+    K, V, lens = synth.prefix_kv(w)
+    Kt, K64 = tensors(w, K)
+    Vt, V64 = tensors(w, V)
+    layer = make_layer(w, residual=True)
+    layer.load_prefix(Kt, Vt, lens)
+    base = synth.block_base(w, 0)
+    nsteps = w.steps if steps is None else steps
+    Qs, Kbs, Vbs, outs = [], [], [], []
+    for s in range(nsteps):
+        Q, Kb, Vb = synth.step_inputs(w, 0, s, base)
+        Qt, Q64 = tensors(w, Q)
+        Kbt, Kb64 = tensors(w, Kb)
+        Vbt, Vb64 = tensors(w, Vb)
+        if s in w.refresh:
+            layer.refresh(Qt)
+        outs.append(layer.step(Qt, Kbt, Vbt).float().cpu().numpy())
+        Qs.append(Q64)
+        Kbs.append(Kb64)
+        Vbs.append(Vb64)
+    layer.check()
+    ref = ora.residual_block(Qs, Kbs, Vbs, K64, V64, lens.astype(np.int64), w.softmax_scale, w.refresh, w.topk,
+                             w.chunk_size)
+    return [compare(f"residual O s{s}", outs[s], ref[s], w.dtype) for s in range(nsteps)]

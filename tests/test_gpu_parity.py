@@ -10,6 +10,7 @@ import torch
 
 import gpu_cases
 from block_diffusion_attention_b200 import synth
+from oracle import flashblock_oracle as ora
 from block_diffusion_attention_b200 import flashblock as fbl
 
 pytestmark = pytest.mark.gpu
@@ -137,3 +138,28 @@ def test_block_graph_replay_matches_eager():
     layer.check()
     for s in range(w.steps):
         assert torch.equal(outs[s], eager[s]), f"step {s}"
+
+
+def test_residual_sparse_reuse():
+    # residual reuse: cached unselected-chunk partial + fresh selected chunks + block
+    w = W["batched_sparse"].scaled(batch=3, num_q_heads=8, num_kv_heads=2, prefix_len=1500,
+                                   prefix_min=600, topk=3, steps=6)
+    gpu_cases.run_residual(w)
+
+
+def test_merge_partials_matches_oracle():
+    rng = np.random.default_rng(5)
+    B, S, Hq, D = 2, 9, 4, 128
+    f32 = lambda x: x.astype(np.float32).astype(np.float64)  # noqa: E731
+    Oa, Ob = f32(rng.standard_normal((B, S, Hq, D))), f32(rng.standard_normal((B, S, Hq, D)))
+    La, Lb = f32(rng.standard_normal((B, Hq, S)) * 4), f32(rng.standard_normal((B, Hq, S)) * 4)
+    La[0, 0, 0] = -np.inf
+    La[1, 2, 3] = Lb[1, 2, 3] = -np.inf
+    d = fbl.make_desc(B, Hq, Hq, D, S)
+    t = lambda x: torch.tensor(x, dtype=torch.float32, device="cuda")  # noqa: E731
+    Oo, Lo = torch.empty(B, S, Hq, D, device="cuda"), torch.empty(B, Hq, S, device="cuda")
+    fbl.fb_merge_partials(d, t(Oa), t(La), t(Ob), t(Lb), Oo, Lo)
+    ref_o, ref_l = ora.merge_partials(Oa, La.transpose(0, 2, 1), Ob, Lb.transpose(0, 2, 1))
+    # fp32 on the GPU against float64 from the same (fp32-representable) inputs
+    gpu_cases.compare("merge O", Oo.cpu().numpy(), ref_o, "fp32")
+    gpu_cases.compare("merge LSE", Lo.cpu().numpy(), ref_l.transpose(0, 2, 1), "fp32")
