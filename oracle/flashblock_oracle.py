@@ -23,6 +23,9 @@ Efficient Long-Context Block Diffusion" (gist.science explainer of arXiv
   (:func:`select_chunks`, :func:`chunk_token_positions`); their cached
   residual is merged with the freshly computed selected keys
   (:func:`complement_chunks`, :func:`residual_block`).
+* §2 Methodology, Adaptive Reuse Strategies, "Threshold-based Reuse" and
+  "Head-wise Selection" -- refresh decisions by updated-token count tau and by
+  per-head similarity gamma (:func:`threshold_block`, :func:`headwise_block`).
 
 Readings where the page is silent (each listed in the design doc):
   L is the natural log of the unnormalised sum Z; J_out is the finalized
@@ -30,7 +33,10 @@ Readings where the page is silent (each listed in the design doc):
   reads KV head h // G; an empty key set gives (O = 0, L = -inf); the sparse
   chunk score is mean(block Q over tokens and group heads) . mean(chunk keys),
   top-k by descending score with ties broken towards the lower chunk index,
-  returned in ascending chunk order and padded with -1.
+  returned in ascending chunk order and padded with -1; head-wise
+  similarity is the cosine of a (b, kv head) unit's block queries against
+  the queries its cached pair was computed with; an updated token is a block
+  token whose K or V moved by more than eps since the previous step.
 
 Arrays are float64 numpy.  Layouts follow the C library's:
   Q, O           [B, S, Hq, D]
@@ -342,6 +348,86 @@ def residual_block(Qs, Kbs, Vbs, Kc, Vc, prefix_lens, scale, refresh_steps, topk
     return outs
 
 
+def unit_query_similarity(Q, Qref, hkv):
+    """Cosine similarity per (b, kv head) unit between the block's queries now
+    and the queries the unit's cached pair was computed with, over the unit's
+    S x G x D values ([B, Hkv])."""
+    B, S, Hq, D = Q.shape
+    G = _group(Hq, hkv)
+    sim = np.zeros((B, hkv))
+    for b in range(B):
+        for kvh in range(hkv):
+            a = Q[b, :, kvh * G:(kvh + 1) * G, :].ravel()
+            r = Qref[b, :, kvh * G:(kvh + 1) * G, :].ravel()
+            den = np.linalg.norm(a) * np.linalg.norm(r)
+            sim[b, kvh] = (a @ r) / den if den > 0 else 1.0
+    return sim
+
+
+def headwise_block(Qs, Kbs, Vbs, Kc, Vc, prefix_lens, scale, gamma):
+    """Head-wise selective reuse (Adaptive Reuse Strategies, Head-wise
+    Selection): step 0 computes every unit's block-external pair; at a later
+    step a (b, kv head) unit reuses its pair only if the similarity of its
+    queries to the ones the pair was computed with is at least gamma,
+    otherwise its pair is recomputed with the current queries.
+    Returns (list of O_s, list of refresh masks [B, Hkv])."""
+    B, S, Hq, D = Qs[0].shape
+    Hkv = Kc.shape[2]
+    G = _group(Hq, Hkv)
+    Op, Lp = prefix_partial(Qs[0], Kc, Vc, prefix_lens, scale)
+    Qref = Qs[0].copy()
+    outs, masks = [], []
+    for s, Q in enumerate(Qs):
+        if s == 0:
+            mask = np.ones((B, Hkv), dtype=bool)
+        else:
+            mask = unit_query_similarity(Q, Qref, Hkv) < gamma
+            if mask.any():
+                On, Ln = prefix_partial(Q, Kc, Vc, prefix_lens, scale)
+                for b in range(B):
+                    for kvh in range(Hkv):
+                        if mask[b, kvh]:
+                            hs = slice(kvh * G, (kvh + 1) * G)
+                            Op[b, :, hs] = On[b, :, hs]
+                            Lp[b, hs] = Ln[b, hs]
+                            Qref[b, :, hs] = Q[b, :, hs]
+        o, _ = block_step(Q, Kbs[s], Vbs[s], Op, Lp, scale)
+        outs.append(o)
+        masks.append(mask)
+    return outs, masks
+
+
+def updated_tokens(Kprev, Vprev, Know, Vnow, eps):
+    """M: per sequence, the block tokens whose key or value moved by more than
+    eps (max abs change over heads and dims) since the previous step ([B])."""
+    dk = np.abs(Know - Kprev).max(axis=(2, 3))
+    dv = np.abs(Vnow - Vprev).max(axis=(2, 3))
+    return ((dk > eps) | (dv > eps)).sum(axis=1)
+
+
+def threshold_block(Qs, Kbs, Vbs, Kc, Vc, prefix_lens, scale, tau, eps):
+    """Threshold-based reuse (Adaptive Reuse Strategies): step 0 refreshes;
+    at step s + 1 a sequence reuses its block-external pair if the number of
+    updated tokens M^{s+1} is below tau, else recomputes it.
+    Returns (list of O_s, list of per-sequence refresh flags [B])."""
+    B, S, Hq, D = Qs[0].shape
+    Op, Lp = prefix_partial(Qs[0], Kc, Vc, prefix_lens, scale)
+    outs, flags = [], []
+    for s, Q in enumerate(Qs):
+        if s == 0:
+            flag = np.ones(B, dtype=bool)
+        else:
+            flag = updated_tokens(Kbs[s - 1], Vbs[s - 1], Kbs[s], Vbs[s], eps) >= tau
+            if flag.any():
+                On, Ln = prefix_partial(Q, Kc, Vc, prefix_lens, scale)
+                Op[flag] = On[flag]
+                Lp[flag] = Ln[flag]
+        o, _ = block_step(Q, Kbs[s], Vbs[s], Op, Lp, scale)
+        outs.append(o)
+        flags.append(flag)
+    return outs, flags
+
+
 def attention_weights(q, k, scale):
     """Explicit softmax weight matrix e^{z - L} of one partial ([R, N])."""
     _, lse = attention_partial(q, k, np.zeros((k.shape[0], 1)), scale)
@@ -353,5 +439,6 @@ __all__ = [
     "NEG_INF", "attention_partial", "merge_partials", "chunk_token_positions",
     "prefix_partial", "inblock_partial", "block_step", "full_attention",
     "chunk_means", "chunk_scores", "select_chunks", "cached_block",
-    "complement_chunks", "residual_block", "attention_weights",
+    "complement_chunks", "residual_block", "unit_query_similarity", "headwise_block",
+    "updated_tokens", "threshold_block", "attention_weights",
 ]

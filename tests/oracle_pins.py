@@ -322,6 +322,66 @@ def pin_residual_reuse(ora):
             assert a == [c for c in range(valid.shape[1]) if valid[b, c]], "selection + complement"
 
 
+def _drift_block(rng, B=2, S=3, Hq=4, Hkv=2, D=4, Lcap=20, steps=4, sig=0.3):
+    Kc, Vc = _rand(rng, B, Lcap, Hkv, D), _rand(rng, B, Lcap, Hkv, D)
+    lens = np.array([Lcap, Lcap - 7], dtype=np.int32)[:B]
+    Q0, K0, V0 = _rand(rng, B, S, Hq, D), _rand(rng, B, S, Hkv, D), _rand(rng, B, S, Hkv, D)
+    Qs = [Q0 + sig * _rand(rng, B, S, Hq, D) for _ in range(steps)]
+    Ks = [K0 + sig * _rand(rng, B, S, Hkv, D) for _ in range(steps)]
+    Vs = [V0 + sig * _rand(rng, B, S, Hkv, D) for _ in range(steps)]
+    return Kc, Vc, lens, Qs, Ks, Vs
+
+
+def pin_headwise_refresh(ora):
+    """gamma above 1 refreshes every unit every step (= full attention);
+    gamma at -1 never refreshes after step 0 (= the cached schedule); the
+    similarity is 1 for identical queries and symmetric."""
+    rng = np.random.default_rng(22)
+    Kc, Vc, lens, Qs, Ks, Vs = _drift_block(rng)
+    outs, masks = ora.headwise_block(Qs, Ks, Vs, Kc, Vc, lens, 0.6, 1.5)
+    for s in range(len(Qs)):
+        Of, _ = ora.full_attention(Qs[s], Kc, Vc, lens, Ks[s], Vs[s], 0.6)
+        _close(outs[s], Of, 1e-12, f"head-wise, gamma 1.5, step {s}")
+        assert masks[s].all()
+    outs, masks = ora.headwise_block(Qs, Ks, Vs, Kc, Vc, lens, 0.6, -1.0)
+    cached, _ = ora.cached_block(Qs, Ks, Vs, Kc, Vc, lens, 0.6, (0,))
+    for s in range(len(Qs)):
+        _close(outs[s], cached[s], 1e-12, f"head-wise, gamma -1, step {s}")
+        assert masks[s].all() if s == 0 else not masks[s].any()
+    # refresh decisions: a big query jump refreshes, a repeat of the new
+    # queries then reuses (the reference moved with the refresh)
+    Qj = [Qs[0], Qs[0] + 5.0 * _rand(rng, *Qs[0].shape)]
+    Qj.append(Qj[1].copy())
+    outs, masks = ora.headwise_block(Qj, Ks[:3], Vs[:3], Kc, Vc, lens, 0.6, 0.999)
+    assert masks[1].all() and not masks[2].any(), [m.tolist() for m in masks]
+    sim = ora.unit_query_similarity(Qs[1], Qs[2], 2)
+    _close(sim, ora.unit_query_similarity(Qs[2], Qs[1], 2), 1e-14, "similarity symmetric")
+    _close(ora.unit_query_similarity(Qs[1], Qs[1], 2), np.ones((2, 2)), 1e-14, "self-similarity")
+    # a unit whose queries are a positive multiple of the reference: similarity 1
+    _close(ora.unit_query_similarity(3.0 * Qs[1], Qs[1], 2), np.ones((2, 2)), 1e-14, "scale invariance")
+
+
+def pin_threshold_refresh(ora):
+    """tau = 0 refreshes every step (= full attention); tau above S never
+    refreshes (= the cached schedule); the updated-token count by hand."""
+    rng = np.random.default_rng(23)
+    Kc, Vc, lens, Qs, Ks, Vs = _drift_block(rng)
+    outs, flags = ora.threshold_block(Qs, Ks, Vs, Kc, Vc, lens, 0.6, 0, 1e-3)
+    for s in range(len(Qs)):
+        Of, _ = ora.full_attention(Qs[s], Kc, Vc, lens, Ks[s], Vs[s], 0.6)
+        _close(outs[s], Of, 1e-12, f"threshold, tau 0, step {s}")
+    outs, flags = ora.threshold_block(Qs, Ks, Vs, Kc, Vc, lens, 0.6, 99, 1e-3)
+    cached, _ = ora.cached_block(Qs, Ks, Vs, Kc, Vc, lens, 0.6, (0,))
+    for s in range(len(Qs)):
+        _close(outs[s], cached[s], 1e-12, f"threshold, tau 99, step {s}")
+    K1, V1 = Ks[0].copy(), Vs[0].copy()
+    K1[0, 1, 1, 2] += 0.5      # token 1 of sequence 0 moves in K
+    V1[1, 0, 0, 0] -= 0.01     # token 0 of sequence 1 moves a little in V
+    V1[1, 2, 1, 3] += 0.2      # token 2 of sequence 1 moves in V
+    m = ora.updated_tokens(Ks[0], Vs[0], K1, V1, 0.05)
+    assert m.tolist() == [1, 1], m
+
+
 def pin_selection_ties(ora):
     """Equal scores: the lower chunk index wins."""
     D = 2
@@ -339,7 +399,7 @@ def pin_selection_ties(ora):
 ALL_PINS = [pin_brute_partial, pin_brute_layer, pin_golden, pin_closed_forms,
             pin_merge_is_concat, pin_merge_algebra, pin_refresh_step_exact,
             pin_reuse_unchanged_queries, pin_refresh_recomputes, pin_rows_sum_to_one, pin_sparse,
-            pin_residual_reuse, pin_selection_ties]
+            pin_residual_reuse, pin_headwise_refresh, pin_threshold_refresh, pin_selection_ties]
 
 
 def failing_pins(ora):

@@ -41,6 +41,11 @@ MUTANTS = {
     "reuse_never_refresh": ("if s in refresh_steps or pre is None:", "if pre is None:"),
     "residual_stale_selected": ("sel = prefix_partial(Q, Kc, Vc, prefix_lens, scale, idx, chunk_size)",
                                 "sel = prefix_partial(Qs[0], Kc, Vc, prefix_lens, scale, idx, chunk_size)"),
+    "headwise_keeps_stale_ref": ("                            Qref[b, :, hs] = Q[b, :, hs]\n", ""),
+    "similarity_unnormalised": ("sim[b, kvh] = (a @ r) / den if den > 0 else 1.0", "sim[b, kvh] = (a @ r) if den > 0 else 1.0"),
+    "threshold_inverted": ("updated_tokens(Kbs[s - 1], Vbs[s - 1], Kbs[s], Vbs[s], eps) >= tau",
+                           "updated_tokens(Kbs[s - 1], Vbs[s - 1], Kbs[s], Vbs[s], eps) < tau"),
+    "updated_ignores_v": ("return ((dk > eps) | (dv > eps)).sum(axis=1)", "return (dk > eps).sum(axis=1)"),
     "complement_drops_last": ("comp[b, kvh, :len(rest)] = rest", "comp[b, kvh, :len(rest) - 1] = rest[:-1]"),
 }
 
