@@ -253,12 +253,17 @@ size_t fb_workspace_bytes(const fb_desc* d) {
   dense.topk = 0;
   const int ns_full = choose_splits(dense, prefix_tiles_estimate(dense) + (d->block_len + TC_BN - 1) / TC_BN);
   const size_t a = split_bytes(*d, ns_pre), b = split_bytes(*d, ns_full);
-  return a > b ? a : b;
+  const size_t c = threshold_ws_bytes(*d);
+  return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
-fb_status fb_prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const void* Vc,
-                            const int32_t* chunk_idx, float* O_pre, float* LSE_pre, void* ws,
-                            size_t ws_bytes, int32_t* dev_status, fb_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+fb_status prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const void* Vc,
+                         const int32_t* chunk_idx, const int32_t* unit_mask, float* O_pre, float* LSE_pre,
+                         void* ws, size_t ws_bytes, int32_t* dev_status, fb_stream_t stream) {
   fb_status st = check_desc(d);
   if (st != FB_OK) return st;
   if ((st = check_cache(d)) != FB_OK) return st;
@@ -272,6 +277,7 @@ fb_status fb_prefix_partial(const fb_desc* d, const void* Q, const void* Kc, con
   p.src = key_source(*d, true, false, chunk_idx);
   p.epi = EPI_PARTIAL;
   p.dev_status = dev_status;
+  p.unit_mask = unit_mask;
   if (d->dtype == FB_FP32) {
     p.out_o32 = O_pre;
     p.out_lse = LSE_pre;
@@ -307,7 +313,54 @@ fb_status fb_prefix_partial(const fb_desc* d, const void* Q, const void* Kc, con
   c.part_lse = part_l;
   c.out_o32 = O_pre;
   c.out_lse = LSE_pre;
+  c.G = p.G;
+  c.unit_mask = unit_mask;
   return from_cuda(launch_combine(c, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+fb_status fb_prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const void* Vc,
+                            const int32_t* chunk_idx, float* O_pre, float* LSE_pre, void* ws,
+                            size_t ws_bytes, int32_t* dev_status, fb_stream_t stream) {
+  return prefix_partial(d, Q, Kc, Vc, chunk_idx, nullptr, O_pre, LSE_pre, ws, ws_bytes, dev_status, stream);
+}
+
+fb_status fb_prefix_partial_masked(const fb_desc* d, const void* Q, const void* Kc, const void* Vc,
+                                   const int32_t* chunk_idx, const int32_t* unit_mask, float* O_pre,
+                                   float* LSE_pre, void* ws, size_t ws_bytes, int32_t* dev_status,
+                                   fb_stream_t stream) {
+  if (!unit_mask) return FB_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(unit_mask) & 3u) return FB_ERR_ALIGNMENT;
+  return prefix_partial(d, Q, Kc, Vc, chunk_idx, unit_mask, O_pre, LSE_pre, ws, ws_bytes, dev_status, stream);
+}
+
+fb_status fb_headwise_refresh_mask(const fb_desc* d, const void* Q_now, void* Q_ref, float gamma,
+                                   int32_t* unit_mask, float* sim_out, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!Q_now || !Q_ref || !unit_mask || std::isnan(gamma)) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q_now) || !aligned16(Q_ref) || (reinterpret_cast<uintptr_t>(unit_mask) & 3u) ||
+      (reinterpret_cast<uintptr_t>(sim_out) & 3u))
+    return FB_ERR_ALIGNMENT;
+  return from_cuda(launch_headwise_mask(*d, Q_now, Q_ref, gamma, unit_mask, sim_out,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fb_status fb_threshold_refresh_mask(const fb_desc* d, void* K_prev, void* V_prev, const void* K_now,
+                                    const void* V_now, float eps, int32_t tau, int32_t* unit_mask,
+                                    int32_t* count_out, void* ws, size_t ws_bytes, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!K_prev || !V_prev || !K_now || !V_now || !unit_mask || std::isnan(eps)) return FB_ERR_INVALID_ARG;
+  if (!aligned16(K_prev) || !aligned16(V_prev) || !aligned16(K_now) || !aligned16(V_now) ||
+      (reinterpret_cast<uintptr_t>(unit_mask) & 3u) || (reinterpret_cast<uintptr_t>(count_out) & 3u))
+    return FB_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < threshold_ws_bytes(*d) || !aligned16(ws)) return FB_ERR_WORKSPACE;
+  return from_cuda(launch_threshold_mask(*d, K_prev, V_prev, K_now, V_now, eps, tau, unit_mask, count_out,
+                                         static_cast<int32_t*>(ws), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const void* Vb,

@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(WARPS * 32)
   const int b = blockIdx.z;
   if (t >= p.S) return;
   const int kvh = h / p.G;
+  if (p.unit_mask && p.unit_mask[b * p.Hkv + kvh] == 0) return;  // unit not refreshed: outputs kept
   const int D = p.D;
   const int nd = D >> 5;  // output columns per lane
   const size_t qrow = ((size_t)b * p.S + t) * p.Hq + h;

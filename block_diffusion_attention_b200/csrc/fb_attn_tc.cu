@@ -281,7 +281,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   pdl_wait();
   pdl_launch_dependents();
 
-  const UnitTiles u = unit_tiles(p, b, kvh, threadIdx.x == 0);
+  // a unit the refresh mask leaves out keeps its cached outputs: no work
+  const bool skip = p.unit_mask != nullptr && p.unit_mask[b * p.Hkv + kvh] == 0;
+  const UnitTiles u = skip ? UnitTiles{0, 0, 0} : unit_tiles(p, b, kvh, threadIdx.x == 0);
   const int ntot = u.n0 + u.n1;
   const int j0 = (int)(((long long)split * ntot) / p.nsplit);
   const int j1 = (int)(((long long)(split + 1) * ntot) / p.nsplit);
@@ -291,7 +293,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   // two ring slots free: the cached O_pre rows are prefetched into them.
   const bool pre_smem = (EPI == EPI_MERGE) && nt <= 2;
 
-  if (warp == 4) {
+  if (skip) {
+    // nothing to load, multiply or write
+  } else if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_map(&tmQ);
@@ -674,6 +678,7 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombinePa
   const size_t so = (size_t)nrows * c.D;              // split stride of the partial O
   const size_t sl = (size_t)c.B * c.Hq * c.S;         // split stride of the partial LSE
   const size_t lrow = ((size_t)b * c.Hq + h) * c.S + t;
+  if (c.unit_mask && c.unit_mask[b * (c.Hq / c.G) + h / c.G] == 0) return;  // unit not refreshed
   // lane l holds the LSE (then the weight) of splits l, l + 32, l + 64, l + 96
   constexpr int PER_LANE = TC_MAX_SPLITS / 32;
   float wreg[PER_LANE];

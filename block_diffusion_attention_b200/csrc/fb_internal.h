@@ -42,6 +42,7 @@ struct AttnParams {
   float scale_log2;  // scale * log2(e)
   int epi;
   int kv_stream_once;  // 1: prefix K/V is read once (evict-first L2 hint)
+  const int32_t* unit_mask;  // [B, Hkv] or null: units with 0 are skipped (their outputs kept)
   KeySource src;
   // outputs
   float* out_o32;         // EPI_PARTIAL: [nsplit][B][S][Hq][D]
@@ -54,6 +55,8 @@ struct AttnParams {
 
 struct CombineParams {
   int B, Hq, S, D, nsplit;
+  int G;                  // query heads per kv head (for unit_mask)
+  const int32_t* unit_mask;  // [B, Hkv] or null: rows of units with 0 are left as they are
   const float* part_o;    // [nsplit][B][S][Hq][D]
   const float* part_lse;  // [nsplit][B][Hq][S]
   float* out_o32;         // f32 output (prefix pass) or null
@@ -89,6 +92,12 @@ cudaError_t launch_complement_chunks(const fb_desc& d, const int32_t* idx, int32
                                      int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_merge_partials(const fb_desc& d, const float* Oa, const float* La, const float* Ob,
                                   const float* Lb, float* Oo, float* Lo, cudaStream_t stream);
+cudaError_t launch_headwise_mask(const fb_desc& d, const void* Qnow, void* Qref, float gamma, int32_t* mask,
+                                 float* sim, cudaStream_t stream);
+cudaError_t launch_threshold_mask(const fb_desc& d, void* Kprev, void* Vprev, const void* Know, const void* Vnow,
+                                  float eps, int32_t tau, int32_t* mask, int32_t* count, int32_t* ws,
+                                  cudaStream_t stream);
+size_t threshold_ws_bytes(const fb_desc& d);  // per-slice token counts of the threshold pass
 cudaError_t launch_kv_append(const fb_desc& d, const void* Kb, const void* Vb, void* Kc, void* Vc,
                              int32_t* lens_inout, int32_t* dev_status, cudaStream_t stream);
 

@@ -76,6 +76,9 @@ def load() -> ctypes.CDLL:
             "fb_kv_append": (I32, [D, P, P, P, P, P, P, P]),
             "fb_complement_chunks": (I32, [D, P, P, I32, P, P]),
             "fb_merge_partials": (I32, [D, P, P, P, P, P, P, P]),
+            "fb_headwise_refresh_mask": (I32, [D, P, P, ctypes.c_float, P, P, P]),
+            "fb_threshold_refresh_mask": (I32, [D, P, P, P, P, ctypes.c_float, I32, P, P, P, SZ, P]),
+            "fb_prefix_partial_masked": (I32, [D, P, P, P, P, P, P, P, P, SZ, P, P]),
             "fb_status_string": (ctypes.c_char_p, [I32]),
             "fb_launch_count": (ctypes.c_uint64, []),
             "fb_abi_version": (I32, []),
@@ -189,6 +192,26 @@ def fb_complement_chunks(d, chunk_idx, comp_idx, comp_cap, dev_status, stream=No
 def fb_merge_partials(d, O_a, LSE_a, O_b, LSE_b, O_out, LSE_out, stream=None):
     _ok("fb_merge_partials", load().fb_merge_partials(
         ctypes.byref(d), _p(O_a), _p(LSE_a), _p(O_b), _p(LSE_b), _p(O_out), _p(LSE_out), _s(stream)))
+
+
+def fb_headwise_refresh_mask(d, Q_now, Q_ref, gamma, unit_mask, sim_out=None, stream=None):
+    _ok("fb_headwise_refresh_mask", load().fb_headwise_refresh_mask(
+        ctypes.byref(d), _p(Q_now), _p(Q_ref), float(gamma), _p(unit_mask), _p(sim_out), _s(stream)))
+
+
+def fb_threshold_refresh_mask(d, K_prev, V_prev, K_now, V_now, eps, tau, unit_mask, count_out, workspace,
+                              stream=None):
+    _ok("fb_threshold_refresh_mask", load().fb_threshold_refresh_mask(
+        ctypes.byref(d), _p(K_prev), _p(V_prev), _p(K_now), _p(V_now), float(eps), int(tau), _p(unit_mask),
+        _p(count_out), _p(workspace), _nbytes(workspace), _s(stream)))
+
+
+def fb_prefix_partial_masked(d, Q, Kcache, Vcache, chunk_idx, unit_mask, O_pre, LSE_pre, workspace, dev_status,
+                             stream=None):
+    """fb_prefix_partial for the units whose unit_mask entry is non-zero."""
+    _ok("fb_prefix_partial_masked", load().fb_prefix_partial_masked(
+        ctypes.byref(d), _p(Q), _p(Kcache), _p(Vcache), _p(chunk_idx), _p(unit_mask), _p(O_pre), _p(LSE_pre),
+        _p(workspace), _nbytes(workspace), _p(dev_status), _s(stream)))
 
 
 def fb_status_string(status: int) -> str:

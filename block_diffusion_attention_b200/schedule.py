@@ -6,6 +6,7 @@
 chunk list -- and exposes the calls of one block of denoising steps:
 
     refresh(Q)            prefix partial with this step's queries (refresh step)
+    adapt(Q, Kblk, Vblk)  policy mode: refresh mask, then the masked prefix partial
     step(Q, Kblk, Vblk)   in-block partial merged with the cached pair -> O
     full(Q, Kblk, Vblk)   uncached attention over [prefix ; block] -> O
     append(Kblk, Vblk)    finalized block joins the cache
@@ -27,6 +28,7 @@ class CachedBlockAttention:
                  capacity: int, dtype: str = "bf16", softmax_scale: float = 1.0, page_size: int = 0,
                  block_table: Optional[torch.Tensor] = None, num_pages: int = 0,
                  chunk_size: int = 0, topk: int = 0, num_splits: int = 0, residual: bool = False,
+                 policy: Optional[str] = None, gamma: float = 0.9, tau: int = 1, eps: float = 0.25,
                  device="cuda"):
         self.device = torch.device(device)
         self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -78,6 +80,19 @@ class CachedBlockAttention:
             self.LSE_res = torch.empty(shape_l, dtype=torch.float32, device=dev)
             self.O_sel = torch.empty(shape_o, dtype=torch.float32, device=dev)
             self.LSE_sel = torch.empty(shape_l, dtype=torch.float32, device=dev)
+        # adaptive reuse: a policy decides at every step which units refresh
+        assert policy in (None, "headwise", "threshold")
+        assert policy is None or (topk == 0 and not residual), "refresh policies use the dense prefix"
+        self.policy, self.gamma, self.tau, self.eps = policy, gamma, tau, eps
+        if policy is not None:
+            self.unit_mask = torch.ones((batch, num_kv_heads), dtype=torch.int32, device=dev)
+        if policy == "headwise":
+            self.Q_ref = torch.zeros((batch, block_len, num_q_heads, head_dim), dtype=self.tdtype, device=dev)
+            self.sim = torch.zeros((batch, num_kv_heads), dtype=torch.float32, device=dev)
+        elif policy == "threshold":
+            self.K_prev = torch.zeros((batch, block_len, num_kv_heads, head_dim), dtype=self.tdtype, device=dev)
+            self.V_prev = torch.zeros_like(self.K_prev)
+            self.updated = torch.zeros(batch, dtype=torch.int32, device=dev)
         self.workspace = torch.empty(max(ws, 16) // 4 + 4, dtype=torch.float32, device=dev) if ws else None
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         if topk > 0:
@@ -132,6 +147,30 @@ class CachedBlockAttention:
         fbl.fb_prefix_partial(self.desc, Q, self.K, self.V, idx, self.O_pre, self.LSE_pre,
                               self.workspace, self.status)
 
+    def adapt(self, Q, Kblk, Vblk, first: bool) -> None:
+        """Adaptive refresh (policy mode): decide per unit whether the cached
+        pair is recomputed at this step, then recompute the chosen units.  The
+        first step of a block refreshes every unit."""
+        if self.policy == "headwise":
+            fbl.fb_headwise_refresh_mask(self.desc, Q, self.Q_ref, float("inf") if first else self.gamma,
+                                         self.unit_mask, self.sim)
+        else:
+            fbl.fb_threshold_refresh_mask(self.desc, self.K_prev, self.V_prev, Kblk, Vblk, self.eps,
+                                          0 if first else self.tau, self.unit_mask, self.updated,
+                                          self.workspace)
+        fbl.fb_prefix_partial_masked(self.desc, Q, self.K, self.V, None, self.unit_mask, self.O_pre,
+                                     self.LSE_pre, self.workspace, self.status)
+
+    def cached_step(self, s: int, Q, Kblk, Vblk, refresh_steps=(0,), out: Optional[torch.Tensor] = None,
+                    lse: bool = False):
+        """Step s of a block: the refresh its schedule (or policy) asks for,
+        then the fused step."""
+        if self.policy is not None:
+            self.adapt(Q, Kblk, Vblk, first=(s == 0))
+        elif s in refresh_steps:
+            self.refresh(Q)
+        return self.step(Q, Kblk, Vblk, out=out, lse=lse)
+
     def step(self, Q, Kblk, Vblk, out: Optional[torch.Tensor] = None, lse: bool = False):
         """Cached denoising step: O = merge(cached pair, in-block partial).
 
@@ -180,9 +219,7 @@ class CachedBlockAttention:
         every step.  Ends with the append of ``append_kv`` when given."""
         for s, (Q, Kb, Vb) in enumerate(steps):
             if cached:
-                if s in refresh_steps:
-                    self.refresh(Q)
-                self.step(Q, Kb, Vb, out=outs[s])
+                self.cached_step(s, Q, Kb, Vb, refresh_steps, out=outs[s])
             else:
                 self.full(Q, Kb, Vb, out=outs[s])
         if append_kv is not None:
@@ -205,9 +242,7 @@ class CachedBlockAttention:
                 if prologue is not None:
                     prologue(s)
                 if cached:
-                    if s in refresh_steps:
-                        self.refresh(Q)
-                    self.step(Q, Kb, Vb, out=outs[s])
+                    self.cached_step(s, Q, Kb, Vb, refresh_steps, out=outs[s])
                 else:
                     self.full(Q, Kb, Vb, out=outs[s])
                 if epilogue is not None:

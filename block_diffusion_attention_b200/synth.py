@@ -33,6 +33,7 @@ import numpy as np
 
 # tensor ids of the seed tuple
 T_Q, T_K, T_V, T_PREFIX_K, T_LENS, T_PREFIX_V, T_PAGES = 0, 1, 2, 3, 4, 5, 6
+T_JUMP, T_UPDATE = 7, 8
 BASE_STEP = 0xBA5E  # "step" slot of the seed tuple used for a block's base draw
 
 
@@ -146,6 +147,65 @@ def step_inputs(w: Workload, block: int, step: int, base=None, drift: Optional[f
     K = K0 + sig * rng(w, block, step, T_K).standard_normal(K0.shape, dtype=np.float32)
     V = V0 + sig * rng(w, block, step, T_V).standard_normal(V0.shape, dtype=np.float32)
     return Q, K, V
+
+
+def headwise_steps(w: Workload, block: int, steps: int, p_jump: float = 0.35, rel_drift: float = 0.05,
+                   base=None):
+    """Steps for the head-wise reuse policy: per (b, kv head) unit, the
+    queries either stay near their current values (independent
+    N(0, (rel_drift * q_std)^2) noise per step) or, with probability p_jump at
+    each step after the first, are redrawn as a whole (N(0, q_std^2)).  K and
+    V drift as in ``step_inputs``.  Returns lists of float32 (Q, K, V)."""
+    if base is None:
+        base = block_base(w, block)
+    Q0 = base[0]
+    B, S, Hq, D = Q0.shape
+    G = w.group
+    cur = Q0.copy()
+    out = []
+    for s in range(steps):
+        if s > 0:
+            r = rng(w, block, s, T_JUMP)
+            jump = r.random((B, w.num_kv_heads)) < p_jump
+            fresh = r.standard_normal(Q0.shape, dtype=np.float32) * np.float32(w.q_std)
+            for b in range(B):
+                for kvh in range(w.num_kv_heads):
+                    if jump[b, kvh]:
+                        cur[b, :, kvh * G:(kvh + 1) * G] = fresh[b, :, kvh * G:(kvh + 1) * G]
+        noise = rng(w, block, s, T_Q).standard_normal(Q0.shape, dtype=np.float32)
+        Q = cur + np.float32(rel_drift * w.q_std) * noise
+        _, K, V = step_inputs(w, block, s, base, q_drift=False)
+        out.append((Q, K, V))
+    return out
+
+
+def threshold_steps(w: Workload, block: int, steps: int, max_updates: Optional[int] = None,
+                    noise: float = 0.01, base=None):
+    """Steps for the threshold reuse policy: at each step after the first,
+    every sequence redraws the K and V (N(0, 1)) of a seeded number of its
+    block tokens, uniform in [0, max_updates] (default S/2), chosen at
+    random; all tokens also carry independent N(0, noise^2) noise per step.
+    Queries drift as in ``step_inputs``.  Returns lists of float32 (Q, K, V)."""
+    if base is None:
+        base = block_base(w, block)
+    Q0, K0, V0 = base
+    B, S = K0.shape[0], K0.shape[1]
+    top = S // 2 if max_updates is None else max_updates
+    K, V = K0.copy(), V0.copy()
+    out = []
+    for s in range(steps):
+        if s > 0:
+            r = rng(w, block, s, T_UPDATE)
+            n = r.integers(0, top, size=B, endpoint=True)
+            for b in range(B):
+                toks = r.choice(S, size=int(n[b]), replace=False)
+                K[b, toks] = r.standard_normal((len(toks),) + K0.shape[2:], dtype=np.float32)
+                V[b, toks] = r.standard_normal((len(toks),) + V0.shape[2:], dtype=np.float32)
+        Q, _, _ = step_inputs(w, block, s, base)
+        nk = rng(w, block, s, T_K).standard_normal(K0.shape, dtype=np.float32)
+        nv = rng(w, block, s, T_V).standard_normal(V0.shape, dtype=np.float32)
+        out.append((Q, K + np.float32(noise) * nk, V + np.float32(noise) * nv))
+    return out
 
 
 def page_table(w: Workload, page_size: int, lens_cap: Optional[int] = None):

@@ -170,6 +170,53 @@ fb_status fb_merge_partials(const fb_desc* d, const float* O_a, const float* LSE
                             const float* O_b, const float* LSE_b, float* O_out,
                             float* LSE_out, fb_stream_t stream);
 
+/* ---- Adaptive reuse: refresh masks ("Adaptive Reuse Strategies") ----------
+ * Instead of refreshing the cached block-external pair at fixed steps, a
+ * policy decides at every step which work units recompute it.  A refresh
+ * mask is device int32 [B, Hkv] (1 = recompute the (b, kv head) unit's pair
+ * with this step's queries, 0 = keep the cached one); the policy calls below
+ * write it and fb_prefix_partial_masked consumes it. */
+
+/* Head-wise Selection: unit (b, kvh) refreshes when the cosine similarity of
+ * its queries now (Q_now [B,S,Hq,D], heads kvh*G .. kvh*G+G-1) to the
+ * reference queries (Q_ref, same layout: the queries the unit's cached pair
+ * was computed with) is below gamma, i.e. sim < gamma; a NaN similarity
+ * refreshes, and a unit whose two query sets are all zero has similarity 1.
+ * The similarity is taken over the unit's S x G x D values, accumulated in
+ * float32.  A refreshed unit's Q_now values are copied into Q_ref (which the
+ * caller owns and keeps between steps).  gamma = +inf refreshes every unit
+ * whatever Q_ref holds (use it on the first step of a block).  sim_out (device
+ * float32 [B, Hkv]) may be NULL.  Q pointers 16-byte aligned.  Returns
+ * FB_ERR_INVALID_ARG for a NaN gamma. */
+fb_status fb_headwise_refresh_mask(const fb_desc* d, const void* Q_now, void* Q_ref, float gamma,
+                                   int32_t* unit_mask, float* sim_out, fb_stream_t stream);
+
+/* Threshold-based Reuse: sequence b refreshes (all its units) when M_b >= tau,
+ * M_b the number of block tokens t whose key or value moved by more than eps
+ * since the previous step: max over kv heads and dims of |K_now - K_prev| or
+ * of |V_now - V_prev| above eps (differences taken in float32).  K/V blocks
+ * [B,S,Hkv,D] in the descriptor's dtype, 16-byte aligned.  K_prev / V_prev
+ * are state the caller owns: the call overwrites them with K_now / V_now, so
+ * the next step compares with this one.  tau <= 0 refreshes every sequence
+ * whatever K_prev / V_prev hold (use it on the first step of a block).
+ * count_out (device int32 [B], M_b) may be NULL.  ws: device workspace of at
+ * least fb_workspace_bytes(d) bytes (16-byte aligned; it may be the one the
+ * prefix pass uses).  Returns FB_ERR_INVALID_ARG for a NaN eps. */
+fb_status fb_threshold_refresh_mask(const fb_desc* d, void* K_prev, void* V_prev, const void* K_now,
+                                    const void* V_now, float eps, int32_t tau, int32_t* unit_mask,
+                                    int32_t* count_out, void* ws, size_t ws_bytes, fb_stream_t stream);
+
+/* fb_prefix_partial restricted to the units a refresh mask selects: units
+ * with unit_mask[b*Hkv + kvh] != 0 get (O_pre, LSE_pre) rows recomputed
+ * exactly as fb_prefix_partial computes them; the rows of the other units are
+ * not read or written (they keep the cached pair).  unit_mask: device int32
+ * [B, Hkv], read on the device (no host synchronisation).  Other arguments,
+ * workspace rule and errors as for fb_prefix_partial. */
+fb_status fb_prefix_partial_masked(const fb_desc* d, const void* Q, const void* Kcache,
+                                   const void* Vcache, const int32_t* chunk_idx,
+                                   const int32_t* unit_mask, float* O_pre, float* LSE_pre, void* ws,
+                                   size_t ws_bytes, int32_t* dev_status, fb_stream_t stream);
+
 /* Block end ("KV caching with block-wise causal inference", Technical Summary
  * §1): copy the finalized block's K/V [B,S,Hkv,D] into cache rows
  * [L_b, L_b + S) (contiguous or paged).  When lens_inout is not NULL

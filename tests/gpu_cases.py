@@ -132,3 +132,64 @@ def run_residual(w, steps=None):
     ref = ora.residual_block(Qs, Kbs, Vbs, K64, V64, lens.astype(np.int64), w.softmax_scale, w.refresh, w.topk,
                              w.chunk_size)
     return [compare(f"residual O s{s}", outs[s], ref[s], w.dtype) for s in range(nsteps)]
+
+
+def run_policy(w, policy, steps, gamma=0.9, tau=None, eps=0.25, margin=1e-3):
+    """Adaptive reuse on the GPU vs the oracle's ``headwise_block`` /
+    ``threshold_block`` on the policy input generators.
+
+    The decisions are compared exactly; the inputs are first checked to keep
+    every decision at least ``margin`` away from its threshold (computed from
+    the oracle's own decisions), so that rounding cannot flip one."""
+    K, V, lens = synth.prefix_kv(w)
+    Kt, K64 = tensors(w, K)
+    Vt, V64 = tensors(w, V)
+    gen = synth.headwise_steps if policy == "headwise" else synth.threshold_steps
+    raw = gen(w, 0, steps)
+    if tau is None:
+        tau = max(1, w.block_len // 4)
+    layer = CachedBlockAttention(
+        w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_len, w.capacity, dtype=w.dtype,
+        softmax_scale=w.softmax_scale, policy=policy, gamma=gamma, tau=tau, eps=eps)
+    layer.load_prefix(Kt, Vt, lens)
+    Qs, Kbs, Vbs, outs, masks, stats = [], [], [], [], [], []
+    for s, (Q, Kb, Vb) in enumerate(raw):
+        Qt, Q64 = tensors(w, Q)
+        Kbt, Kb64 = tensors(w, Kb)
+        Vbt, Vb64 = tensors(w, Vb)
+        outs.append(layer.cached_step(s, Qt, Kbt, Vbt).float().cpu().numpy())
+        masks.append(layer.unit_mask.cpu().numpy().astype(bool))
+        stats.append((layer.sim if policy == "headwise" else layer.updated).cpu().numpy())
+        Qs.append(Q64)
+        Kbs.append(Kb64)
+        Vbs.append(Vb64)
+    layer.check()
+    L64 = lens.astype(np.int64)
+    if policy == "headwise":
+        ref, ref_masks = ora.headwise_block(Qs, Kbs, Vbs, K64, V64, L64, w.softmax_scale, gamma)
+        # the similarity each decision was taken on, with the oracle's reference queries
+        Qref = Qs[0].copy()
+        G = w.group
+        for s in range(1, steps):
+            sim = ora.unit_query_similarity(Qs[s], Qref, w.num_kv_heads)
+            assert np.abs(sim - gamma).min() > margin, f"step {s}: a similarity is within {margin} of gamma"
+            np.testing.assert_allclose(stats[s], sim, atol=1e-4, err_msg=f"similarity at step {s}")
+            for b in range(w.batch):
+                for kvh in range(w.num_kv_heads):
+                    if ref_masks[s][b, kvh]:
+                        Qref[b, :, kvh * G:(kvh + 1) * G] = Qs[s][b, :, kvh * G:(kvh + 1) * G]
+        for s in range(steps):
+            assert np.array_equal(masks[s], ref_masks[s]), f"step {s}: refresh mask differs"
+    else:
+        ref, ref_flags = ora.threshold_block(Qs, Kbs, Vbs, K64, V64, L64, w.softmax_scale, tau, eps)
+        for s in range(1, steps):
+            dk = np.abs(Kbs[s] - Kbs[s - 1]).max(axis=(2, 3))
+            dv = np.abs(Vbs[s] - Vbs[s - 1]).max(axis=(2, 3))
+            assert np.abs(np.maximum(dk, dv) - eps).min() > margin, f"step {s}: a token change is near eps"
+            count = ora.updated_tokens(Kbs[s - 1], Vbs[s - 1], Kbs[s], Vbs[s], eps)
+            assert np.array_equal(stats[s], count), f"step {s}: updated-token counts differ"
+        for s in range(steps):
+            want = np.repeat(ref_flags[s][:, None], w.num_kv_heads, axis=1)
+            assert np.array_equal(masks[s], want), f"step {s}: refresh flags differ"
+    errs = [compare(f"{policy} O s{s}", outs[s], ref[s], w.dtype) for s in range(steps)]
+    return errs, masks

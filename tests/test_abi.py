@@ -77,5 +77,28 @@ def test_workspace_bytes_formula(lib):
     d = _desc(kv_capacity=131072, num_splits=5)
     # splits x rows x (D + 1) floats
     assert fbl.fb_workspace_bytes(d) == 5 * 32 * 32 * 129 * 4
-    assert fbl.fb_workspace_bytes(_desc(dtype=fbl.FB_FP32, head_dim=64)) == 0
+    # fp32 has no split partials: only the threshold policy's per-4-token counts
+    assert fbl.fb_workspace_bytes(_desc(dtype=fbl.FB_FP32, head_dim=64)) == 1 * 8 * 4
+    assert fbl.fb_workspace_bytes(_desc(dtype=fbl.FB_FP32, head_dim=64, batch=3, block_len=33)) == 3 * 9 * 4
     assert fbl.fb_cache_rows(_desc(page_size=256, max_pages=3, num_pages=9)) == 768
+
+
+def test_policy_validation_codes(lib):
+    d = _desc()
+    hw = lib.fb_headwise_refresh_mask
+    assert hw(ctypes.byref(d), None, FAKE, ctypes.c_float(0.9), FAKE, None, None) == 1
+    assert hw(ctypes.byref(d), FAKE, FAKE, ctypes.c_float(float("nan")), FAKE, None, None) == 1
+    assert hw(ctypes.byref(d), FAKE + 8, FAKE, ctypes.c_float(0.9), FAKE, None, None) == 3
+    assert hw(ctypes.byref(d), FAKE, FAKE, ctypes.c_float(0.9), FAKE + 2, None, None) == 3
+    th = lib.fb_threshold_refresh_mask
+    args = (FAKE, FAKE, FAKE, FAKE)
+    assert th(ctypes.byref(d), *args, ctypes.c_float(float("nan")), 1, FAKE, None, FAKE, 4096, None) == 1
+    assert th(ctypes.byref(d), *args, ctypes.c_float(0.25), 1, None, None, FAKE, 4096, None) == 1
+    assert th(ctypes.byref(d), FAKE + 4, FAKE, FAKE, FAKE, ctypes.c_float(0.25), 1, FAKE, None, FAKE, 4096,
+              None) == 3
+    assert th(ctypes.byref(d), *args, ctypes.c_float(0.25), 1, FAKE, None, None, 0, None) == 4
+    assert th(ctypes.byref(d), *args, ctypes.c_float(0.25), 1, FAKE, None, FAKE, 4, None) == 4  # needs 8 * 4
+    pm = lib.fb_prefix_partial_masked
+    assert pm(ctypes.byref(d), FAKE, FAKE, FAKE, None, None, FAKE, FAKE, None, 0, None, None) == 1
+    assert pm(ctypes.byref(d), FAKE, FAKE, FAKE, None, FAKE + 2, FAKE, FAKE, None, 0, None, None) == 3
+    assert pm(ctypes.byref(_desc(batch=0)), FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, 0, None, None) == 1
