@@ -203,10 +203,13 @@ bool q_map(CUtensorMap* m, const fb_desc& d, const void* Q) {
 }
 
 // Cached O_pre [B, S, Hq, D] f32 in the packed query-row order of a tile:
-// 32-float column blocks (128 B) of G heads x 128/G tokens.
-bool pre_map(CUtensorMap* m, const fb_desc& d, const float* O_pre) {
+// 32-float column blocks (128 B) of G heads x 128/G tokens; also the map the
+// prefix pass stores its partials through,
+// `outer` sequences of that layout (B, or splits x B for the split partials).
+bool pre_map(CUtensorMap* m, const fb_desc& d, const float* O_pre, int outer = 0) {
   const int G = d.num_q_heads / d.num_kv_heads;
-  const uint64_t D = d.head_dim, Hq = d.num_q_heads, S = d.block_len, B = d.batch;
+  const uint64_t D = d.head_dim, Hq = d.num_q_heads, S = d.block_len;
+  const uint64_t B = outer > 0 ? (uint64_t)outer : (uint64_t)d.batch;
   const uint64_t dims[4] = {D, Hq, S, B};
   const uint64_t str[3] = {D * 4, Hq * D * 4, S * Hq * D * 4};
   const uint32_t box[4] = {32, (uint32_t)G, (uint32_t)(TC_BM / G), 1};
@@ -299,8 +302,10 @@ fb_status prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const 
   }
   p.out_o32 = part_o;
   p.out_lse = part_l;
+  CUtensorMap tm_out;
+  if (!pre_map(&tm_out, *d, part_o, d->batch * ns)) return FB_ERR_LAUNCH;
   const long long grid = (long long)d->batch * d->num_kv_heads * p.n_rt * ns;
-  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kp, m.vp, m.q, (int)grid, s);
+  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kp, m.vp, m.q, tm_out, (int)grid, s);
   if (e != cudaSuccess || ns == 1) return from_cuda(e);
   CombineParams c;
   std::memset(&c, 0, sizeof(c));
@@ -385,12 +390,12 @@ fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const v
     return from_cuda(launch_attn_simt(p, static_cast<const float*>(Q), nullptr, nullptr,
                                       static_cast<const float*>(Kb), static_cast<const float*>(Vb), s));
   Maps m;
-  CUtensorMap tm_pre;
+  CUtensorMap tm_pre, tm_out;
   if (!q_map(&m.q, *d, Q) || !block_map(&m.kb, *d, Kb) || !block_map(&m.vb, *d, Vb) ||
-      !pre_map(&tm_pre, *d, O_pre))
+      !pre_map(&tm_pre, *d, O_pre) || !q_map(&tm_out, *d, O))
     return FB_ERR_LAUNCH;
   const long long grid = (long long)d->batch * d->num_kv_heads * p.n_rt;
-  return from_cuda(launch_attn_tc(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_pre, (int)grid, s));
+  return from_cuda(launch_attn_tc(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_pre, tm_out, (int)grid, s));
 }
 
 fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc, const void* Vc,
@@ -429,7 +434,9 @@ fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc,
     p.epi = EPI_NORM;
     p.out_o = O;
     p.out_lse = LSE_out;
-    return from_cuda(launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, (int)units, s));
+    CUtensorMap tm_out;
+    if (!q_map(&tm_out, dense, O)) return FB_ERR_LAUNCH;
+    return from_cuda(launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, tm_out, (int)units, s));
   }
   p.epi = EPI_PARTIAL;
   p.nsplit = ns;
@@ -437,7 +444,9 @@ fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc,
   float* part_l = part_o + (size_t)ns * d->batch * d->block_len * d->num_q_heads * d->head_dim;
   p.out_o32 = part_o;
   p.out_lse = part_l;
-  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, (int)(units * ns), s);
+  CUtensorMap tm_out;
+  if (!pre_map(&tm_out, dense, part_o, d->batch * ns)) return FB_ERR_LAUNCH;
+  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, tm_out, (int)(units * ns), s);
   if (e != cudaSuccess) return from_cuda(e);
   CombineParams c;
   std::memset(&c, 0, sizeof(c));

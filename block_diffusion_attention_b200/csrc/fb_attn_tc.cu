@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKp,
                    const __grid_constant__ CUtensorMap tmVp, const __grid_constant__ CUtensorMap tmKb,
                    const __grid_constant__ CUtensorMap tmVb, const __grid_constant__ CUtensorMap tmPre,
-                   const AttnParams p) {
+                   const __grid_constant__ CUtensorMap tmO, const AttnParams p) {
   static_assert(NC == 32 || NC == 64 || NC == 128, "column count");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -276,6 +276,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *sh.tmem_slot;
+  if (warp == 4 && lane == 0) {
+    // tensor maps are kernel parameters: fetch them while the previous kernel finishes
+    tma_prefetch_map(&tmQ);
+    tma_prefetch_map(&tmKp);
+    tma_prefetch_map(&tmVp);
+    tma_prefetch_map(&tmKb);
+    tma_prefetch_map(&tmVb);
+    tma_prefetch_map(&tmPre);
+    tma_prefetch_map(&tmO);
+  }
   // Everything above touches no global memory; from here on inputs may come
   // from the previous kernel in the stream.
   pdl_wait();
@@ -298,9 +308,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   } else if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      tma_prefetch_map(&tmQ);
-      tma_prefetch_map(&tmKp);
-      tma_prefetch_map(&tmVp);
       const uint64_t policy = p.kv_stream_once ? l2_policy_evict_first() : l2_policy_evict_normal();
       mbar_arrive_expect_tx(sh.q_full, Q_BYTES);
       const int t0 = rt * (BM / p.G);
@@ -584,18 +591,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
       for (int i = 0; i < HD; ++i) ov[i] = 0u;
     }
+    // The output tile is staged in ring slots 0-1 (every K/V tile has been
+    // consumed once the last PV is done; slots 4-5 may hold O_pre) in the
+    // 128-byte-swizzled packed-row layout of its tensor map, then written by
+    // one TMA store per 128-byte column block: coalesced, and rows past the
+    // block's last token are dropped by the copy.
+    uint8_t* stage = sRing;
+    const uint32_t st_row = smem_u32(stage) + r * 128;
     if (EPI == EPI_PARTIAL) {
-      const size_t orow = (((size_t)split * p.B + b) * p.S + tok) * p.Hq + h;
-      float* dst = p.out_o32 + orow * HD;
-      if (row_ok) {
+      if (ok) {
 #pragma unroll
-        for (int i = 0; i < HD; i += 4) {
-          const float4 v = make_float4(__uint_as_float(ov[i]) * inv_l, __uint_as_float(ov[i + 1]) * inv_l,
-                                       __uint_as_float(ov[i + 2]) * inv_l, __uint_as_float(ov[i + 3]) * inv_l);
-          *reinterpret_cast<float4*>(dst + i) = v;
-        }
-        p.out_lse[(((size_t)split * p.B + b) * p.Hq + h) * p.S + tok] = lse2 * LN2;
+        for (int c = 0; c < HD / 32; ++c)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const int i = c * 32 + ch * 4;
+            st_shared_v4(st_row + c * (BM * 128) + ((ch ^ (r & 7)) << 4),
+                         __float_as_uint(__uint_as_float(ov[i]) * inv_l),
+                         __float_as_uint(__uint_as_float(ov[i + 1]) * inv_l),
+                         __float_as_uint(__uint_as_float(ov[i + 2]) * inv_l),
+                         __float_as_uint(__uint_as_float(ov[i + 3]) * inv_l));
+          }
       }
+      if (row_ok) p.out_lse[(((size_t)split * p.B + b) * p.Hq + h) * p.S + tok] = lse2 * LN2;
     } else {
       const size_t orow = ((size_t)b * p.S + tok) * p.Hq + h;
       float wp = 0.f, wo = inv_l, inv_den = 1.f, lse_out2 = lse2;
@@ -611,7 +628,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         wo = empty ? 0.f : ex2_approx(m_run - Ms);  // = wi / l_run
         lse_out2 = den > 0.f ? Ms + log2f(den) : -CUDART_INF_F;
       }
-      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out_o) + orow * HD;
       const float* pre = (EPI == EPI_MERGE) ? p.pre_o + orow * HD : nullptr;
       if (row_ok) {
 #pragma unroll
@@ -631,15 +647,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               o[i + 3] = (o[i + 3] + wp * q.w) * inv_den;
             }
           }
+          // 32 columns = chunks (c & 1) * 4 .. + 3 of the 64-dim half c >> 1
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
-            uint4 v = make_uint4(pack_bf16x2(o[i], o[i + 1]), pack_bf16x2(o[i + 2], o[i + 3]),
-                                 pack_bf16x2(o[i + 4], o[i + 5]), pack_bf16x2(o[i + 6], o[i + 7]));
-            *reinterpret_cast<uint4*>(dst + c * 32 + i) = v;
+            const int ch = (c & 1) * 4 + (i >> 3);
+            st_shared_v4(st_row + (c >> 1) * (BM * 128) + ((ch ^ (r & 7)) << 4), pack_bf16x2(o[i], o[i + 1]),
+                         pack_bf16x2(o[i + 2], o[i + 3]), pack_bf16x2(o[i + 4], o[i + 5]),
+                         pack_bf16x2(o[i + 6], o[i + 7]));
           }
         }
         if (p.out_lse) p.out_lse[((size_t)b * p.Hq + h) * p.S + tok] = lse_out2 * LN2;
       }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1, 4 * 32);
+    if (r == 0 && !*sh.abort_flag) {
+      const int t0 = rt * (BM / p.G);
+      if (EPI == EPI_PARTIAL) {
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c)
+          tma_store_4d(&tmO, stage + c * (BM * 128), c * 32, kvh * p.G, t0, split * p.B + b);
+      } else {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) tma_store_4d(&tmO, stage + hf * (BM * 128), hf * 64, kvh * p.G, t0, b);
+      }
+      tma_store_commit();
+      tma_store_wait_read();
     }
   }
 
@@ -751,7 +784,7 @@ size_t tc_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
                            const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
-                           const CUtensorMap& tmPre, int grid, cudaStream_t stream) {
+                           const CUtensorMap& tmPre, const CUtensorMap& tmO, int grid, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -759,7 +792,8 @@ cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CU
   const bool short_block = (p.epi == EPI_MERGE) && !p.src.has_prefix;
   const int nc = (short_block && p.S <= 32) ? 32 : (short_block && p.S <= 64) ? 64 : 128;
   int which;
-  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, AttnParams);
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+               AttnParams);
   if (p.epi == EPI_PARTIAL) {
     kern = attn_tc_kernel<EPI_PARTIAL, 128>;
     which = 0;
@@ -787,7 +821,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CU
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tmQ, tmKp, tmVp, tmKb, tmVb, tmPre, p);
+  e = cudaLaunchKernelEx(&cfg, kern, tmQ, tmKp, tmVp, tmKb, tmVb, tmPre, tmO, p);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

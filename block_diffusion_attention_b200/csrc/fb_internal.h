@@ -75,7 +75,7 @@ constexpr int TC_MAX_SPLITS = 128;  // key-range splits per work unit
 size_t tc_smem_bytes();
 cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
                            const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
-                           const CUtensorMap& tmPre, int grid, cudaStream_t stream);
+                           const CUtensorMap& tmPre, const CUtensorMap& tmO, int grid, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& c, cudaStream_t stream);
 
 // CUDA-core (fp32) path.
