@@ -41,6 +41,15 @@ sys.path.insert(0, ROOT)
 
 METRIC = "attention µs/denoise-step and tokens/s, cached vs uncached; prefix-pass HBM GB/s"
 
+# DRAM bytes read + written by one launch of the prefix-pass attention kernel,
+# from one `ncu --set full --clock-control none` capture of that launch on the
+# workload (dram__bytes_read.sum + dram__bytes_write.sum).  An entry holds only
+# for the kernel source it was captured with: re-capture, or drop it, when the
+# kernel changes.
+NCU_TRAFFIC = {
+    "long_ctx": 537214208 + 3851008,
+}
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -512,7 +521,10 @@ def report(args, w0, w, world, res):
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_source": f"{peak_kind} hbm_gbs",
                 "tensor_tflops": tflops, "tensor_frac": tflops / tc_peak}
-    roof.update({"traffic": None, "kernel": "prefix pass: attn_tc_kernel<EPI_PARTIAL> (+ combine_kernel when split)",
+    traffic = None if args.residual else NCU_TRAFFIC.get(w.name)
+    roof.update({"traffic": traffic,
+                 "traffic_over_algorithmic": (traffic / abytes) if traffic else None,
+                 "kernel": "prefix pass: attn_tc_kernel<EPI_PARTIAL> (+ combine_kernel when split)",
                  "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": pflops,
                  "intensity_flop_per_byte": intensity})
     ms_c = res["ms_cached"]
