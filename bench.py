@@ -63,6 +63,11 @@ def parse():
                     help="sparse workloads: residual reuse (cache the unselected chunks, recompute the selected ones)")
     ap.add_argument("--no-graph", action="store_true",
                     help="issue every call from the host instead of replaying one CUDA graph per block")
+    ap.add_argument("--policy", choices=["headwise", "threshold"], default=None,
+                    help="adaptive reuse: decide per step which units refresh (dense workloads)")
+    ap.add_argument("--gamma", type=float, default=0.9, help="head-wise policy: similarity threshold")
+    ap.add_argument("--tau", type=int, default=None, help="threshold policy: updated-token count (default S/4)")
+    ap.add_argument("--eps", type=float, default=0.25, help="threshold policy: change that marks a token updated")
     ap.add_argument("--phases", default="cached,uncached,e2e",
                     help="comma list of timed phases (profiling runs may keep only 'cached')")
     return ap.parse_args()
@@ -294,10 +299,17 @@ def run_ours(args):
     Vt = synth.as_dtype(w, V)[0].cuda()
     del K, V
     base = synth.block_base(w, 0)
-    step_in = []
-    for s in range(w.steps):
-        Q, Kb, Vb = synth.step_inputs(w, 0, s, base)
-        step_in.append(tuple(synth.as_dtype(w, x)[0] for x in (Q, Kb, Vb)))
+    if args.policy is not None and (w.topk or args.residual):
+        raise SystemExit("--policy runs on the dense workloads")
+    tau = args.tau if args.tau is not None else max(1, w.block_len // 4)
+    if args.policy == "headwise":
+        raw = synth.headwise_steps(w, 0, w.steps, base=base)
+    elif args.policy == "threshold":
+        raw = synth.threshold_steps(w, 0, w.steps, base=base)
+    else:
+        raw = [synth.step_inputs(w, 0, s, base) for s in range(w.steps)]
+    step_in = [tuple(synth.as_dtype(w, x)[0] for x in t) for t in raw]
+    del raw
     dev_in = [tuple(x.cuda() for x in t) for t in step_in]
     outs = [torch.empty_like(dev_in[0][0]) for _ in range(w.steps)]
     stream = torch.cuda.current_stream()
@@ -306,9 +318,12 @@ def run_ours(args):
         layer = CachedBlockAttention(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_len, w.capacity,
                                      dtype=w.dtype, softmax_scale=w.softmax_scale,
                                      chunk_size=w.chunk_size if w.topk else 0, topk=w.topk,
-                                     residual=args.residual)
+                                     residual=args.residual, policy=policy, gamma=args.gamma, tau=tau,
+                                     eps=args.eps)
         layer.load_prefix(Kt, Vt, lens)
         return layer
+
+    policy = None
 
     def barrier():
         ranks.barrier()
@@ -338,22 +353,37 @@ def run_ours(args):
         return max_over_ranks(t0.elapsed_time(t1))
 
     # ---- cached (FlashBlock) path
+    policy = args.policy
     cached = new_layer()
-    nref = len(w.refresh)
+    nref = 1 if policy else len(w.refresh)
     use_graph = not args.no_graph
 
     def issue_block(pre_events=None):
-        """One block of calls; pre_events[i] = (start, end) around refresh i."""
+        """One block of calls; pre_events[i] = (select start, prefix start,
+        prefix end) around refresh i."""
         pi = 0
         for s in range(w.steps):
             Q, Kb, Vb = dev_in[s]
-            if s in w.refresh:
+            if policy:
+                # every step decides which units refresh; step 0 refreshes all
+                # of them (its mask + masked prefix pass is the timed pair)
+                if s == 0 and pre_events is not None:
+                    pre_events[0][0].record()
+                    pre_events[0][1].record()  # no separate selection step
+                    cached.adapt(Q, Kb, Vb, first=True)
+                    pre_events[0][2].record()
+                else:
+                    cached.adapt(Q, Kb, Vb, first=(s == 0))
+            elif s in w.refresh:
                 # current stream: the capture stream while a graph is recorded
                 if pre_events is not None:
                     pre_events[pi][0].record()
-                cached.refresh(Q)
+                cached.select(Q)
                 if pre_events is not None:
                     pre_events[pi][1].record()
+                cached.prefix(Q)
+                if pre_events is not None:
+                    pre_events[pi][2].record()
                 pi += 1
             cached.step(Q, Kb, Vb, out=outs[s])
         cached.append(dev_in[-1][1], dev_in[-1][2], advance=False)
@@ -370,8 +400,7 @@ def run_ours(args):
         # its own copy of the graph, whose external event nodes around the
         # prefix pass time that kernel on the GPU inside the timed region.
         def ev_pair():
-            return (torch.cuda.Event(enable_timing=True, external=True),
-                    torch.cuda.Event(enable_timing=True, external=True))
+            return tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(3))
 
         def capture(pre_events):
             g = torch.cuda.CUDAGraph()
@@ -388,15 +417,26 @@ def run_ours(args):
             (warm if k is None else graphs[k]).replay()
 
         res["ms_cached"] = timed(replay, cached)
-        res["pre_ms"] = [a.elapsed_time(b) for evs in ev_pre for a, b in evs]
+        res["pre_ms"] = [b.elapsed_time(c) for evs in ev_pre for a, b, c in evs]
+        res["sel_ms"] = [a.elapsed_time(b) for evs in ev_pre for a, b, c in evs]
         del graphs, warm
     else:
-        ev_pre = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        ev_pre = [[tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
                    for _ in range(nref)] for _ in range(args.steps)]
         res["ms_cached"] = timed(lambda k: issue_block(None if k is None else ev_pre[k]), cached)
-        res["pre_ms"] = [a.elapsed_time(b) for evs in ev_pre for a, b in evs]
+        res["pre_ms"] = [b.elapsed_time(c) for evs in ev_pre for a, b, c in evs]
+        res["sel_ms"] = [a.elapsed_time(b) for evs in ev_pre for a, b, c in evs]
     res["launches"] = int(res["launches_per_block"] * args.steps)
     res["lens1"] = [int(x) for x in cached.lens.cpu()]
+    if policy:
+        # share of the units the policy refreshes after the first step (one
+        # eager block after the timed region, the masks read at each step)
+        frac = []
+        for s, (Q, Kb, Vb) in enumerate(dev_in):
+            cached.cached_step(s, Q, Kb, Vb, out=outs[s])
+            if s > 0:
+                frac.append(float(cached.unit_mask.float().mean()))
+        res["refresh_fraction"] = sum(frac) / len(frac) if frac else None
     # block-step latency on its own: 64 back-to-back denoising steps in one graph
     reps = 64
     Q, Kb, Vb = dev_in[1 % w.steps]
@@ -472,9 +512,7 @@ def run_ours(args):
                 for s in range(w.steps):
                     copy_in(s)
                     Q, Kb, Vb = stage[s]
-                    if s in w.refresh:
-                        e2e_layer.refresh(Q)
-                    e2e_layer.step(Q, Kb, Vb, out=e2e_outs[s])
+                    e2e_layer.cached_step(s, Q, Kb, Vb, w.refresh, out=e2e_outs[s])
                     copy_out(s)
                 e2e_layer.append(stage[-1][1], stage[-1][2], advance=False)
             res["ms_e2e"] = timed(e2e_block, e2e_layer)
@@ -494,6 +532,8 @@ def run_ours(args):
 
 
 def report(args, w0, w, world, res):
+    policy = args.policy
+    tau = args.tau if args.tau is not None else max(1, w.block_len // 4)
     from block_diffusion_attention_b200 import synth
     tokens = world * w.batch * w.block_len * args.steps
 
@@ -537,7 +577,13 @@ def report(args, w0, w, world, res):
         "config": workload_config(w0, {"prefix_rows_during_timing": [min(res["lens0"]), max(res["lens1"])],
                                        **({"sparse_mode": "residual reuse (refresh caches the unselected "
                                                           "chunks; every step recomputes the selected ones)"}
-                                          if args.residual else {})}),
+                                          if args.residual else {}),
+                                       **({"policy": ({"name": "headwise", "gamma": args.gamma,
+                                                       "inputs": "per-unit query jumps (p = 0.35 per step)"}
+                                                      if policy == "headwise" else
+                                                      {"name": "threshold", "tau": tau, "eps": args.eps,
+                                                       "inputs": "per-sequence token updates, uniform in [0, S/2]"})}
+                                          if policy else {})}),
         "cached_us_per_denoise_step": ms_c * 1e3 / (args.steps * w.steps),
         "cached_eager_us_per_denoise_step": res["ms_cached_eager"] * 1e3 / (args.steps * w.steps),
         "launch_mode": "one CUDA graph per block" if res["graph"] else "eager host launches",
@@ -545,7 +591,9 @@ def report(args, w0, w, world, res):
         "uncached_tokens_per_s": tps(ms_u),
         "cached_over_uncached_speedup": (ms_u / ms_c) if ms_u else None,
         "prefix_pass_us": pre_avg * 1e3,
+        "chunk_select_us": (sum(res["sel_ms"]) / len(res["sel_ms"]) * 1e3) if w.topk else None,
         "block_step_us": blk_avg * 1e3,
+        "refresh_fraction": res.get("refresh_fraction"),
         "prefix_gbs": achieved,
         "roofline": roof,
         "clocks": res["clocks"],

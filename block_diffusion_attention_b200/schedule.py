@@ -129,23 +129,31 @@ class CachedBlockAttention:
 
     # ------------------------------------------------------------------ steps
     def refresh(self, Q: torch.Tensor) -> None:
-        """Refresh step: recompute the cached block-external pair with Q.
+        """Refresh step: recompute the cached block-external pair with Q
+        (``select`` then ``prefix``)."""
+        self.select(Q)
+        self.prefix(Q)
 
-        Residual mode: select the chunks, and cache the partial over the
-        chunks left out (the residual); the selected chunks are recomputed at
-        every step."""
-        idx = None
+    def select(self, Q: torch.Tensor) -> None:
+        """Sparse prefix: pick this refresh's chunks (and, in residual mode,
+        their complement).  Nothing to do for a dense prefix."""
         if self.topk > 0:
             fbl.fb_select_chunks(self.desc, Q, self.Kmean, self.chunk_idx, self.status)
-            idx = self.chunk_idx
         if self.residual:
             cap = self.comp_idx.shape[2]
             fbl.fb_complement_chunks(self.desc, self.chunk_idx, self.comp_idx, cap, self.status)
+
+    def prefix(self, Q: torch.Tensor) -> None:
+        """The prefix partial of a refresh (after ``select``): over the whole
+        prefix or the selected chunks into (O_pre, LSE_pre); in residual mode
+        over the chunks left out, into the cached residual (the selected
+        chunks are recomputed at every step)."""
+        if self.residual:
             fbl.fb_prefix_partial(self.desc_res, Q, self.K, self.V, self.comp_idx, self.O_res, self.LSE_res,
                                   self.workspace, self.status)
             return
-        fbl.fb_prefix_partial(self.desc, Q, self.K, self.V, idx, self.O_pre, self.LSE_pre,
-                              self.workspace, self.status)
+        fbl.fb_prefix_partial(self.desc, Q, self.K, self.V, self.chunk_idx if self.topk > 0 else None,
+                              self.O_pre, self.LSE_pre, self.workspace, self.status)
 
     def adapt(self, Q, Kblk, Vblk, first: bool) -> None:
         """Adaptive refresh (policy mode): decide per unit whether the cached

@@ -1,0 +1,66 @@
+"""bench.py's JSON line, built on the CPU from a synthetic record of timings:
+every key of the benchmark contract is present and the derived figures follow
+from the record (no GPU: the timed phases are not run)."""
+import argparse
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from block_diffusion_attention_b200 import synth  # noqa: E402
+
+
+def _args(**kw):
+    base = dict(gpus=1, steps=4, warmup=3, workload="long_ctx", impl="ours", no_cpu_baseline=True,
+                residual=False, no_graph=False, policy=None, gamma=0.9, tau=None, eps=0.25,
+                phases="cached,uncached,e2e")
+    base.update(kw)
+    return argparse.Namespace(**base)
+
+
+def _res(w, with_e2e=True, **kw):
+    res = {"pre_ms": [0.1, 0.1], "sel_ms": [0.02, 0.02], "blk_ms": [0.005], "lens0": [w.prefix_len] * w.batch,
+           "lens1": [w.prefix_len] * w.batch, "ms_cached": 0.6, "ms_cached_eager": 0.7, "ms_unc": 3.0,
+           "graph": True, "launches": 44, "clocks": {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}}
+    if with_e2e:
+        res.update({"ms_e2e": 1.2, "h2d": 1000, "d2h": 500})
+    res.update(kw)
+    return res
+
+
+@pytest.mark.parametrize("kw", [{}, {"policy": "headwise"}, {"policy": "threshold", "tau": 5},
+                                {"workload": "batched_sparse"}, {"workload": "batched_sparse", "residual": True}])
+def test_report_line_has_contract_keys(capsys, kw):
+    args = _args(**kw)
+    w = synth.WORKLOADS[args.workload].scaled(blocks=1)
+    bench.report(args, synth.WORKLOADS[args.workload], w, 1, _res(w, refresh_fraction=0.25))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in line, key
+    assert line["n_gpus"] == 1 and line["steps"] == 4 and line["higher_is_better"] is True
+    # value = B * S tokens per block over the timed blocks
+    assert line["value"] == pytest.approx(w.batch * w.block_len * 4 / 0.6e-3)
+    roof = line["roofline"]
+    assert roof["bound"] in ("hbm", "tensor") and roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"])
+    assert line["e2e"]["h2d_bytes_per_step"] == 1000 and line["e2e"]["d2h_bytes_per_step"] == 500
+    if args.policy:
+        assert line["config"]["policy"]["name"] == args.policy
+        assert line["refresh_fraction"] == 0.25
+    if args.workload == "batched_sparse":
+        assert line["chunk_select_us"] == pytest.approx(20.0)
+    if args.workload == "long_ctx" and not args.residual:
+        assert roof["traffic"] == bench.NCU_TRAFFIC["long_ctx"]
+
+
+def test_report_without_e2e_phase(capsys):
+    args = _args(phases="cached")
+    w = synth.WORKLOADS["long_ctx"].scaled(blocks=1)
+    bench.report(args, synth.WORKLOADS["long_ctx"], w, 1, _res(w, with_e2e=False, ms_unc=None))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["e2e"] is None and line["uncached_us_per_denoise_step"] is None
