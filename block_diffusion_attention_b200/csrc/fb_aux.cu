@@ -8,7 +8,8 @@
 //     qbar . kbar_c,
 // qbar the mean query of the block over its tokens and the G heads of the
 // group, kbar_c the mean key of chunk c over its valid rows.
-// Append (Technical Summary §1: KV caching with block-wise causal inference):
+// Append (Technical Summary §1: block diffusion keeps a KV cache of the blocks
+// already generated, each block causal with respect to the earlier ones):
 // a finalized block's K/V joins the prefix.
 #include <cuda_bf16.h>
 #include <math_constants.h>

@@ -217,8 +217,8 @@ fb_status fb_prefix_partial_masked(const fb_desc* d, const void* Q, const void* 
                                    const int32_t* unit_mask, float* O_pre, float* LSE_pre, void* ws,
                                    size_t ws_bytes, int32_t* dev_status, fb_stream_t stream);
 
-/* Block end ("KV caching with block-wise causal inference", Technical Summary
- * §1): copy the finalized block's K/V [B,S,Hkv,D] into cache rows
+/* Block end (Technical Summary §1: the KV cache of finished blocks, which
+ * later blocks attend to causally): copy the finalized block's K/V [B,S,Hkv,D] into cache rows
  * [L_b, L_b + S) (contiguous or paged).  When lens_inout is not NULL
  * (device [B]), it is read for L_b and then advanced by S.  A block that does
  * not fit records FB_ERR_BOUNDS in dev_status and is not written. */

@@ -27,7 +27,7 @@ Efficient Long-Context Block Diffusion" (gist.science explainer of arXiv
   "Head-wise Selection" -- refresh decisions by updated-token count tau and by
   per-head similarity gamma (:func:`threshold_block`, :func:`headwise_block`).
 
-Readings where the page is silent (each listed in the design doc):
+Readings where the page is silent:
   L is the natural log of the unnormalised sum Z; J_out is the finalized
   prefix; the block is attended bidirectionally with no mask; query head h
   reads KV head h // G; an empty key set gives (O = 0, L = -inf); the sparse
@@ -407,8 +407,9 @@ def updated_tokens(Kprev, Vprev, Know, Vnow, eps):
 
 def threshold_block(Qs, Kbs, Vbs, Kc, Vc, prefix_lens, scale, tau, eps):
     """Threshold-based reuse (Adaptive Reuse Strategies): step 0 refreshes;
-    at step s + 1 a sequence reuses its block-external pair if the number of
-    updated tokens M^{s+1} is below tau, else recomputes it.
+    at step s + 1 a sequence keeps its block-external pair while its count
+    M^{s+1} of tokens changed since step s stays under tau, and recomputes it
+    otherwise.
     Returns (list of O_s, list of per-sequence refresh flags [B])."""
     B, S, Hq, D = Qs[0].shape
     Op, Lp = prefix_partial(Qs[0], Kc, Vc, prefix_lens, scale)
