@@ -92,8 +92,30 @@ __global__ void chunk_means_kernel(const CacheGeom g, const int32_t* lens, int c
 }
 
 // grid (Hkv, B), block SEL_THREADS.  Dynamic shared memory:
-// (SEL_WARPS + 1) * D floats for the query mean, nch scores, nch flags.
+// SEL_PART_FLOATS + D floats for the query mean, nch scores, nch flags.
 constexpr int SEL_WARPS = 8, SEL_THREADS = SEL_WARPS * 32;
+constexpr int SEL_PART_FLOATS = SEL_THREADS * 8;  // row-group sums of the query mean (16-bit inputs)
+
+// Adds the eight bf16 or four f32 values of a 16-byte vector to acc.
+template <typename T>
+__device__ __forceinline__ void add_vec16(const uint4& v, float* acc);
+template <>
+__device__ __forceinline__ void add_vec16<__nv_bfloat16>(const uint4& v, float* acc) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __bfloat1622float2(h[i]);
+    acc[2 * i] += x.x;
+    acc[2 * i + 1] += x.y;
+  }
+}
+template <>
+__device__ __forceinline__ void add_vec16<float>(const uint4& v, float* acc) {
+  acc[0] += __uint_as_float(v.x);
+  acc[1] += __uint_as_float(v.y);
+  acc[2] += __uint_as_float(v.z);
+  acc[3] += __uint_as_float(v.w);
+}
 
 template <typename T>
 __global__ void __launch_bounds__(SEL_THREADS)
@@ -104,10 +126,16 @@ __global__ void __launch_bounds__(SEL_THREADS)
   const int kvh = blockIdx.x;
   const int b = blockIdx.y;
   const int G = Hq / g.Hkv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* part = sm;                       // [SEL_WARPS][D] per-warp row sums
-  float* qbar = sm + SEL_WARPS * g.D;     // [D]
-  float* score = qbar + g.D;              // [nch_total]
+  // query mean over the S block tokens and the G heads of the group: the
+  // unit's S x G rows of D values are read as 16-byte vectors, thread i taking
+  // vector i % vpr of rows i / vpr, i / vpr + rpi, ...; the rpi row sums of
+  // each column are then added in a fixed order
+  constexpr int VEC = 16 / sizeof(T);
+  const int vpr = g.D / VEC;                // vectors per row
+  const int rpi = SEL_THREADS / vpr;        // rows per iteration
+  float* part = sm;                         // [rpi][D] row-group sums
+  float* qbar = sm + SEL_PART_FLOATS;       // [D]
+  float* score = qbar + g.D;                // [nch_total]
   int* sel = reinterpret_cast<int*>(score + nch_total);
   int L = lens[b];
   if (L < 0 || L > g.cap) {
@@ -115,32 +143,50 @@ __global__ void __launch_bounds__(SEL_THREADS)
     L = max(0, min(L, g.cap));
   }
   const int nch = (L + chunk_size - 1) / chunk_size;
-  // query mean over the S block tokens and the G heads of the group: warp w
-  // sums rows w, w + SEL_WARPS, ...; lanes cover the D columns
   const int rows = S * G;
-  for (int d = lane; d < g.D; d += 32) {
-    float acc = 0.f;
-    for (int rr = warp; rr < rows; rr += SEL_WARPS) {
-      const int t = rr / G, gg = rr - (rr / G) * G;
-      acc += to_f<T>(Q[(((size_t)b * S + t) * Hq + kvh * G + gg) * g.D + d]);
+  {
+    const int vi = threadIdx.x % vpr, r0 = threadIdx.x / vpr;
+    if (r0 < rpi) {
+      float acc[VEC];
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
+#pragma unroll 4
+      for (int rr = r0; rr < rows; rr += rpi) {
+        const int t = rr / G, gg = rr - t * G;
+        const uint4 v =
+            *reinterpret_cast<const uint4*>(Q + (((size_t)b * S + t) * Hq + kvh * G + gg) * g.D + vi * VEC);
+        add_vec16<T>(v, acc);
+      }
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) part[r0 * g.D + vi * VEC + k] = acc[k];
     }
-    part[warp * g.D + d] = acc;
   }
   __syncthreads();
   for (int d = threadIdx.x; d < g.D; d += SEL_THREADS) {
     float acc = 0.f;
-    for (int w2 = 0; w2 < SEL_WARPS; ++w2) acc += part[w2 * g.D + d];
+    for (int w2 = 0; w2 < rpi; ++w2) acc += part[w2 * g.D + d];
     qbar[d] = acc / (float)rows;
   }
   __syncthreads();
-  // score of chunk c: one warp per chunk, lanes over D, shuffle reduction
+  // score of chunk c: four lanes per chunk, each over a quarter of D with
+  // 16-byte loads (all independent), then two shuffles
   const float* km = Kmean + ((size_t)b * g.Hkv + kvh) * nch_total * g.D;
-  for (int c = warp; c < nch; c += SEL_WARPS) {
+  const int q4 = threadIdx.x & 3, dq = g.D / 4;
+  for (int base = 0; base < nch; base += SEL_THREADS / 4) {
+    const int c = base + (threadIdx.x >> 2);
     float acc = 0.f;
-    for (int d = lane; d < g.D; d += 32) acc = fmaf(qbar[d], km[(size_t)c * g.D + d], acc);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) score[c] = acc;
+    if (c < nch) {
+      const float4* kr = reinterpret_cast<const float4*>(km + (size_t)c * g.D + q4 * dq);
+      const float4* qr = reinterpret_cast<const float4*>(qbar + q4 * dq);
+#pragma unroll 8
+      for (int i = 0; i < dq / 4; ++i) {
+        const float4 k = kr[i], q = qr[i];
+        acc = fmaf(q.x, k.x, fmaf(q.y, k.y, fmaf(q.z, k.z, fmaf(q.w, k.w, acc))));
+      }
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (q4 == 0 && c < nch) score[c] = acc;
   }
   __syncthreads();
   // rank = chunks that beat c (higher score, or equal score and lower index)
@@ -302,7 +348,7 @@ cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* K
                                  int32_t* status, cudaStream_t stream) {
   const CacheGeom g = geom_of(d);
   const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
-  const size_t smem = (size_t)((SEL_WARPS + 1) * g.D + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int);
+  const size_t smem = (size_t)(SEL_PART_FLOATS + g.D + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int);
   dim3 grid(g.Hkv, g.B);
   if (d.dtype == FB_BF16) {
     auto k = select_chunks_kernel<__nv_bfloat16>;
