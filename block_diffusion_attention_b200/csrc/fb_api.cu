@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -181,6 +182,13 @@ long long prefix_tiles_estimate(const fb_desc& d) {
   return (cache_rows(d) + TC_BN - 1) / TC_BN;
 }
 
+// The masked prefix pass shares its grid out among the selected units (one
+// slot of 128 partial rows per CTA) when the full pass fills at most two
+// waves: there, dropping units would not shorten the pass.
+bool use_active_split(const fb_desc& d, long long grid) { return grid <= 2LL * device_sms(); }
+
+size_t active_split_bytes(long long grid) { return (size_t)grid * TC_BM * (TC_D + 1) * sizeof(float); }
+
 size_t split_bytes(const fb_desc& d, int ns) {
   if (ns <= 1) return 0;
   const size_t rows = (size_t)d.batch * d.block_len * d.num_q_heads;
@@ -214,6 +222,17 @@ bool pre_map(CUtensorMap* m, const fb_desc& d, const float* O_pre, int outer = 0
   const uint64_t str[3] = {D * 4, Hq * D * 4, S * Hq * D * 4};
   const uint32_t box[4] = {32, (uint32_t)G, (uint32_t)(TC_BM / G), 1};
   return make_map(m, O_pre, dims, str, box, true);
+}
+
+// Active-unit split partials: `slots` blocks of 128 packed rows x D f32, in
+// the same 32-float column boxes as pre_map.
+bool slot_map(CUtensorMap* m, const fb_desc& d, const float* base, int slots) {
+  const int G = d.num_q_heads / d.num_kv_heads;
+  const uint64_t D = d.head_dim;
+  const uint64_t dims[4] = {D, (uint64_t)G, (uint64_t)(TC_BM / G), (uint64_t)slots};
+  const uint64_t str[3] = {D * 4, (uint64_t)G * D * 4, (uint64_t)TC_BM * D * 4};
+  const uint32_t box[4] = {32, (uint32_t)G, (uint32_t)(TC_BM / G), 1};
+  return make_map(m, base, dims, str, box, true);
 }
 
 bool block_map(CUtensorMap* m, const fb_desc& d, const void* X) {
@@ -255,9 +274,15 @@ size_t fb_workspace_bytes(const fb_desc* d) {
   fb_desc dense = *d;
   dense.topk = 0;
   const int ns_full = choose_splits(dense, prefix_tiles_estimate(dense) + (d->block_len + TC_BN - 1) / TC_BN);
-  const size_t a = split_bytes(*d, ns_pre), b = split_bytes(*d, ns_full);
-  const size_t c = threshold_ws_bytes(*d);
-  return a > b ? (a > c ? a : c) : (b > c ? b : c);
+  size_t need = split_bytes(*d, ns_pre);
+  need = std::max(need, split_bytes(*d, ns_full));
+  need = std::max(need, threshold_ws_bytes(*d));
+  if (d->dtype == FB_BF16) {
+    // the masked prefix pass's active-unit slots
+    const long long grid = (long long)d->batch * d->num_kv_heads * ((d->block_len * (d->num_q_heads / d->num_kv_heads) + TC_BM - 1) / TC_BM) * ns_pre;
+    if (use_active_split(*d, grid)) need = std::max(need, active_split_bytes(grid));
+  }
+  return need;
 }
 
 }  // extern "C"
@@ -288,11 +313,41 @@ fb_status prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const 
                                       static_cast<const float*>(Vc), nullptr, nullptr, s));
   }
   const int ns = choose_splits(*d, prefix_tiles_estimate(*d));
-  const size_t need = split_bytes(*d, ns);
+  const long long grid = (long long)d->batch * d->num_kv_heads * p.n_rt * ns;
+  const bool active = unit_mask != nullptr && use_active_split(*d, grid);
+  const size_t need = active ? active_split_bytes(grid) : split_bytes(*d, ns);
   if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return FB_ERR_WORKSPACE;
   Maps m;
   if (!q_map(&m.q, *d, Q) || !cache_map(&m.kp, *d, Kc) || !cache_map(&m.vp, *d, Vc))
     return FB_ERR_LAUNCH;
+  if (active) {
+    // partials in per-CTA slots, merged per active unit by the combine
+    float* part_o = static_cast<float*>(ws);
+    float* part_l = part_o + (size_t)grid * TC_BM * TC_D;
+    p.dyn = 1;
+    p.out_o32 = part_o;
+    p.out_lse = part_l;
+    CUtensorMap tm_out;
+    if (!slot_map(&tm_out, *d, part_o, (int)grid)) return FB_ERR_LAUNCH;
+    cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kp, m.vp, m.q, tm_out, (int)grid, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    CombineParams c;
+    std::memset(&c, 0, sizeof(c));
+    c.B = d->batch;
+    c.Hq = d->num_q_heads;
+    c.S = d->block_len;
+    c.D = d->head_dim;
+    c.part_o = part_o;
+    c.part_lse = part_l;
+    c.out_o32 = O_pre;
+    c.out_lse = LSE_pre;
+    c.G = p.G;
+    c.unit_mask = unit_mask;
+    c.dyn = 1;
+    c.grid = (int)grid;
+    c.n_rt = p.n_rt;
+    return from_cuda(launch_combine(c, s));
+  }
   p.nsplit = ns;
   float* part_o = O_pre;
   float* part_l = LSE_pre;
@@ -304,7 +359,6 @@ fb_status prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const 
   p.out_lse = part_l;
   CUtensorMap tm_out;
   if (!pre_map(&tm_out, *d, part_o, d->batch * ns)) return FB_ERR_LAUNCH;
-  const long long grid = (long long)d->batch * d->num_kv_heads * p.n_rt * ns;
   cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kp, m.vp, m.q, tm_out, (int)grid, s);
   if (e != cudaSuccess || ns == 1) return from_cuda(e);
   CombineParams c;

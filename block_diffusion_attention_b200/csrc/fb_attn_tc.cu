@@ -243,13 +243,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  int bid = blockIdx.x;
-  const int split = bid % p.nsplit;
-  bid /= p.nsplit;
-  const int rt = bid % p.n_rt;
-  bid /= p.n_rt;
-  const int kvh = bid % p.Hkv;
-  const int b = bid / p.Hkv;
 
   if (threadIdx.x == 0) {
     mbar_init(sh.q_full, 1);
@@ -291,12 +284,37 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   pdl_wait();
   pdl_launch_dependents();
 
-  // a unit the refresh mask leaves out keeps its cached outputs: no work
-  const bool skip = p.unit_mask != nullptr && p.unit_mask[b * p.Hkv + kvh] == 0;
+  // This CTA's (b, kv head, query tile, key split).  A unit the refresh mask
+  // leaves out keeps its cached outputs: no work.  In the active-unit split
+  // the grid is shared out among the selected units only (the mask is written
+  // by the previous kernel, so this comes after the dependency wait).
+  int b, kvh, rt, split, nsplit;
+  bool skip;
+  if (p.dyn) {
+    const int na = active_count(p.unit_mask, p.B * p.Hkv);
+    nsplit = active_splits(gridDim.x, na, p.n_rt);
+    const int a = blockIdx.x / (p.n_rt * nsplit);
+    const int un = a < na ? active_unit(p.unit_mask, p.B * p.Hkv, a) : -1;
+    skip = un < 0;
+    b = skip ? 0 : un / p.Hkv;
+    kvh = skip ? 0 : un % p.Hkv;
+    rt = (blockIdx.x / nsplit) % p.n_rt;
+    split = blockIdx.x % nsplit;
+  } else {
+    int bid = blockIdx.x;
+    nsplit = p.nsplit;
+    split = bid % nsplit;
+    bid /= nsplit;
+    rt = bid % p.n_rt;
+    bid /= p.n_rt;
+    kvh = bid % p.Hkv;
+    b = bid / p.Hkv;
+    skip = p.unit_mask != nullptr && p.unit_mask[b * p.Hkv + kvh] == 0;
+  }
   const UnitTiles u = skip ? UnitTiles{0, 0, 0} : unit_tiles(p, b, kvh, threadIdx.x == 0);
   const int ntot = u.n0 + u.n1;
-  const int j0 = (int)(((long long)split * ntot) / p.nsplit);
-  const int j1 = (int)(((long long)(split + 1) * ntot) / p.nsplit);
+  const int j0 = (int)(((long long)split * ntot) / nsplit);
+  const int j1 = (int)(((long long)(split + 1) * ntot) / nsplit);
   const int nt = j1 - j0;
   int32_t* status = p.dev_status;
   // The merge epilogue of a unit with at most two key tiles leaves the last
@@ -612,7 +630,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                          __float_as_uint(__uint_as_float(ov[i + 3]) * inv_l));
           }
       }
-      if (row_ok) p.out_lse[(((size_t)split * p.B + b) * p.Hq + h) * p.S + tok] = lse2 * LN2;
+      if (p.dyn) {
+        if (ok) p.out_lse[(size_t)blockIdx.x * BM + r] = lse2 * LN2;  // slot layout: every row
+      } else if (row_ok) {
+        p.out_lse[(((size_t)split * p.B + b) * p.Hq + h) * p.S + tok] = lse2 * LN2;
+      }
     } else {
       const size_t orow = ((size_t)b * p.S + tok) * p.Hq + h;
       float wp = 0.f, wo = inv_l, inv_den = 1.f, lse_out2 = lse2;
@@ -666,7 +688,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (EPI == EPI_PARTIAL) {
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c)
-          tma_store_4d(&tmO, stage + c * (BM * 128), c * 32, kvh * p.G, t0, split * p.B + b);
+          tma_store_4d(&tmO, stage + c * (BM * 128), c * 32, p.dyn ? 0 : kvh * p.G, p.dyn ? 0 : t0,
+                       p.dyn ? (int)blockIdx.x : split * p.B + b);
       } else {
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) tma_store_4d(&tmO, stage + hf * (BM * 128), hf * 64, kvh * p.G, t0, b);
@@ -715,10 +738,26 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombinePa
   const long long bt = row / c.Hq;
   const int t = (int)(bt % c.S);
   const int b = (int)(bt / c.S);
-  const size_t so = (size_t)nrows * c.D;              // split stride of the partial O
-  const size_t sl = (size_t)c.B * c.Hq * c.S;         // split stride of the partial LSE
+  size_t so = (size_t)nrows * c.D;              // split stride of the partial O
+  size_t sl = (size_t)c.B * c.Hq * c.S;         // split stride of the partial LSE
   const size_t lrow = ((size_t)b * c.Hq + h) * c.S + t;
-  if (c.unit_mask && c.unit_mask[b * (c.Hq / c.G) + h / c.G] == 0) return;  // unit not refreshed
+  const int unit = b * (c.Hq / c.G) + h / c.G;
+  if (c.unit_mask && c.unit_mask[unit] == 0) return;  // unit not refreshed
+  int nsplit = c.nsplit;
+  const float* base = c.part_o + row * c.D;
+  const float* lbase = c.part_lse + lrow;
+  if (c.dyn) {
+    // active-unit slots: (rank of the unit, query tile, split) -> [128][D] rows
+    const int na = active_count(c.unit_mask, c.B * (c.Hq / c.G));
+    const int a = active_rank(c.unit_mask, unit);
+    nsplit = active_splits(c.grid, na, c.n_rt);
+    const int pr = t * c.G + h % c.G;  // packed query row of the unit
+    const size_t slot0 = ((size_t)a * c.n_rt + pr / TC_BM) * nsplit;
+    base = c.part_o + (slot0 * TC_BM + pr % TC_BM) * c.D;
+    lbase = c.part_lse + slot0 * TC_BM + pr % TC_BM;
+    so = (size_t)TC_BM * c.D;
+    sl = TC_BM;
+  }
   // lane l holds the LSE (then the weight) of splits l, l + 32, l + 64, l + 96
   constexpr int PER_LANE = TC_MAX_SPLITS / 32;
   float wreg[PER_LANE];
@@ -726,7 +765,7 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombinePa
 #pragma unroll
   for (int k = 0; k < PER_LANE; ++k) {
     const int s = lane + 32 * k;
-    wreg[k] = s < c.nsplit ? c.part_lse[s * sl + lrow] : -CUDART_INF_F;
+    wreg[k] = s < nsplit ? lbase[s * sl] : -CUDART_INF_F;
     M = fmaxf(M, wreg[k]);
   }
   M = warp_max_f(M);
@@ -739,22 +778,21 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombinePa
   }
   den = warp_sum_f(den);
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  const float* base = c.part_o + row * c.D;
   for (int d0 = lane * 4; d0 < c.D; d0 += 128) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     // CMB_INFLIGHT splits' loads in flight at once, then the weighted sum in
     // split order
-    for (int s0 = 0; s0 < c.nsplit; s0 += CMB_INFLIGHT) {
+    for (int s0 = 0; s0 < nsplit; s0 += CMB_INFLIGHT) {
       float4 v[CMB_INFLIGHT];
 #pragma unroll
       for (int i = 0; i < CMB_INFLIGHT; ++i)
-        if (s0 + i < c.nsplit) v[i] = __ldg(reinterpret_cast<const float4*>(base + (s0 + i) * so + d0));
+        if (s0 + i < nsplit) v[i] = __ldg(reinterpret_cast<const float4*>(base + (s0 + i) * so + d0));
       const int k = s0 >> 5;  // the same for the whole batch (CMB_INFLIGHT divides 32)
       const float wk = k == 0 ? wreg[0] : k == 1 ? wreg[1] : k == 2 ? wreg[2] : wreg[3];
 #pragma unroll
       for (int i = 0; i < CMB_INFLIGHT; ++i) {
         const float w = __shfl_sync(0xffffffffu, wk, (s0 + i) & 31);
-        if (s0 + i < c.nsplit) {
+        if (s0 + i < nsplit) {
           acc.x = fmaf(w, v[i].x, acc.x);
           acc.y = fmaf(w, v[i].y, acc.y);
           acc.z = fmaf(w, v[i].z, acc.z);

@@ -43,6 +43,10 @@ struct AttnParams {
   int epi;
   int kv_stream_once;  // 1: prefix K/V is read once (evict-first L2 hint)
   const int32_t* unit_mask;  // [B, Hkv] or null: units with 0 are skipped (their outputs kept)
+  // 1: the grid's CTAs are shared out among the units unit_mask selects
+  // (active-unit split, EPI_PARTIAL only): CTA i writes its partial rows to
+  // slot i of out_o32 ([grid][128][D]) and out_lse ([grid][128])
+  int dyn;
   KeySource src;
   // outputs
   float* out_o32;         // EPI_PARTIAL: [nsplit][B][S][Hq][D]
@@ -57,6 +61,8 @@ struct CombineParams {
   int B, Hq, S, D, nsplit;
   int G;                  // query heads per kv head (for unit_mask)
   const int32_t* unit_mask;  // [B, Hkv] or null: rows of units with 0 are left as they are
+  int dyn;                // partials in the active-unit slot layout of AttnParams::dyn
+  int grid, n_rt;         // (dyn) the attention launch's CTAs and query tiles per unit
   const float* part_o;    // [nsplit][B][S][Hq][D]
   const float* part_lse;  // [nsplit][B][Hq][S]
   float* out_o32;         // f32 output (prefix pass) or null
@@ -73,6 +79,45 @@ constexpr int TC_SLOTS = 6;     // K/V ring: 32 KB slots (K and V of a tile take
 constexpr int TC_THREADS = 192; // 4 softmax warps + TMA warp + MMA warp
 constexpr int TC_MAX_SPLITS = 128;  // key-range splits per work unit
 size_t tc_smem_bytes();
+// ---- active-unit split plan (shared by the attention kernel and the combine)
+// Every lane of the calling warp must take part (warp ballots over the mask).
+__device__ __forceinline__ int active_count(const int32_t* mask, int nu) {
+  const int lane = threadIdx.x & 31;
+  int n = 0;
+  for (int i0 = 0; i0 < nu; i0 += 32)
+    n += __popc(__ballot_sync(0xffffffffu, i0 + lane < nu && mask[i0 + lane] != 0));
+  return n;
+}
+// Number of active units before unit u.
+__device__ __forceinline__ int active_rank(const int32_t* mask, int u) {
+  const int lane = threadIdx.x & 31;
+  int n = 0;
+  for (int i0 = 0; i0 < u; i0 += 32)
+    n += __popc(__ballot_sync(0xffffffffu, i0 + lane < u && mask[i0 + lane] != 0));
+  return n;
+}
+// Index of the a-th active unit (0-based), or -1.
+__device__ __forceinline__ int active_unit(const int32_t* mask, int nu, int a) {
+  const int lane = threadIdx.x & 31;
+  int base = 0;
+  for (int i0 = 0; i0 < nu; i0 += 32) {
+    unsigned m = __ballot_sync(0xffffffffu, i0 + lane < nu && mask[i0 + lane] != 0);
+    const int c = __popc(m);
+    if (a < base + c) {
+      for (int k = a - base; k > 0; --k) m &= m - 1;  // drop the lower set bits
+      return i0 + __ffs(m) - 1;
+    }
+    base += c;
+  }
+  return -1;
+}
+// Key splits per (active unit, query tile) when `grid` CTAs are shared out.
+__device__ __forceinline__ int active_splits(int grid, int n_active, int n_rt) {
+  if (n_active <= 0) return 1;
+  const int ns = grid / (n_active * n_rt);
+  return ns < 1 ? 1 : (ns > TC_MAX_SPLITS ? TC_MAX_SPLITS : ns);
+}
+
 cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
                            const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
                            const CUtensorMap& tmPre, const CUtensorMap& tmO, int grid, cudaStream_t stream);

@@ -47,3 +47,48 @@ def test_threshold_extremes_bf16():
     assert all(m.all() for m in masks)
     _, masks = run_policy(W_BF16, "threshold", steps=3, tau=W_BF16.block_len + 1)
     assert not any(m.any() for m in masks[1:])
+
+
+@pytest.mark.parametrize("num_splits", [0, 5])
+def test_masked_prefix_pass_random_masks(num_splits):
+    """fb_prefix_partial_masked against the oracle's prefix partial: the rows
+    of selected units are recomputed, the others are left untouched (also
+    when the grid is shared out among the selected units only)."""
+    import torch
+    from block_diffusion_attention_b200 import flashblock as fbl
+    from gpu_cases import compare, make_layer, tensors
+    from oracle import flashblock_oracle as ora
+
+    w = synth.WORKLOADS["lm_gqa"].scaled(batch=2, prefix_len=5000, blocks=1)
+    K, V, lens = synth.prefix_kv(w)
+    Kt, K64 = tensors(w, K)
+    Vt, V64 = tensors(w, V)
+    layer = make_layer(w, num_splits=num_splits)
+    layer.load_prefix(Kt, Vt, lens)
+    Q, _, _ = synth.step_inputs(w, 0, 0)
+    Qt, Q64 = tensors(w, Q)
+    ref_o, ref_l = ora.prefix_partial(Q64, K64, V64, lens.astype(np.int64), w.softmax_scale)
+    rng = np.random.default_rng(7)
+    masks = [np.ones((w.batch, w.num_kv_heads), np.int32), np.zeros((w.batch, w.num_kv_heads), np.int32),
+             (rng.random((w.batch, w.num_kv_heads)) < 0.3).astype(np.int32)]
+    one = np.zeros((w.batch, w.num_kv_heads), np.int32)
+    one[1, 5] = 1
+    masks.append(one)
+    G = w.group
+    for mk in masks:
+        mask = torch.from_numpy(mk).cuda()
+        layer.O_pre.fill_(7.0)
+        layer.LSE_pre.fill_(3.0)
+        fbl.fb_prefix_partial_masked(layer.desc, Qt, layer.K, layer.V, None, mask, layer.O_pre, layer.LSE_pre,
+                                     layer.workspace, layer.status)
+        layer.check()
+        O = layer.O_pre.cpu().numpy()
+        L = layer.LSE_pre.cpu().numpy()
+        for b in range(w.batch):
+            for kvh in range(w.num_kv_heads):
+                hs = slice(kvh * G, (kvh + 1) * G)
+                if mk[b, kvh]:
+                    compare(f"O_pre b{b} kvh{kvh}", O[b, :, hs], ref_o[b, :, hs], w.dtype)
+                    compare(f"LSE_pre b{b} kvh{kvh}", L[b, hs], ref_l[b, hs], w.dtype)
+                else:
+                    assert np.all(O[b, :, hs] == 7.0) and np.all(L[b, hs] == 3.0), f"unit {b},{kvh} was written"
