@@ -98,6 +98,14 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const S
   }
 }
 
+// wait_bar for a whole warp: every lane waits, then the warp agrees on the
+// outcome (a time-out seen by one lane ends the wait for all), so the warp
+// collectives that follow never meet a split warp.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, const Shared& sh,
+                                              int32_t* status) {
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, sh, status));
+}
+
 struct UnitTiles {
   int n0;  // prefix tiles
   int n1;  // block tiles
@@ -118,20 +126,34 @@ __device__ UnitTiles unit_tiles(const AttnParams& p, int b, int kvh, bool rep) {
     }
     u.L = L;
     if (s.chunk_idx) {
+      // 32 list entries per step, one per lane (the calling warp is
+      // converged): the list ends at its first entry that is -1, not above
+      // its predecessor or past the valid prefix (the last two are reported)
       const int32_t* idx = s.chunk_idx + ((size_t)b * p.Hkv + kvh) * s.topk;
       const int nch = (L + s.chunk_size - 1) / s.chunk_size;
+      const int lane = threadIdx.x & 31;
       int n = 0, prev = -1;
-      for (int i = 0; i < s.topk; ++i) {
-        const int c = idx[i];
-        if (c < 0) break;
-        if (c <= prev || c >= nch) {
-          if (rep) report(p.dev_status, FB_ERR_BOUNDS);
-          break;
+      for (int i0 = 0; i0 < s.topk; i0 += 32) {
+        const int i = i0 + lane;
+        const int c = i < s.topk ? idx[i] : -1;
+        int cp = __shfl_up_sync(0xffffffffu, c, 1);
+        if (lane == 0) cp = prev;
+        const bool bad = c >= 0 && (c <= cp || c >= nch);
+        // (every lane takes part in both ballots)
+        const unsigned stops = __ballot_sync(0xffffffffu, c < 0 || bad);
+        const unsigned bads = __ballot_sync(0xffffffffu, bad);
+        const int first = stops ? __ffs(stops) - 1 : 32;  // entries below it are valid
+        if (rep && first < 32 && ((bads >> first) & 1u)) report(p.dev_status, FB_ERR_BOUNDS);
+        int tiles = 0;
+        if (lane < first) {
+          const int lo = c * s.chunk_size;
+          tiles = (min(lo + s.chunk_size, L) - lo + BN - 1) / BN;
         }
-        const int lo = c * s.chunk_size;
-        const int hi = min(lo + s.chunk_size, L);
-        n += (hi - lo + BN - 1) / BN;
-        prev = c;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
+        n += tiles;
+        if (stops) break;
+        prev = __shfl_sync(0xffffffffu, c, 31);
       }
       u.n0 = n;
     } else {
@@ -279,16 +301,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tma_prefetch_map(&tmPre);
     tma_prefetch_map(&tmO);
   }
+  // This CTA's (b, kv head, query tile, key split) from its grid index, and
+  // the key-tile count of a unit that has no prefix (the in-block step):
+  // kernel parameters only, so they are worked out while the previous kernel
+  // finishes.
+  int b = 0, kvh = 0, rt = 0, split = 0, nsplit = p.nsplit;
+  if (!p.dyn) {
+    unsigned bid = blockIdx.x;
+    split = (int)(bid % (unsigned)nsplit);
+    bid /= (unsigned)nsplit;
+    rt = (int)(bid % (unsigned)p.n_rt);
+    bid /= (unsigned)p.n_rt;
+    kvh = (int)(bid % (unsigned)p.Hkv);
+    b = (int)(bid / (unsigned)p.Hkv);
+  }
+  UnitTiles u = p.src.has_prefix ? UnitTiles{0, 0, 0} : unit_tiles(p, b, kvh, false);
+
   // Everything above touches no global memory; from here on inputs may come
   // from the previous kernel in the stream.
   pdl_wait();
   pdl_launch_dependents();
 
-  // This CTA's (b, kv head, query tile, key split).  A unit the refresh mask
-  // leaves out keeps its cached outputs: no work.  In the active-unit split
-  // the grid is shared out among the selected units only (the mask is written
-  // by the previous kernel, so this comes after the dependency wait).
-  int b, kvh, rt, split, nsplit;
+  // A unit the refresh mask leaves out keeps its cached outputs: no work.  In
+  // the active-unit split the grid is shared out among the selected units
+  // only.  The mask, the prefix lengths and the chunk lists may be written by
+  // the previous kernel, so they are read after the dependency wait.
   bool skip;
   if (p.dyn) {
     const int na = active_count(p.unit_mask, p.B * p.Hkv);
@@ -301,20 +338,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     rt = (blockIdx.x / nsplit) % p.n_rt;
     split = blockIdx.x % nsplit;
   } else {
-    int bid = blockIdx.x;
-    nsplit = p.nsplit;
-    split = bid % nsplit;
-    bid /= nsplit;
-    rt = bid % p.n_rt;
-    bid /= p.n_rt;
-    kvh = bid % p.Hkv;
-    b = bid / p.Hkv;
     skip = p.unit_mask != nullptr && p.unit_mask[b * p.Hkv + kvh] == 0;
   }
-  const UnitTiles u = skip ? UnitTiles{0, 0, 0} : unit_tiles(p, b, kvh, threadIdx.x == 0);
+  if (skip)
+    u = UnitTiles{0, 0, 0};
+  else if (p.src.has_prefix)
+    u = unit_tiles(p, b, kvh, threadIdx.x == 0);
   const int ntot = u.n0 + u.n1;
-  const int j0 = (int)(((long long)split * ntot) / nsplit);
-  const int j1 = (int)(((long long)(split + 1) * ntot) / nsplit);
+  // split * ntot < 2^7 * 2^23: 32-bit arithmetic is exact
+  const int j0 = (int)(((unsigned)split * (unsigned)ntot) / (unsigned)nsplit);
+  const int j1 = (int)(((unsigned)(split + 1) * (unsigned)ntot) / (unsigned)nsplit);
   const int nt = j1 - j0;
   int32_t* status = p.dev_status;
   // The merge epilogue of a unit with at most two key tiles leaves the last
@@ -401,10 +434,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // and tile j + 1 located before QK^T(j + 1) is issued.  (This warp shares
     // its scheduler with a softmax warp, so every instruction on that path
     // delays the tensor pipe.)
-    bool ok = wait_bar(sh.q_tmem, 0, sh, status);
+    bool ok = wait_bar_warp(sh.q_tmem, 0, sh, status);
     if (ok && nt > 0) {
       Tile tc = tile_at(p, u, b, kvh, j0);
-      ok = wait_bar(&sh.full[slot_of(0)], 0, sh, status);
+      ok = wait_bar_warp(&sh.full[slot_of(0)], 0, sh, status);
       if (ok) {
         tc_fence_after_sync();
         if (lane == 0) {
@@ -416,7 +449,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       for (int jj = 0; ok && jj < nt; ++jj) {
         const int iv = 2 * jj + 1;
-        if (!(ok = wait_bar(&sh.full[slot_of(iv)], use_of(iv) & 1, sh, status))) break;
+        if (!(ok = wait_bar_warp(&sh.full[slot_of(iv)], use_of(iv) & 1, sh, status))) break;
         if (tc.seg == 0 && (tc.nvalid & 15)) {
           // Cache rows past the prefix may hold anything (even NaN); P is 0
           // there but 0 * NaN is not, so clear the V rows up to the next
@@ -436,7 +469,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (jj + 1 < nt) {
           tn = tile_at(p, u, b, kvh, j0 + jj + 1);
           const int ik = 2 * (jj + 1);
-          if (!(ok = wait_bar(&sh.full[slot_of(ik)], use_of(ik) & 1, sh, status))) break;
+          if (!(ok = wait_bar_warp(&sh.full[slot_of(ik)], use_of(ik) & 1, sh, status))) break;
           tc_fence_after_sync();
           if (lane == 0) {
             issue_qk(jj + 1, tn.nvalid);
@@ -444,7 +477,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tc_commit(&sh.empty[slot_of(ik)]);
           }
         }
-        if (!(ok = wait_bar(&sh.p_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
+        if (!(ok = wait_bar_warp(&sh.p_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
         tc_fence_after_sync();
         if (lane == 0) {
           issue_pv(jj, tc.nvalid);
@@ -473,7 +506,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                                           : -CUDART_INF_F;
     float m_run = -CUDART_INF_F;
     float l_run = 0.f;
-    bool ok = wait_bar(sh.q_full, 0, sh, status);
+    bool ok = wait_bar_warp(sh.q_full, 0, sh, status);
     if (ok) {
       // this thread's Q row (128 bf16, 128-byte swizzled in two 64-dim halves)
       // into TMEM columns [TMEM_Q, TMEM_Q + 64): the A operand of QK^T
@@ -498,7 +531,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (int jj = 0; ok && jj < nt; ++jj) {
       const uint32_t tS = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN + lane_off;
       const Tile t = tile_at(p, u, b, kvh, j0 + jj);
-      if (!(ok = wait_bar(&sh.s_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
+      if (!(ok = wait_bar_warp(&sh.s_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
       tc_fence_after_sync();
       // S row of this thread.  A tail tile (fewer than BN valid keys) sets
       // the columns past its keys to -inf first; full tiles skip that block.
@@ -553,7 +586,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // Wait for the previous tile's PV before publishing this tile's P:
         // o_done then never runs more than one phase ahead of this wait, and
         // the accumulator is stable if rows whose max moved need rescaling.
-        if (!(ok = wait_bar(sh.o_done, (jj - 1) & 1, sh, status))) break;
+        if (!(ok = wait_bar_warp(sh.o_done, (jj - 1) & 1, sh, status))) break;
         tc_fence_after_sync();
         if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
@@ -589,10 +622,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (lane == 0) mbar_arrive(&sh.p_full[jj & 1]);
     }
     if (ok && nt > 0) {
-      ok = wait_bar(sh.o_done, (nt - 1) & 1, sh, status);
+      ok = wait_bar_warp(sh.o_done, (nt - 1) & 1, sh, status);
       tc_fence_after_sync();
     }
-    if (ok && pre_smem) ok = wait_bar(sh.pre_full, 0, sh, status);
+    if (ok && pre_smem) ok = wait_bar_warp(sh.pre_full, 0, sh, status);
     // ---------------------------------------------------------------- epilogue
     const bool row_ok = ok && tok < p.S;
     const bool empty = (nt == 0) || !(l_run > 0.f);
