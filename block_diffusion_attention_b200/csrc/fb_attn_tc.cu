@@ -429,67 +429,61 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (kk < ksteps)
           umma_bf16_ts(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
     };
-    // The loop keeps the work between "P of tile j is ready" and the PV(j)
-    // issue to one barrier test: V(j) is waited for, its tail rows cleared
-    // and tile j + 1 located before QK^T(j + 1) is issued.  (This warp shares
-    // its scheduler with a softmax warp, so every instruction on that path
-    // delays the tensor pipe.)
-    bool ok = wait_bar_warp(sh.q_tmem, 0, sh, status);
-    if (ok && nt > 0) {
-      Tile tc = tile_at(p, u, b, kvh, j0);
-      ok = wait_bar_warp(&sh.full[slot_of(0)], 0, sh, status);
-      if (ok) {
-        tc_fence_after_sync();
-        if (lane == 0) {
+    // One thread (lane 0) runs the issue loop; the other lanes wait at the
+    // warp barrier below.  The loop keeps the work between "P of tile j is
+    // ready" and the PV(j) issue to one barrier test: V(j) is waited for, its
+    // tail rows cleared and tile j + 1 located before QK^T(j + 1) is issued.
+    // (This warp shares its scheduler with a softmax warp, so every
+    // instruction on that path delays the tensor pipe.)
+    if (lane == 0) {
+      bool ok = wait_bar(sh.q_tmem, 0, sh, status);
+      if (ok && nt > 0) {
+        Tile tc = tile_at(p, u, b, kvh, j0);
+        ok = wait_bar(&sh.full[slot_of(0)], 0, sh, status);
+        if (ok) {
+          tc_fence_after_sync();
           issue_qk(0, tc.nvalid);
           tc_commit(&sh.s_full[0]);
           tc_commit(&sh.empty[slot_of(0)]);
         }
-        __syncwarp();
-      }
-      for (int jj = 0; ok && jj < nt; ++jj) {
-        const int iv = 2 * jj + 1;
-        if (!(ok = wait_bar_warp(&sh.full[slot_of(iv)], use_of(iv) & 1, sh, status))) break;
-        if (tc.seg == 0 && (tc.nvalid & 15)) {
-          // Cache rows past the prefix may hold anything (even NaN); P is 0
-          // there but 0 * NaN is not, so clear the V rows up to the next
-          // 16-key step that PV reads.
-          uint8_t* dV = sRing + slot_of(iv) * SLOT_BYTES;
-          const int nrow = ((tc.nvalid + 15) & ~15) - tc.nvalid;
-          for (int i = lane; i < nrow * 16; i += 32) {
-            const int r = tc.nvalid + (i >> 4);
-            const int h = (i >> 3) & 1;
-            const int c = i & 7;
-            *reinterpret_cast<uint4*>(dV + h * HALF_BYTES + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        for (int jj = 0; ok && jj < nt; ++jj) {
+          const int iv = 2 * jj + 1;
+          if (!(ok = wait_bar(&sh.full[slot_of(iv)], use_of(iv) & 1, sh, status))) break;
+          if (tc.seg == 0 && (tc.nvalid & 15)) {
+            // Cache rows past the prefix may hold anything (even NaN); P is 0
+            // there but 0 * NaN is not, so clear the V rows up to the next
+            // 16-key step that PV reads (at most 15 rows, once per unit).
+            uint8_t* dV = sRing + slot_of(iv) * SLOT_BYTES;
+            const int nrow = ((tc.nvalid + 15) & ~15) - tc.nvalid;
+            for (int i = 0; i < nrow * 16; ++i) {
+              const int r = tc.nvalid + (i >> 4);
+              const int h = (i >> 3) & 1;
+              const int c = i & 7;
+              *reinterpret_cast<uint4*>(dV + h * HALF_BYTES + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-        }
-        Tile tn = tc;
-        if (jj + 1 < nt) {
-          tn = tile_at(p, u, b, kvh, j0 + jj + 1);
-          const int ik = 2 * (jj + 1);
-          if (!(ok = wait_bar_warp(&sh.full[slot_of(ik)], use_of(ik) & 1, sh, status))) break;
-          tc_fence_after_sync();
-          if (lane == 0) {
+          Tile tn = tc;
+          if (jj + 1 < nt) {
+            tn = tile_at(p, u, b, kvh, j0 + jj + 1);
+            const int ik = 2 * (jj + 1);
+            if (!(ok = wait_bar(&sh.full[slot_of(ik)], use_of(ik) & 1, sh, status))) break;
+            tc_fence_after_sync();
             issue_qk(jj + 1, tn.nvalid);
             tc_commit(&sh.s_full[(jj + 1) & 1]);
             tc_commit(&sh.empty[slot_of(ik)]);
           }
-        }
-        if (!(ok = wait_bar_warp(&sh.p_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
-        tc_fence_after_sync();
-        if (lane == 0) {
+          if (!(ok = wait_bar(&sh.p_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
+          tc_fence_after_sync();
           issue_pv(jj, tc.nvalid);
           tc_commit(sh.o_done);
           tc_commit(&sh.empty[slot_of(iv)]);
+          tc = tn;
         }
-        tc = tn;
       }
+      // Drain every MMA this thread issued before TMEM can be released.
+      tc_commit(sh.drain);
     }
-    __syncwarp();
-    // Drain every MMA this thread issued before TMEM can be released.
-    if (lane == 0) tc_commit(sh.drain);
     __syncwarp();
     wait_bar(sh.drain, 0, sh, nullptr, false);
   } else {
