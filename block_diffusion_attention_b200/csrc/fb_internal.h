@@ -118,6 +118,13 @@ __device__ __forceinline__ int active_splits(int grid, int n_active, int n_rt) {
   return ns < 1 ? 1 : (ns > TC_MAX_SPLITS ? TC_MAX_SPLITS : ns);
 }
 
+// Block step of a short block on the CUDA cores (one warp per query row):
+// usable when small_step_fits().
+bool small_step_fits(const fb_desc& d, int num_sms);
+cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
+                                    const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
+                                    cudaStream_t stream);
+
 cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
                            const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
                            const CUtensorMap& tmPre, const CUtensorMap& tmO, int grid, cudaStream_t stream);
