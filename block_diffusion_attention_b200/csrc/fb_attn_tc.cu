@@ -15,22 +15,31 @@
 // query heads of the group.
 //
 // Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); online softmax
-//              in fp32 with base-2 exponentials, P written back into tensor
-//              memory as bf16 pairs, lazy rescaling of the accumulator, epilogue;
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); copies its Q
+//              row into tensor memory, then online softmax in fp32 with
+//              base-2 exponentials (a quarter of them on the FMA pipe), P
+//              written back into tensor memory as bf16 pairs, lazy rescaling
+//              of the accumulator, epilogue (output tile staged in shared
+//              memory, written by TMA stores);
 //   warp 4     TMA producer: Q once, then K and V tiles into a ring of six
 //              32 KB shared-memory slots (K and V of a tile take one slot each);
-//   warp 5     TMEM owner and MMA issuer: S = Q K^T (A and B from shared
-//              memory) and O += P V (A = P from tensor memory, B = V from
-//              shared memory) with tcgen05.mma, M = 128, N = 128, K = 16.
+//   warp 5     TMEM owner; its lane 0 issues the tcgen05.mma: S = Q K^T (A = Q
+//              from tensor memory, B = K from shared memory) and O += P V (A =
+//              P from tensor memory, B = V from shared memory), M = 128,
+//              N = 128, K = 16.
 //
 // TMEM (512 columns): S double-buffered at columns [0, 128) and [128, 256) --
-// tile j's P overwrites the first 64 columns of its own S buffer -- and the
-// O accumulator at [256, 384).  QK^T of tile j + 1 therefore overlaps the
-// softmax of tile j, and a K slot is released as soon as its QK^T is done.
+// tile j's P overwrites the first 64 columns of its own S buffer -- the O
+// accumulator at [256, 384) and Q at [384, 448).  QK^T of tile j + 1
+// therefore overlaps the softmax of tile j, and a K slot is released as soon
+// as its QK^T is done.
 // Shared memory (1024-byte aligned, 128-byte swizzle everywhere):
 //   Q     [2 halves of 64 dims][128 rows][128 B]        32 KB
 //   ring  6 x [2 halves][128 keys][128 B]              192 KB
+//
+// A refresh mask can leave units out (their CTAs return after the
+// prologue), or share the grid out among the selected units only (the
+// active-unit split; see AttnParams::dyn).
 //
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // FB_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
