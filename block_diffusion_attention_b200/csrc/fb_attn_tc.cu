@@ -794,6 +794,43 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombinePa
     so = (size_t)TC_BM * c.D;
     sl = TC_BM;
   }
+  if (nsplit <= 32 && c.D == 4 * 32) {
+    // up to 32 splits: every load in flight at once -- lane l reads split l's
+    // LSE and the four output columns 4l..4l+3 of every split
+    const float lse_l = lane < nsplit ? lbase[lane * sl] : -CUDART_INF_F;
+    float4 v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < nsplit) v[i] = __ldg(reinterpret_cast<const float4*>(base + i * so + lane * 4));
+    const float M = warp_max_f(lse_l);
+    const bool empty = (M == -CUDART_INF_F);
+    const float w_l = (empty || lse_l == -CUDART_INF_F) ? 0.f : expf(lse_l - M);
+    const float den = warp_sum_f(w_l);
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float w = __shfl_sync(0xffffffffu, w_l, i);  // split order, as below
+      if (i < nsplit) {
+        acc.x = fmaf(w, v[i].x, acc.x);
+        acc.y = fmaf(w, v[i].y, acc.y);
+        acc.z = fmaf(w, v[i].z, acc.z);
+        acc.w = fmaf(w, v[i].w, acc.w);
+      }
+    }
+    acc = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    const int d0 = lane * 4;
+    if (c.out_o32) {
+      *reinterpret_cast<float4*>(c.out_o32 + row * c.D + d0) = acc;
+    } else if (c.out_bf16) {
+      uint2 u = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(c.out_o) + row * c.D + d0) = u;
+    } else {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(c.out_o) + row * c.D + d0) = acc;
+    }
+    if (lane == 0 && c.out_lse) c.out_lse[lrow] = empty ? -CUDART_INF_F : M + logf(den);
+    return;
+  }
   // lane l holds the LSE (then the weight) of splits l, l + 32, l + 64, l + 96
   constexpr int PER_LANE = TC_MAX_SPLITS / 32;
   float wreg[PER_LANE];
