@@ -163,3 +163,57 @@ def test_merge_partials_matches_oracle():
     # fp32 on the GPU against float64 from the same (fp32-representable) inputs
     gpu_cases.compare("merge O", Oo.cpu().numpy(), ref_o, "fp32")
     gpu_cases.compare("merge LSE", Lo.cpu().numpy(), ref_l.transpose(0, 2, 1), "fp32")
+
+
+def _sparse_layer(prefix_len, chunk_size, topk, batch=2):
+    w = W["lm_gqa"].scaled(batch=batch, prefix_len=prefix_len, blocks=1, steps=1, chunk_size=chunk_size, topk=topk)
+    K, V, lens = synth.prefix_kv(w)
+    Kt, K64 = gpu_cases.tensors(w, K)
+    Vt, V64 = gpu_cases.tensors(w, V)
+    layer = gpu_cases.make_layer(w)
+    layer.load_prefix(Kt, Vt, lens)
+    Q, _, _ = synth.step_inputs(w, 0, 0)
+    Qt, Q64 = gpu_cases.tensors(w, Q)
+    return w, layer, Qt, Q64, K64, V64, lens.astype(np.int64)
+
+
+def test_sparse_chunk_lists_longer_than_a_warp():
+    # 40-entry chunk lists (two 32-entry steps of the list scan), hand-made
+    # with gaps, against the oracle's prefix partial over the same chunks
+    w, layer, Qt, Q64, K64, V64, lens = _sparse_layer(prefix_len=6500, chunk_size=128, topk=40)
+    nch = -(-6500 // 128)
+    rng = np.random.default_rng(11)
+    idx = np.full((w.batch, w.num_kv_heads, w.topk), -1, np.int32)
+    for b in range(w.batch):
+        for kvh in range(w.num_kv_heads):
+            idx[b, kvh] = np.sort(rng.choice(nch, size=w.topk, replace=False))
+    idx[1, 3, 35:] = -1  # a shorter list
+    layer.chunk_idx.copy_(torch.from_numpy(idx))
+    fbl.fb_prefix_partial(layer.desc, Qt, layer.K, layer.V, layer.chunk_idx, layer.O_pre, layer.LSE_pre,
+                          layer.workspace, layer.status)
+    layer.check()
+    ref_o, ref_l = ora.prefix_partial(Q64, K64, V64, lens, w.softmax_scale, idx, w.chunk_size)
+    gpu_cases.compare("O_pre", layer.O_pre.cpu().numpy(), ref_o, w.dtype)
+    gpu_cases.compare("LSE_pre", layer.LSE_pre.cpu().numpy(), ref_l, w.dtype)
+
+
+@pytest.mark.parametrize("bad", ["descending", "past_prefix"])
+def test_sparse_invalid_chunk_list_reported(bad):
+    # a list entry that is not above its predecessor, or lies past the valid
+    # prefix, ends the list and is reported; the entries before it are used
+    w, layer, Qt, Q64, K64, V64, lens = _sparse_layer(prefix_len=3000, chunk_size=256, topk=6, batch=1)
+    idx = np.full((w.batch, w.num_kv_heads, w.topk), -1, np.int32)
+    idx[0, :, :3] = [1, 4, 7]
+    idx[0, 2, 3] = 2 if bad == "descending" else 40
+    idx[0, 2, 4] = 9
+    layer.chunk_idx.copy_(torch.from_numpy(idx))
+    fbl.fb_prefix_partial(layer.desc, Qt, layer.K, layer.V, layer.chunk_idx, layer.O_pre, layer.LSE_pre,
+                          layer.workspace, layer.status)
+    with pytest.raises(fbl.FlashBlockError) as e:
+        layer.check()
+    assert e.value.status == 7
+    used = idx.copy()
+    used[0, 2, 3:] = -1
+    ref_o, ref_l = ora.prefix_partial(Q64, K64, V64, lens, w.softmax_scale, used, w.chunk_size)
+    gpu_cases.compare("O_pre", layer.O_pre.cpu().numpy(), ref_o, w.dtype)
+    gpu_cases.compare("LSE_pre", layer.LSE_pre.cpu().numpy(), ref_l, w.dtype)
