@@ -71,6 +71,18 @@ def test_edge_lengths(L, S, G):
     gpu_cases.run_workload(w)
 
 
+def test_block_step_kernel_choice_both_paths():
+    # short blocks with few query rows run the CUDA-core step kernel (one warp
+    # per row); with many rows the tensor-core kernel's 32- and 48-key
+    # instantiations run instead -- both against the oracle
+    few = W["lm_gqa"].scaled(prefix_len=300, block_len=48, num_q_heads=16, num_kv_heads=2, blocks=1, steps=2)
+    many32 = W["lm_gqa"].scaled(batch=12, prefix_len=300, block_len=32, blocks=1, steps=2)
+    many48 = W["lm_gqa"].scaled(batch=10, prefix_len=300, block_len=48, num_q_heads=16, num_kv_heads=4,
+                                blocks=1, steps=2)
+    for w in (few, many32, many48):
+        gpu_cases.run_workload(w)
+
+
 def test_edge_lengths_fp32_empty_prefix():
     w = W["tiny_fp32"].scaled(prefix_len=0, block_len=5, steps=2, blocks=2)
     gpu_cases.run_workload(w)

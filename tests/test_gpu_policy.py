@@ -49,8 +49,8 @@ def test_threshold_extremes_bf16():
     assert not any(m.any() for m in masks[1:])
 
 
-@pytest.mark.parametrize("num_splits", [0, 5])
-def test_masked_prefix_pass_random_masks(num_splits):
+@pytest.mark.parametrize("num_splits,page_size", [(0, 0), (5, 0), (0, 128), (3, 64)])
+def test_masked_prefix_pass_random_masks(num_splits, page_size):
     """fb_prefix_partial_masked against the oracle's prefix partial: the rows
     of selected units are recomputed, the others are left untouched (also
     when the grid is shared out among the selected units only)."""
@@ -63,7 +63,7 @@ def test_masked_prefix_pass_random_masks(num_splits):
     K, V, lens = synth.prefix_kv(w)
     Kt, K64 = tensors(w, K)
     Vt, V64 = tensors(w, V)
-    layer = make_layer(w, num_splits=num_splits)
+    layer = make_layer(w, page_size=page_size, num_splits=num_splits)
     layer.load_prefix(Kt, Vt, lens)
     Q, _, _ = synth.step_inputs(w, 0, 0)
     Qt, Q64 = tensors(w, Q)
