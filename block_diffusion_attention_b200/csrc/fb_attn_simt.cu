@@ -11,6 +11,7 @@
 #include <math_constants.h>
 
 #include "fb_internal.h"
+#include "fb_ptx.cuh"
 
 namespace fb {
 
@@ -103,6 +104,9 @@ __global__ void __launch_bounds__(WARPS * 32)
     attn_simt_kernel(const AttnParams p, const float* __restrict__ Q, const float* __restrict__ Kp,
                      const float* __restrict__ Vp, const float* __restrict__ Kb,
                      const float* __restrict__ Vb) {
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float sq[WARPS][MAXD];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -201,19 +205,13 @@ __global__ void __launch_bounds__(WARPS * 32)
 cudaError_t launch_attn_simt(const AttnParams& p, const float* Q, const float* Kp, const float* Vp,
                              const float* Kb, const float* Vb, cudaStream_t stream) {
   dim3 grid((p.S + WARPS - 1) / WARPS, p.Hq, p.B);
-  switch (p.epi) {
-    case EPI_PARTIAL:
-      attn_simt_kernel<EPI_PARTIAL><<<grid, WARPS * 32, 0, stream>>>(p, Q, Kp, Vp, Kb, Vb);
-      break;
-    case EPI_MERGE:
-      attn_simt_kernel<EPI_MERGE><<<grid, WARPS * 32, 0, stream>>>(p, Q, Kp, Vp, Kb, Vb);
-      break;
-    default:
-      attn_simt_kernel<EPI_NORM><<<grid, WARPS * 32, 0, stream>>>(p, Q, Kp, Vp, Kb, Vb);
-      break;
-  }
+  void (*kern)(const AttnParams, const float*, const float*, const float*, const float*, const float*) =
+      p.epi == EPI_PARTIAL ? attn_simt_kernel<EPI_PARTIAL>
+      : p.epi == EPI_MERGE ? attn_simt_kernel<EPI_MERGE>
+                           : attn_simt_kernel<EPI_NORM>;
+  cudaError_t e = launch_pdl(kern, grid, dim3(WARPS * 32), 0, stream, p, Q, Kp, Vp, Kb, Vb);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace fb

@@ -15,6 +15,7 @@
 #include <math_constants.h>
 
 #include "fb_internal.h"
+#include "fb_ptx.cuh"
 
 namespace fb {
 
@@ -67,6 +68,9 @@ template <typename T>
 __global__ void chunk_means_kernel(const CacheGeom g, const int32_t* lens, int chunk_size,
                                    int c0, int nch_total, const T* __restrict__ K,
                                    float* __restrict__ Kmean, int32_t* status) {
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
   const int c = c0 + blockIdx.x;
   const int kvh = blockIdx.y;
   const int b = blockIdx.z;
@@ -122,6 +126,9 @@ __global__ void __launch_bounds__(SEL_THREADS)
     select_chunks_kernel(const CacheGeom g, const int32_t* lens, int chunk_size, int nch_total, int S, int Hq,
                          int topk, const T* __restrict__ Q, const float* __restrict__ Kmean,
                          int32_t* __restrict__ idx, int32_t* status) {
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ float sm[];
   const int kvh = blockIdx.x;
   const int b = blockIdx.y;
@@ -218,6 +225,9 @@ template <typename T>
 __global__ void kv_append_kernel(const CacheGeom g, const int32_t* lens, int S,
                                  const T* __restrict__ Kb, const T* __restrict__ Vb,
                                  T* __restrict__ Kc, T* __restrict__ Vc, int32_t* status) {
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int VEC = 16 / sizeof(T);
   const long long nvec_row = g.D / VEC;
   const long long total = (long long)g.B * S * g.Hkv * nvec_row;
@@ -250,6 +260,9 @@ __global__ void kv_append_kernel(const CacheGeom g, const int32_t* lens, int S,
 __global__ void complement_chunks_kernel(const CacheGeom g, const int32_t* lens, int chunk_size,
                                          int nch_total, int topk, const int32_t* __restrict__ idx,
                                          int32_t* __restrict__ comp, int comp_cap, int32_t* status) {
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ int flag[];
   const int kvh = blockIdx.x, b = blockIdx.y;
   int L = lens[b];
@@ -287,6 +300,9 @@ __global__ void complement_chunks_kernel(const CacheGeom g, const int32_t* lens,
 __global__ void merge_partials_kernel(int B, int S, int Hq, int D, const float* __restrict__ Oa,
                                       const float* __restrict__ La, const float* __restrict__ Ob,
                                       const float* __restrict__ Lb, float* Oo, float* Lo) {
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
   const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const long long nrows = (long long)B * S * Hq;
@@ -319,6 +335,9 @@ __global__ void merge_partials_kernel(int B, int S, int Hq, int D, const float* 
 
 // Runs after the copy: advance each length by S when the block fitted.
 __global__ void lens_advance_kernel(int32_t* lens, int B, int S, int cap) {
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) {
     const int L = lens[b];
@@ -334,14 +353,15 @@ cudaError_t launch_chunk_means(const fb_desc& d, const void* K, int c0, int c1, 
   const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
   if (c1 <= c0) return cudaSuccess;
   dim3 grid(c1 - c0, g.Hkv, g.B);
+  cudaError_t e;
   if (d.dtype == FB_BF16)
-    chunk_means_kernel<__nv_bfloat16><<<grid, g.D, 0, stream>>>(
-        g, d.prefix_lens, d.chunk_size, c0, nch_total, static_cast<const __nv_bfloat16*>(K), Kmean, status);
+    e = launch_pdl(chunk_means_kernel<__nv_bfloat16>, grid, dim3(g.D), 0, stream, g, d.prefix_lens, d.chunk_size,
+                   c0, nch_total, static_cast<const __nv_bfloat16*>(K), Kmean, status);
   else
-    chunk_means_kernel<float><<<grid, g.D, 0, stream>>>(g, d.prefix_lens, d.chunk_size, c0, nch_total,
-                                                        static_cast<const float*>(K), Kmean, status);
+    e = launch_pdl(chunk_means_kernel<float>, grid, dim3(g.D), 0, stream, g, d.prefix_lens, d.chunk_size, c0,
+                   nch_total, static_cast<const float*>(K), Kmean, status);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* Kmean, int32_t* idx,
@@ -350,21 +370,20 @@ cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* K
   const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
   const size_t smem = (size_t)(SEL_PART_FLOATS + g.D + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int);
   dim3 grid(g.Hkv, g.B);
+  cudaError_t e;
   if (d.dtype == FB_BF16) {
     auto k = select_chunks_kernel<__nv_bfloat16>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, SEL_THREADS, smem, stream>>>(g, d.prefix_lens, d.chunk_size, nch_total, d.block_len,
-                                           d.num_q_heads, d.topk, static_cast<const __nv_bfloat16*>(Q), Kmean,
-                                           idx, status);
+    e = launch_pdl(k, grid, dim3(SEL_THREADS), smem, stream, g, d.prefix_lens, d.chunk_size, nch_total,
+                   d.block_len, d.num_q_heads, d.topk, static_cast<const __nv_bfloat16*>(Q), Kmean, idx, status);
   } else {
     auto k = select_chunks_kernel<float>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, SEL_THREADS, smem, stream>>>(g, d.prefix_lens, d.chunk_size, nch_total, d.block_len,
-                                           d.num_q_heads, d.topk, static_cast<const float*>(Q), Kmean, idx,
-                                           status);
+    e = launch_pdl(k, grid, dim3(SEL_THREADS), smem, stream, g, d.prefix_lens, d.chunk_size, nch_total,
+                   d.block_len, d.num_q_heads, d.topk, static_cast<const float*>(Q), Kmean, idx, status);
   }
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_complement_chunks(const fb_desc& d, const int32_t* idx, int32_t* comp, int comp_cap,
@@ -375,20 +394,20 @@ cudaError_t launch_complement_chunks(const fb_desc& d, const int32_t* idx, int32
   const size_t smem = (size_t)nch_total * sizeof(int);
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(complement_chunks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  complement_chunks_kernel<<<grid, 32, smem, stream>>>(
-      g, d.prefix_lens, d.chunk_size, nch_total, d.topk, idx, comp, comp_cap, status);
+  cudaError_t e = launch_pdl(complement_chunks_kernel, grid, dim3(32), smem, stream, g, d.prefix_lens,
+                             d.chunk_size, nch_total, d.topk, idx, comp, comp_cap, status);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_merge_partials(const fb_desc& d, const float* Oa, const float* La, const float* Ob,
                                   const float* Lb, float* Oo, float* Lo, cudaStream_t stream) {
   const long long rows = (long long)d.batch * d.block_len * d.num_q_heads;
   const int warps = 8;
-  merge_partials_kernel<<<(unsigned)((rows + warps - 1) / warps), warps * 32, 0, stream>>>(
-      d.batch, d.block_len, d.num_q_heads, d.head_dim, Oa, La, Ob, Lb, Oo, Lo);
+  cudaError_t e = launch_pdl(merge_partials_kernel, dim3((unsigned)((rows + warps - 1) / warps)), dim3(warps * 32),
+                             0, stream, d.batch, d.block_len, d.num_q_heads, d.head_dim, Oa, La, Ob, Lb, Oo, Lo);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_kv_append(const fb_desc& d, const void* Kb, const void* Vb, void* Kc, void* Vc,
@@ -400,20 +419,23 @@ cudaError_t launch_kv_append(const fb_desc& d, const void* Kb, const void* Vb, v
   const int threads = 256;
   const long long want = (total + threads - 1) / threads;
   const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
+  cudaError_t e;
   if (d.dtype == FB_BF16)
-    kv_append_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(
-        g, lens, d.block_len, static_cast<const __nv_bfloat16*>(Kb), static_cast<const __nv_bfloat16*>(Vb),
-        static_cast<__nv_bfloat16*>(Kc), static_cast<__nv_bfloat16*>(Vc), status);
+    e = launch_pdl(kv_append_kernel<__nv_bfloat16>, dim3(grid), dim3(threads), 0, stream, g, lens, d.block_len,
+                   static_cast<const __nv_bfloat16*>(Kb), static_cast<const __nv_bfloat16*>(Vb),
+                   static_cast<__nv_bfloat16*>(Kc), static_cast<__nv_bfloat16*>(Vc), status);
   else
-    kv_append_kernel<float><<<grid, threads, 0, stream>>>(
-        g, lens, d.block_len, static_cast<const float*>(Kb), static_cast<const float*>(Vb),
-        static_cast<float*>(Kc), static_cast<float*>(Vc), status);
+    e = launch_pdl(kv_append_kernel<float>, dim3(grid), dim3(threads), 0, stream, g, lens, d.block_len,
+                   static_cast<const float*>(Kb), static_cast<const float*>(Vb), static_cast<float*>(Kc),
+                   static_cast<float*>(Vc), status);
   note_launch();
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || !lens_inout) return e;
-  lens_advance_kernel<<<(g.B + 127) / 128, 128, 0, stream>>>(lens_inout, g.B, d.block_len, g.cap);
+  // (waits for the append above to complete before it moves the lengths)
+  e = launch_pdl(lens_advance_kernel, dim3((g.B + 127) / 128), dim3(128), 0, stream, lens_inout, g.B, d.block_len,
+                 g.cap);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace fb

@@ -79,6 +79,25 @@ constexpr int TC_SLOTS = 6;     // K/V ring: 32 KB slots (K and V of a tile take
 constexpr int TC_THREADS = 192; // 4 softmax warps + TMA warp + MMA warp
 constexpr int TC_MAX_SPLITS = 128;  // key-range splits per work unit
 size_t tc_smem_bytes();
+// Launch with programmatic stream serialization: the kernel may start while
+// its predecessor in the stream finishes; it must call griddepcontrol.wait
+// (pdl_wait) before reading anything that predecessor writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // ---- active-unit split plan (shared by the attention kernel and the combine)
 // Every lane of the calling warp must take part (warp ballots over the mask).
 __device__ __forceinline__ int active_count(const int32_t* mask, int nu) {

@@ -28,6 +28,7 @@
 #include <math_constants.h>
 
 #include "fb_internal.h"
+#include "fb_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -64,6 +65,9 @@ template <bool BF16>
 __global__ void __cluster_dims__(HW_CLUSTER, 1, 1) __launch_bounds__(HW_THREADS)
     headwise_mask_kernel(const uint4* __restrict__ Qnow, uint4* __restrict__ Qref, int S, int Hq, int Hkv,
                          int D, float gamma, int32_t* __restrict__ mask, float* __restrict__ sim_out) {
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float red[HW_THREADS / 32][3];
   __shared__ float part[3];
   cg::cluster_group cluster = cg::this_cluster();
@@ -150,6 +154,9 @@ __global__ void __launch_bounds__(TH_TOKENS * 32)
     threshold_flag_kernel(uint4* __restrict__ Kprev, uint4* __restrict__ Vprev, const uint4* __restrict__ Know,
                           const uint4* __restrict__ Vnow, int S, int vpt, float eps, int nslice,
                           int32_t* __restrict__ counts) {
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ int flags[TH_TOKENS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slice = blockIdx.x, b = blockIdx.y;
@@ -187,6 +194,9 @@ __global__ void __launch_bounds__(TH_TOKENS * 32)
 
 __global__ void threshold_decide_kernel(const int32_t* __restrict__ counts, int nslice, int Hkv, int32_t tau,
                                         int32_t* __restrict__ mask, int32_t* __restrict__ count_out) {
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
   const int b = blockIdx.x;
   int c = 0;
   for (int i = threadIdx.x; i < nslice; i += 32) c += counts[(size_t)b * nslice + i];
@@ -206,16 +216,11 @@ size_t threshold_ws_bytes(const fb_desc& d) {
 cudaError_t launch_headwise_mask(const fb_desc& d, const void* Qnow, void* Qref, float gamma, int32_t* mask,
                                  float* sim, cudaStream_t stream) {
   const dim3 grid((unsigned)(d.batch * d.num_kv_heads * HW_CLUSTER));
-  if (d.dtype == FB_BF16)
-    headwise_mask_kernel<true><<<grid, HW_THREADS, 0, stream>>>(
-        static_cast<const uint4*>(Qnow), static_cast<uint4*>(Qref), d.block_len, d.num_q_heads, d.num_kv_heads,
-        d.head_dim, gamma, mask, sim);
-  else
-    headwise_mask_kernel<false><<<grid, HW_THREADS, 0, stream>>>(
-        static_cast<const uint4*>(Qnow), static_cast<uint4*>(Qref), d.block_len, d.num_q_heads, d.num_kv_heads,
-        d.head_dim, gamma, mask, sim);
+  cudaError_t e = launch_pdl(d.dtype == FB_BF16 ? headwise_mask_kernel<true> : headwise_mask_kernel<false>, grid,
+                             dim3(HW_THREADS), 0, stream, static_cast<const uint4*>(Qnow), static_cast<uint4*>(Qref),
+                             d.block_len, d.num_q_heads, d.num_kv_heads, d.head_dim, gamma, mask, sim);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_threshold_mask(const fb_desc& d, void* Kprev, void* Vprev, const void* Know, const void* Vnow,
@@ -225,20 +230,17 @@ cudaError_t launch_threshold_mask(const fb_desc& d, void* Kprev, void* Vprev, co
   const int epv = d.dtype == FB_BF16 ? 8 : 4;
   const int vpt = d.num_kv_heads * d.head_dim / epv;
   const dim3 grid((unsigned)nslice, (unsigned)d.batch);
-  if (d.dtype == FB_BF16)
-    threshold_flag_kernel<true><<<grid, TH_TOKENS * 32, 0, stream>>>(
-        static_cast<uint4*>(Kprev), static_cast<uint4*>(Vprev), static_cast<const uint4*>(Know),
-        static_cast<const uint4*>(Vnow), d.block_len, vpt, eps, nslice, ws);
-  else
-    threshold_flag_kernel<false><<<grid, TH_TOKENS * 32, 0, stream>>>(
-        static_cast<uint4*>(Kprev), static_cast<uint4*>(Vprev), static_cast<const uint4*>(Know),
-        static_cast<const uint4*>(Vnow), d.block_len, vpt, eps, nslice, ws);
+  cudaError_t e =
+      launch_pdl(d.dtype == FB_BF16 ? threshold_flag_kernel<true> : threshold_flag_kernel<false>, grid,
+                 dim3(TH_TOKENS * 32), 0, stream, static_cast<uint4*>(Kprev), static_cast<uint4*>(Vprev),
+                 static_cast<const uint4*>(Know), static_cast<const uint4*>(Vnow), d.block_len, vpt, eps, nslice, ws);
   note_launch();
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  threshold_decide_kernel<<<d.batch, 32, 0, stream>>>(ws, nslice, d.num_kv_heads, tau, mask, count);
+  e = launch_pdl(threshold_decide_kernel, dim3(d.batch), dim3(32), 0, stream, (const int32_t*)ws, nslice,
+                 d.num_kv_heads, tau, mask, count);
   note_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace fb
