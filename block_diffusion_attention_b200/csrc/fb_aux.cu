@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(SEL_THREADS)
       float acc[VEC];
 #pragma unroll
       for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
-#pragma unroll 4
+#pragma unroll 16
       for (int rr = r0; rr < rows; rr += rpi) {
         const int t = rr / G, gg = rr - t * G;
         const uint4 v =
@@ -178,22 +178,30 @@ __global__ void __launch_bounds__(SEL_THREADS)
   // score of chunk c: four lanes per chunk, each over a quarter of D with
   // 16-byte loads (all independent), then two shuffles
   const float* km = Kmean + ((size_t)b * g.Hkv + kvh) * nch_total * g.D;
+  // two chunks per lane group per pass, so a 128-chunk prefix needs one pass
+  // with all of its loads in flight
   const int q4 = threadIdx.x & 3, dq = g.D / 4;
-  for (int base = 0; base < nch; base += SEL_THREADS / 4) {
-    const int c = base + (threadIdx.x >> 2);
-    float acc = 0.f;
-    if (c < nch) {
-      const float4* kr = reinterpret_cast<const float4*>(km + (size_t)c * g.D + q4 * dq);
-      const float4* qr = reinterpret_cast<const float4*>(qbar + q4 * dq);
+  constexpr int CPP = SEL_THREADS / 4;  // chunks per half-pass
+  for (int base = 0; base < nch; base += 2 * CPP) {
+    const int c0 = base + (threadIdx.x >> 2), c1 = c0 + CPP;
+    float acc0 = 0.f, acc1 = 0.f;
+    const float4* qr = reinterpret_cast<const float4*>(qbar + q4 * dq);
+    const float4* kr0 = reinterpret_cast<const float4*>(km + (size_t)c0 * g.D + q4 * dq);
+    const float4* kr1 = reinterpret_cast<const float4*>(km + (size_t)c1 * g.D + q4 * dq);
 #pragma unroll 8
-      for (int i = 0; i < dq / 4; ++i) {
-        const float4 k = kr[i], q = qr[i];
-        acc = fmaf(q.x, k.x, fmaf(q.y, k.y, fmaf(q.z, k.z, fmaf(q.w, k.w, acc))));
-      }
+    for (int i = 0; i < dq / 4; ++i) {
+      const float4 q = qr[i];
+      const float4 k0 = c0 < nch ? kr0[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 k1 = c1 < nch ? kr1[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      acc0 = fmaf(q.x, k0.x, fmaf(q.y, k0.y, fmaf(q.z, k0.z, fmaf(q.w, k0.w, acc0))));
+      acc1 = fmaf(q.x, k1.x, fmaf(q.y, k1.y, fmaf(q.z, k1.z, fmaf(q.w, k1.w, acc1))));
     }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (q4 == 0 && c < nch) score[c] = acc;
+    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
+    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
+    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
+    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
+    if (q4 == 0 && c0 < nch) score[c0] = acc0;
+    if (q4 == 0 && c1 < nch) score[c1] = acc1;
   }
   __syncthreads();
   // rank = chunks that beat c (higher score, or equal score and lower index)
