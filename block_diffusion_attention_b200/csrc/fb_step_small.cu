@@ -61,6 +61,15 @@ __device__ __forceinline__ void dot8x4(const uint4& a, const uint4& b, float* ac
   }
 }
 
+__device__ __forceinline__ void pv_fma(float w, const uint2& v, float4& acc) {
+  const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+  const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+  acc.x = fmaf(w, v01.x, acc.x);
+  acc.y = fmaf(w, v01.y, acc.y);
+  acc.z = fmaf(w, v23.x, acc.z);
+  acc.w = fmaf(w, v23.y, acc.w);
+}
+
 __device__ __forceinline__ void pv_step(float w, const uint8_t* vrow, float4& acc) {
   const uint2 v = *reinterpret_cast<const uint2*>(vrow);
   const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
@@ -107,21 +116,26 @@ __global__ void __launch_bounds__(SS_WARPS * 32) block_step_small_kernel(const S
   __syncthreads();
   if (!has_row) return;
 
-  // scores of keys lane and lane + 32, in base 2 (four partial chains each)
+  // scores of keys lane and lane + 32, in base 2 (four partial chains each);
+  // the query row and the key row are read into registers first, so the 16
+  // shared-memory loads of each are in flight together
   float s0 = -CUDART_INF_F, s1 = -CUDART_INF_F;
   {
-    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint8_t* k0 = sK + lane * SS_ROW_BYTES;
-    const uint8_t* k1 = sK + (lane + 32) * SS_ROW_BYTES;
-    const bool has0 = lane < p.S, has1 = lane + 32 < p.S;
+    uint4 qv[SS_D / 8];
 #pragma unroll
-    for (int c = 0; c < SS_D / 8; ++c) {
-      const uint4 q = sQ[warp][c];
-      if (has0) dot8x4(q, *reinterpret_cast<const uint4*>(k0 + c * 16), a0);
-      if (has1) dot8x4(q, *reinterpret_cast<const uint4*>(k1 + c * 16), a1);
-    }
-    if (has0) s0 = ((a0[0] + a0[1]) + (a0[2] + a0[3])) * p.scale_log2;
-    if (has1) s1 = ((a1[0] + a1[1]) + (a1[2] + a1[3])) * p.scale_log2;
+    for (int c = 0; c < SS_D / 8; ++c) qv[c] = sQ[warp][c];
+    auto score = [&](int key) {
+      uint4 kv[SS_D / 8];
+      const uint8_t* kr = sK + key * SS_ROW_BYTES;
+#pragma unroll
+      for (int c = 0; c < SS_D / 8; ++c) kv[c] = *reinterpret_cast<const uint4*>(kr + c * 16);
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < SS_D / 8; ++c) dot8x4(qv[c], kv[c], a);
+      return ((a[0] + a[1]) + (a[2] + a[3])) * p.scale_log2;
+    };
+    if (lane < p.S) s0 = score(lane);
+    if (lane + 32 < p.S) s1 = score(lane + 32);
   }
   float m = fmaxf(s0, s1);
 #pragma unroll
@@ -134,10 +148,18 @@ __global__ void __launch_bounds__(SS_WARPS * 32) block_step_small_kernel(const S
   float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
   const uint8_t* vcol = sV + lane * 8;
   if (p.S == 32) {
+    // the 32 V values of this lane's dims and the 32 weights first, then the FMAs
+    uint2 vv[32];
+    float ww[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      vv[k] = *reinterpret_cast<const uint2*>(vcol + k * SS_ROW_BYTES);
+      ww[k] = __shfl_sync(0xffffffffu, p0, k);
+    }
 #pragma unroll
     for (int k = 0; k < 32; k += 2) {
-      pv_step(__shfl_sync(0xffffffffu, p0, k), vcol + k * SS_ROW_BYTES, acc0);
-      pv_step(__shfl_sync(0xffffffffu, p0, k + 1), vcol + (k + 1) * SS_ROW_BYTES, acc1);
+      pv_fma(ww[k], vv[k], acc0);
+      pv_fma(ww[k + 1], vv[k + 1], acc1);
     }
   } else {
     const int nk0 = min(p.S, 32);
