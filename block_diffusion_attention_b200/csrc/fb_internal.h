@@ -137,8 +137,8 @@ __device__ __forceinline__ int active_splits(int grid, int n_active, int n_rt) {
   return ns < 1 ? 1 : (ns > TC_MAX_SPLITS ? TC_MAX_SPLITS : ns);
 }
 
-// Block step of a short block on the CUDA cores (one warp per query row):
-// usable when small_step_fits().
+// Block step of a short block on warp-level MMA (16 query rows per CTA, the
+// tile in registers): usable when small_step_fits().
 bool small_step_fits(const fb_desc& d, int num_sms);
 cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
                                     const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,

@@ -1,4 +1,4 @@
-// fb_step_small.cu -- the block step for short blocks on the CUDA cores.
+// fb_step_small.cu -- the block step for short blocks on warp-level MMA.
 //
 // The in-block partial and the merge of the Core Mechanism ("FlashBlock:
 // Attention Caching for Efficient Long-Context Block Diffusion", Technical
@@ -8,18 +8,20 @@
 //     m = max(L_pre, L_in),  O = (e^{L_pre-m} O_pre + e^{L_in-m} O_in) / (e^{L_pre-m} + e^{L_in-m}).
 //
 // With a short block (S <= 64) and few query rows the step is pure latency:
-// the tensor-core kernel runs one CTA per 128-row tile, i.e. a handful of SMs.
-// Here one warp takes one query row and a CTA takes eight rows of one
-// (b, kv head), so the rows spread over ~all SMs:
-//  * the unit's K and V block rows go to shared memory once per CTA (rows
-//    padded to 272 bytes, so a warp reading 32 different key rows at the same
-//    column hits distinct banks);
-//  * scores: lane k owns key k (and k + 32), a 128-term dot product against
-//    the query row broadcast from shared memory;
-//  * softmax over the lanes with warp shuffles, P kept in fp32;
-//  * PV: lane l owns output dims 4l .. 4l+3, the S weights broadcast by
-//    shuffle;
-//  * merge and the bf16 store of the row (256 contiguous bytes per warp).
+// a 16-row x S-key x 128-dim tile is far too small to pay for tensor-memory
+// allocation and mbarrier round trips of tcgen05, so each CTA keeps its whole
+// tile in registers and runs it on warp-level mma.sync (m16n8k16, bf16
+// operands, f32 accumulators):
+//  * a CTA takes 16 packed query rows (token, group head) of one (b, kv head)
+//    and the unit's K and V block rows; every global load of the CTA is in
+//    flight at once right after the grid-dependency wait (K, V and Q into
+//    shared memory rows padded to 272 bytes, so ldmatrix hits distinct banks;
+//    the cached O_pre and LSE_pre entries straight into registers);
+//  * each of the four warps computes S = Q K^T for all 16 rows and S_pad
+//    keys (the whole tile: 16 S_pad 128-term dot products), the softmax of
+//    its rows in base 2 with quad shuffles, and then its quarter (32 dims)
+//    of O = P V with P taken from the score registers as bf16 A fragments;
+//  * the merge in base 2 and bf16 stores of the warp's 32 dims of each row.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -30,12 +32,15 @@ namespace fb {
 
 namespace {
 
-constexpr int SS_WARPS = 8;
-constexpr int SS_ROWS_PER_CTA = SS_WARPS;  // query rows of one unit per CTA, one per warp
+constexpr int SS_WARPS = 4;
+constexpr int SS_THREADS = SS_WARPS * 32;
+constexpr int SS_ROWS = 16;                  // packed query rows per CTA: one m16 tile
 constexpr int SS_D = 128;
 constexpr int SS_MAX_S = 64;
-constexpr int SS_ROW_BYTES = SS_D * 2 + 16;  // padded K/V row in shared memory
+constexpr int SS_ROW_BYTES = SS_D * 2 + 16;  // padded K/V/Q row in shared memory
 constexpr float SS_LN2 = 0.6931471805599453f;
+constexpr float SS_LOG2E = 1.4426950408889634f;
+static_assert(SS_D == 32 * SS_WARPS, "one 32-dim quarter of the output per warp");
 
 struct SmallStepParams {
   int B, Hq, Hkv, G, S;
@@ -49,151 +54,200 @@ struct SmallStepParams {
   float* out_lse;           // [B, Hq, S] or null
 };
 
-// acc[0..3] += the four bf16 pairs of a . b (one chain per pair)
-__device__ __forceinline__ void dot8x4(const uint4& a, const uint4& b, float* acc) {
-  const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
-  const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 u = __bfloat1622float2(x[i]);
-    const float2 v = __bfloat1622float2(y[i]);
-    acc[i] = fmaf(u.x, v.x, fmaf(u.y, v.y, acc[i]));
-  }
-}
-
-__device__ __forceinline__ void pv_fma(float w, const uint2& v, float4& acc) {
-  const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
-  const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
-  acc.x = fmaf(w, v01.x, acc.x);
-  acc.y = fmaf(w, v01.y, acc.y);
-  acc.z = fmaf(w, v23.x, acc.z);
-  acc.w = fmaf(w, v23.y, acc.w);
-}
-
-__device__ __forceinline__ void pv_step(float w, const uint8_t* vrow, float4& acc) {
-  const uint2 v = *reinterpret_cast<const uint2*>(vrow);
-  const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
-  const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
-  acc.x = fmaf(w, v01.x, acc.x);
-  acc.y = fmaf(w, v01.y, acc.y);
-  acc.z = fmaf(w, v23.x, acc.z);
-  acc.w = fmaf(w, v23.y, acc.w);
-}
-
-__global__ void __launch_bounds__(SS_WARPS * 32) block_step_small_kernel(const SmallStepParams p) {
-  __shared__ __align__(16) uint8_t sK[SS_MAX_S * SS_ROW_BYTES];
-  __shared__ __align__(16) uint8_t sV[SS_MAX_S * SS_ROW_BYTES];
-  __shared__ __align__(16) uint4 sQ[SS_WARPS][SS_D / 8];
+// SP: keys padded to a multiple of 16 (16, 32 or 64); keys S .. SP - 1 are
+// zero rows in shared memory and masked out of the softmax.
+template <int SP>
+__global__ void __launch_bounds__(SS_THREADS) block_step_small_kernel(const SmallStepParams p) {
+  static_assert(SP % 16 == 0 && SP <= SS_MAX_S, "padded key count");
+  __shared__ __align__(16) uint8_t sQ[SS_ROWS * SS_ROW_BYTES];
+  __shared__ __align__(16) uint8_t sK[SP * SS_ROW_BYTES];
+  __shared__ __align__(16) uint8_t sV[SP * SS_ROW_BYTES];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows_unit = p.S * p.G;
-  const int cpu = (rows_unit + SS_ROWS_PER_CTA - 1) / SS_ROWS_PER_CTA;  // CTAs per unit
+  const int cpu = (rows_unit + SS_ROWS - 1) / SS_ROWS;  // CTAs per unit
   const int unit = blockIdx.x / cpu;
   const int b = unit / p.Hkv, kvh = unit % p.Hkv;
-  const int pr = (blockIdx.x % cpu) * SS_ROWS_PER_CTA + warp;  // this warp's packed row
-  const bool has_row = pr < rows_unit;
-  const int t = has_row ? pr / p.G : 0, h = kvh * p.G + (has_row ? pr % p.G : 0);
-  const size_t qrow = ((size_t)b * p.S + t) * p.Hq + h;
+  const int pr0 = (blockIdx.x % cpu) * SS_ROWS;
+  // the two tile rows of this lane's accumulator entries: lane / 4 and + 8
+  bool row_ok[2];
+  int row_t[2], row_h[2];
+  size_t row_q[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int pr = pr0 + (lane >> 2) + 8 * i;
+    row_ok[i] = pr < rows_unit;
+    row_t[i] = row_ok[i] ? pr / p.G : 0;
+    row_h[i] = kvh * p.G + (row_ok[i] ? pr % p.G : 0);
+    row_q[i] = ((size_t)b * p.S + row_t[i]) * p.Hq + row_h[i];
+  }
 
   pdl_wait();
   pdl_launch_dependents();
 
-  // every global load of the CTA in flight at once: the unit's K and V block
-  // rows (S x 16 chunks of 16 bytes), this warp's query row, its cached
-  // output dims and LSE
-  for (int i = threadIdx.x; i < p.S * (SS_D / 8); i += SS_WARPS * 32) {
+  // ---- every global load of the CTA in flight at once
+  constexpr int KCH = SP * 16 / SS_THREADS;       // 16-byte chunks of K (and of V) per thread
+  constexpr int QCH = SS_ROWS * 16 / SS_THREADS;  // of Q
+  uint4 kr[KCH], vr[KCH], qr[QCH];
+#pragma unroll
+  for (int j = 0; j < KCH; ++j) {
+    const int i = threadIdx.x + j * SS_THREADS;
     const int k = i >> 4, c = i & 15;
-    const size_t src = (((size_t)b * p.S + k) * p.Hkv + kvh) * SS_D + c * 8;
-    *reinterpret_cast<uint4*>(sK + k * SS_ROW_BYTES + c * 16) = *reinterpret_cast<const uint4*>(p.Kb + src);
-    *reinterpret_cast<uint4*>(sV + k * SS_ROW_BYTES + c * 16) = *reinterpret_cast<const uint4*>(p.Vb + src);
+    kr[j] = vr[j] = make_uint4(0u, 0u, 0u, 0u);  // padding keys: zero rows (never NaN)
+    if (k < p.S) {
+      const size_t src = (((size_t)b * p.S + k) * p.Hkv + kvh) * SS_D + c * 8;
+      kr[j] = __ldg(reinterpret_cast<const uint4*>(p.Kb + src));
+      vr[j] = __ldg(reinterpret_cast<const uint4*>(p.Vb + src));
+    }
   }
-  float4 op = make_float4(0.f, 0.f, 0.f, 0.f);
-  float lp = -CUDART_INF_F;
-  if (has_row) {
-    if (lane < 16) sQ[warp][lane] = *reinterpret_cast<const uint4*>(p.Q + qrow * SS_D + lane * 8);
-    op = *reinterpret_cast<const float4*>(p.pre_o + qrow * SS_D + lane * 4);
-    lp = p.pre_lse[((size_t)b * p.Hq + h) * p.S + t];
+#pragma unroll
+  for (int j = 0; j < QCH; ++j) {
+    const int i = threadIdx.x + j * SS_THREADS;
+    const int row = i >> 4, c = i & 15;
+    const int pr = pr0 + row;
+    qr[j] = make_uint4(0u, 0u, 0u, 0u);  // rows past the unit: zero queries, not stored
+    if (pr < rows_unit) {
+      const size_t q = ((size_t)b * p.S + pr / p.G) * p.Hq + kvh * p.G + pr % p.G;
+      qr[j] = __ldg(reinterpret_cast<const uint4*>(p.Q + q * SS_D + c * 8));
+    }
+  }
+  // cached pair of this lane's entries: dims 32 warp + 8 j + 2 (lane % 4) + {0, 1}
+  float2 op[2][4];
+  float lp[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    lp[i] = -CUDART_INF_F;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) op[i][j] = make_float2(0.f, 0.f);
+    if (row_ok[i]) {
+      const float* src = p.pre_o + row_q[i] * SS_D + 32 * warp + 2 * (lane & 3);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) op[i][j] = __ldg(reinterpret_cast<const float2*>(src + 8 * j));
+      lp[i] = __ldg(p.pre_lse + ((size_t)b * p.Hq + row_h[i]) * p.S + row_t[i]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < KCH; ++j) {
+    const int i = threadIdx.x + j * SS_THREADS;
+    const int k = i >> 4, c = i & 15;
+    *reinterpret_cast<uint4*>(sK + k * SS_ROW_BYTES + c * 16) = kr[j];
+    *reinterpret_cast<uint4*>(sV + k * SS_ROW_BYTES + c * 16) = vr[j];
+  }
+#pragma unroll
+  for (int j = 0; j < QCH; ++j) {
+    const int i = threadIdx.x + j * SS_THREADS;
+    *reinterpret_cast<uint4*>(sQ + (i >> 4) * SS_ROW_BYTES + (i & 15) * 16) = qr[j];
   }
   __syncthreads();
-  if (!has_row) return;
 
-  // scores of keys lane and lane + 32, in base 2 (four partial chains each);
-  // the query row and the key row are read into registers first, so the 16
-  // shared-memory loads of each are in flight together
-  float s0 = -CUDART_INF_F, s1 = -CUDART_INF_F;
-  {
-    uint4 qv[SS_D / 8];
+  // ---- S = Q K^T over the whole tile (16 rows x SP keys, 8 steps of 16 dims)
+  const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+  // A fragments: lanes 0-15 address rows 0-15 at the step's first 8 dims,
+  // lanes 16-31 the same rows at its last 8
+  uint32_t qa[SS_D / 16][4];
 #pragma unroll
-    for (int c = 0; c < SS_D / 8; ++c) qv[c] = sQ[warp][c];
-    auto score = [&](int key) {
-      uint4 kv[SS_D / 8];
-      const uint8_t* kr = sK + key * SS_ROW_BYTES;
+  for (int kk = 0; kk < SS_D / 16; ++kk)
+    ldmatrix_x4(qa[kk], q_base + ((lane & 7) + 8 * ((lane >> 3) & 1)) * SS_ROW_BYTES + (16 * kk + 8 * (lane >> 4)) * 2);
+  float sacc[SP / 8][4];
 #pragma unroll
-      for (int c = 0; c < SS_D / 8; ++c) kv[c] = *reinterpret_cast<const uint4*>(kr + c * 16);
-      float a[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int nt = 0; nt < SP / 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
 #pragma unroll
-      for (int c = 0; c < SS_D / 8; ++c) dot8x4(qv[c], kv[c], a);
-      return ((a[0] + a[1]) + (a[2] + a[3])) * p.scale_log2;
-    };
-    if (lane < p.S) s0 = score(lane);
-    if (lane + 32 < p.S) s1 = score(lane + 32);
+  for (int np = 0; np < SP / 16; ++np) {
+#pragma unroll
+    for (int kk = 0; kk < SS_D / 16; ++kk) {
+      // B fragments of key tiles 2 np and 2 np + 1: K rows are the n index,
+      // their dims the k index (no transpose)
+      uint32_t bf[4];
+      ldmatrix_x4(bf, k_base + (16 * np + 8 * (lane >> 4) + (lane & 7)) * SS_ROW_BYTES +
+                          (16 * kk + 8 * ((lane >> 3) & 1)) * 2);
+      mma_bf16_16816(sacc[2 * np], qa[kk], bf[0], bf[1]);
+      mma_bf16_16816(sacc[2 * np + 1], qa[kk], bf[2], bf[3]);
+    }
   }
-  float m = fmaxf(s0, s1);
+
+  // ---- softmax of rows lane / 4 (entries 0, 1) and lane / 4 + 8 (entries 2, 3)
+  float m[2] = {-CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  const float p0 = exp2f(s0 - m), p1 = exp2f(s1 - m);  // 0 for missing keys (-inf)
-  float l = p0 + p1;
+  for (int nt = 0; nt < SP / 8; ++nt)
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-  // O_in (unnormalised): dims 4 lane .. 4 lane + 3, two accumulators
-  float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-  const uint8_t* vcol = sV + lane * 8;
-  if (p.S == 32) {
-    // the 32 V values of this lane's dims and the 32 weights first, then the FMAs
-    uint2 vv[32];
-    float ww[32];
+    for (int e = 0; e < 4; ++e) {
+      const int key = 8 * nt + 2 * (lane & 3) + (e & 1);
+      sacc[nt][e] = key < p.S ? sacc[nt][e] * p.scale_log2 : -CUDART_INF_F;
+      m[e >> 1] = fmaxf(m[e >> 1], sacc[nt][e]);
+    }
+  float l[2] = {0.f, 0.f};
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      vv[k] = *reinterpret_cast<const uint2*>(vcol + k * SS_ROW_BYTES);
-      ww[k] = __shfl_sync(0xffffffffu, p0, k);
+  for (int i = 0; i < 2; ++i) {
+    // the four lanes of a quad hold one row
+    m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], 1));
+    m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], 2));
+  }
+#pragma unroll
+  for (int nt = 0; nt < SP / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      sacc[nt][e] = exp2f(sacc[nt][e] - m[e >> 1]);  // 0 for the masked keys
+      l[e >> 1] += sacc[nt][e];
     }
 #pragma unroll
-    for (int k = 0; k < 32; k += 2) {
-      pv_fma(ww[k], vv[k], acc0);
-      pv_fma(ww[k + 1], vv[k + 1], acc1);
-    }
-  } else {
-    const int nk0 = min(p.S, 32);
-#pragma unroll 8
-    for (int k = 0; k < nk0; ++k) pv_step(__shfl_sync(0xffffffffu, p0, k), vcol + k * SS_ROW_BYTES, acc0);
-#pragma unroll 8
-    for (int k = 32; k < p.S; ++k) pv_step(__shfl_sync(0xffffffffu, p1, k - 32), vcol + k * SS_ROW_BYTES, acc1);
+  for (int i = 0; i < 2; ++i) {
+    l[i] += __shfl_xor_sync(0xffffffffu, l[i], 1);
+    l[i] += __shfl_xor_sync(0xffffffffu, l[i], 2);
   }
-  const float4 acc = make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
-  // merge equation in base 2 (the block always has keys, so l > 0)
-  const float lin2 = m + log2f(l);
-  const float lp2 = lp * 1.4426950408889634f;
-  const float M = fmaxf(lp2, lin2);
-  const float wp = exp2f(lp2 - M);  // 0 when the prefix is empty (lp = -inf)
-  const float wi = exp2f(lin2 - M);
-  const float inv_den = 1.f / (wp + wi);
-  const float ao = exp2f(m - M) * inv_den;  // = wi / l / den
-  const float ap = wp * inv_den;
-  const float4 o = make_float4(fmaf(ap, op.x, ao * acc.x), fmaf(ap, op.y, ao * acc.y), fmaf(ap, op.z, ao * acc.z),
-                               fmaf(ap, op.w, ao * acc.w));
-  *reinterpret_cast<uint2*>(p.out_o + qrow * SS_D + lane * 4) =
-      make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
-  if (lane == 0 && p.out_lse) p.out_lse[((size_t)b * p.Hq + h) * p.S + t] = (M + log2f(wp + wi)) * SS_LN2;
+
+  // ---- O_in = P V for this warp's 32 dims (unnormalised)
+  float oacc[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < SP / 16; ++kk) {
+    // the score accumulators of key tiles 2 kk and 2 kk + 1 are the A
+    // fragment of this 16-key step
+    const uint32_t pa[4] = {pack_bf16x2(sacc[2 * kk][0], sacc[2 * kk][1]),
+                            pack_bf16x2(sacc[2 * kk][2], sacc[2 * kk][3]),
+                            pack_bf16x2(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]),
+                            pack_bf16x2(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3])};
+#pragma unroll
+    for (int jp = 0; jp < 2; ++jp) {
+      // B fragments of dim tiles 2 jp and 2 jp + 1: V rows are the k index,
+      // so the 8 x 8 blocks are transposed on load
+      uint32_t bf[4];
+      ldmatrix_x4_trans(bf, v_base + (16 * kk + 8 * ((lane >> 3) & 1) + (lane & 7)) * SS_ROW_BYTES +
+                                (32 * warp + 16 * jp + 8 * (lane >> 4)) * 2);
+      mma_bf16_16816(oacc[2 * jp], pa, bf[0], bf[1]);
+      mma_bf16_16816(oacc[2 * jp + 1], pa, bf[2], bf[3]);
+    }
+  }
+
+  // ---- merge in base 2 (the block always has keys, so l > 0) and store
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    if (!row_ok[i]) continue;
+    const float lin2 = m[i] + log2f(l[i]);
+    const float lp2 = lp[i] * SS_LOG2E;
+    const float M = fmaxf(lp2, lin2);
+    const float wp = exp2f(lp2 - M);  // 0 when the prefix is empty (lp = -inf)
+    const float wi = exp2f(lin2 - M);
+    const float inv_den = 1.f / (wp + wi);
+    const float ao = exp2f(m[i] - M) * inv_den;  // = wi / l / den
+    const float ap = wp * inv_den;
+    __nv_bfloat16* dst = p.out_o + row_q[i] * SS_D + 32 * warp + 2 * (lane & 3);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<uint32_t*>(dst + 8 * j) = pack_bf16x2(fmaf(ap, op[i][j].x, ao * oacc[j][2 * i]),
+                                                              fmaf(ap, op[i][j].y, ao * oacc[j][2 * i + 1]));
+    if (warp == 0 && (lane & 3) == 0 && p.out_lse)
+      p.out_lse[((size_t)b * p.Hq + row_h[i]) * p.S + row_t[i]] = (M + log2f(wp + wi)) * SS_LN2;
+  }
 }
 
 }  // namespace
 
 bool small_step_fits(const fb_desc& d, int num_sms) {
-  const long long rows = (long long)d.batch * d.block_len * d.num_q_heads;
   const long long ctas = (long long)d.batch * d.num_kv_heads *
-                         ((d.block_len * (d.num_q_heads / d.num_kv_heads) + SS_ROWS_PER_CTA - 1) / SS_ROWS_PER_CTA);
-  // short blocks whose rows fill at most two waves of these CTAs
-  return d.dtype == FB_BF16 && d.head_dim == SS_D && d.block_len <= SS_MAX_S && rows > 0 &&
-         ctas <= 2LL * num_sms;
+                         ((d.block_len * (d.num_q_heads / d.num_kv_heads) + SS_ROWS - 1) / SS_ROWS);
+  // short blocks whose tiles fit one wave of these CTAs
+  return d.dtype == FB_BF16 && d.head_dim == SS_D && d.block_len <= SS_MAX_S && ctas > 0 &&
+         ctas <= (long long)num_sms;
 }
 
 cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
@@ -205,7 +259,7 @@ cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void*
   p.Hkv = d.num_kv_heads;
   p.G = d.num_q_heads / d.num_kv_heads;
   p.S = d.block_len;
-  p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  p.scale_log2 = d.softmax_scale * SS_LOG2E;
   p.Q = static_cast<const __nv_bfloat16*>(Q);
   p.Kb = static_cast<const __nv_bfloat16*>(Kb);
   p.Vb = static_cast<const __nv_bfloat16*>(Vb);
@@ -213,17 +267,15 @@ cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void*
   p.pre_lse = LSE_pre;
   p.out_o = static_cast<__nv_bfloat16*>(O);
   p.out_lse = LSE_out;
-  const int cpu = (p.S * p.G + SS_ROWS_PER_CTA - 1) / SS_ROWS_PER_CTA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(p.B * p.Hkv * cpu));
-  cfg.blockDim = dim3(SS_WARPS * 32);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, block_step_small_kernel, p);
+  const int cpu = (p.S * p.G + SS_ROWS - 1) / SS_ROWS;
+  const dim3 grid((unsigned)(p.B * p.Hkv * cpu));
+  cudaError_t e;
+  if (p.S <= 16)
+    e = launch_pdl(block_step_small_kernel<16>, grid, dim3(SS_THREADS), 0, stream, p);
+  else if (p.S <= 32)
+    e = launch_pdl(block_step_small_kernel<32>, grid, dim3(SS_THREADS), 0, stream, p);
+  else
+    e = launch_pdl(block_step_small_kernel<64>, grid, dim3(SS_THREADS), 0, stream, p);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -72,9 +72,9 @@ def test_edge_lengths(L, S, G):
 
 
 def test_block_step_kernel_choice_both_paths():
-    # short blocks with few query rows run the CUDA-core step kernel (one warp
-    # per row); with many rows the tensor-core kernel's 32- and 48-key
-    # instantiations run instead -- both against the oracle
+    # short blocks with few query rows run the warp-level MMA step kernel (16
+    # rows per CTA, all in registers); with many rows the tcgen05 kernel's 32-
+    # and 48-key instantiations run instead -- both against the oracle
     few = W["lm_gqa"].scaled(prefix_len=300, block_len=48, num_q_heads=16, num_kv_heads=2, blocks=1, steps=2)
     many32 = W["lm_gqa"].scaled(batch=12, prefix_len=300, block_len=32, blocks=1, steps=2)
     many48 = W["lm_gqa"].scaled(batch=10, prefix_len=300, block_len=48, num_q_heads=16, num_kv_heads=4,
