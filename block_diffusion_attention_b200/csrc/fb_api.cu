@@ -445,6 +445,8 @@ fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const v
                                       static_cast<const float*>(Kb), static_cast<const float*>(Vb), s));
   if (small_step_fits(*d, device_sms()))
     return from_cuda(launch_block_step_small(*d, Q, Kb, Vb, O_pre, LSE_pre, O, LSE_out, s));
+  if (rows_step_fits(*d))
+    return from_cuda(launch_block_step_rows(*d, Q, Kb, Vb, O_pre, LSE_pre, O, LSE_out, s));
   Maps m;
   CUtensorMap tm_pre, tm_out;
   if (!q_map(&m.q, *d, Q) || !block_map(&m.kb, *d, Kb) || !block_map(&m.vb, *d, Vb) ||

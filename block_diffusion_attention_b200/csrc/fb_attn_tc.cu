@@ -243,15 +243,13 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* dst, const CUtensorMap* pr
 __device__ __forceinline__ int slot_of(int item) { return item % NSLOT; }
 __device__ __forceinline__ uint32_t use_of(int item) { return (uint32_t)(item / NSLOT); }
 
-// NC: key columns a tile can hold valid keys in (128, or 32/64 for the
-// in-block step of a short block, where every tile has at most NC keys).
-template <int EPI, int NC>
+template <int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKp,
                    const __grid_constant__ CUtensorMap tmVp, const __grid_constant__ CUtensorMap tmKb,
                    const __grid_constant__ CUtensorMap tmVb, const __grid_constant__ CUtensorMap tmPre,
                    const __grid_constant__ CUtensorMap tmO, const AttnParams p) {
-  static_assert(NC == 32 || NC == 64 || NC == 128, "column count");
+  constexpr int NC = BN;  // key columns of a tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -605,19 +603,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       // P as bf16 pairs over the first 64 columns of this S buffer: the
       // A operand of PV, read from tensor memory.
-      if (NC >= 64) {
 #pragma unroll
-        for (int c = 0; c < NC / 64; ++c) {
-          uint32_t pk[32];
+      for (int c = 0; c < NC / 64; ++c) {
+        uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[c * 64 + 2 * i], s[c * 64 + 2 * i + 1]);
-          tmem_st_32x32(tS + c * 32, pk);
-        }
-      } else {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
-        tmem_st_32x16(tS, pk);
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[c * 64 + 2 * i], s[c * 64 + 2 * i + 1]);
+        tmem_st_32x32(tS + c * 32, pk);
       }
       tmem_st_wait();
       tc_fence_before_sync();
@@ -899,24 +890,20 @@ cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CU
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  // short in-block steps run the 32- or 64-column instantiation
-  const bool short_block = (p.epi == EPI_MERGE) && !p.src.has_prefix;
-  const int nc = (short_block && p.S <= 32) ? 32 : (short_block && p.S <= 64) ? 64 : 128;
   int which;
   void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
                AttnParams);
   if (p.epi == EPI_PARTIAL) {
-    kern = attn_tc_kernel<EPI_PARTIAL, 128>;
+    kern = attn_tc_kernel<EPI_PARTIAL>;
     which = 0;
   } else if (p.epi == EPI_MERGE) {
-    kern = nc == 32 ? attn_tc_kernel<EPI_MERGE, 32> : nc == 64 ? attn_tc_kernel<EPI_MERGE, 64>
-                                                               : attn_tc_kernel<EPI_MERGE, 128>;
-    which = nc == 32 ? 1 : nc == 64 ? 2 : 3;
+    kern = attn_tc_kernel<EPI_MERGE>;
+    which = 1;
   } else {
-    kern = attn_tc_kernel<EPI_NORM, 128>;
-    which = 4;
+    kern = attn_tc_kernel<EPI_NORM>;
+    which = 2;
   }
-  static bool configured[64][5] = {};
+  static bool configured[64][3] = {};
   if (dev < 64 && !configured[dev][which]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;

@@ -143,6 +143,12 @@ bool small_step_fits(const fb_desc& d, int num_sms);
 cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
                                     const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
                                     cudaStream_t stream);
+// The same on 64 query rows per CTA (16 per warp), for short blocks with more
+// rows than small_step_fits() takes: usable when rows_step_fits().
+bool rows_step_fits(const fb_desc& d);
+cudaError_t launch_block_step_rows(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
+                                   const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
+                                   cudaStream_t stream);
 
 cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
                            const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,

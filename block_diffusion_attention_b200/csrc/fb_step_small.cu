@@ -240,6 +240,178 @@ __global__ void __launch_bounds__(SS_THREADS) block_step_small_kernel(const Smal
   }
 }
 
+// The same step for many query rows: a CTA takes 64 packed rows of one
+// (b, kv head), 16 per warp, and each warp runs its own rows over all 128
+// dims (no work repeated across warps).  K, V and Q reach shared memory by
+// cp.async (52 KB at 64 keys, so four CTAs share an SM and the grid runs in
+// about one wave where the tcgen05 kernel, one CTA per SM, needs several).
+// The cached O_pre entries are loaded at the start straight into the P V
+// accumulators: the merge is taken as one more online-softmax update,
+//     M* = max(m, L2_pre),  a = 2^(L2_pre - M*),  P' = 2^(s - M*),
+//     O = (a O_pre + P' V) / (a + sum P'),  L2 = M* + log2(a + sum P'),
+// which is the merge equation with both weights at most 1, so the O_pre
+// loads are in flight with those of K, V and Q.
+constexpr int SR_ROWS = 16 * SS_WARPS;  // packed query rows per CTA
+
+template <int SP>
+constexpr uint32_t rows_smem_bytes() {
+  return (uint32_t)(SR_ROWS + 2 * SP) * SS_ROW_BYTES;
+}
+
+template <int SP>
+__global__ void __launch_bounds__(SS_THREADS, 4) block_step_rows_kernel(const SmallStepParams p) {
+  static_assert(SP % 16 == 0 && SP <= SS_MAX_S, "padded key count");
+  extern __shared__ __align__(16) uint8_t rows_smem[];
+  uint8_t* sQ = rows_smem;                      // [SR_ROWS][272]
+  uint8_t* sK = sQ + SR_ROWS * SS_ROW_BYTES;    // [SP][272]
+  uint8_t* sV = sK + SP * SS_ROW_BYTES;         // [SP][272]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows_unit = p.S * p.G;
+  const int cpu = (rows_unit + SR_ROWS - 1) / SR_ROWS;  // CTAs per unit
+  const int unit = blockIdx.x / cpu;
+  const int b = unit / p.Hkv, kvh = unit % p.Hkv;
+  const int pr0 = (blockIdx.x % cpu) * SR_ROWS;
+  const int wr0 = 16 * warp;  // this warp's first row in the CTA tile
+  const int dl = 2 * (lane & 3);
+  bool row_ok[2];
+  int row_t[2], row_h[2];
+  size_t row_q[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int pr = pr0 + wr0 + (lane >> 2) + 8 * i;
+    row_ok[i] = pr < rows_unit;
+    row_t[i] = row_ok[i] ? pr / p.G : 0;
+    row_h[i] = kvh * p.G + (row_ok[i] ? pr % p.G : 0);
+    row_q[i] = ((size_t)b * p.S + row_t[i]) * p.Hq + row_h[i];
+  }
+
+  pdl_wait();
+  pdl_launch_dependents();
+
+  // ---- K, V and Q into shared memory (padding keys and rows past the unit
+  // zero-filled); the cached pair of this lane's entries into registers:
+  // O_pre dims 8 j + 2 (lane % 4) + {0, 1} of the rows lane / 4 (entries 0,
+  // 1 of accumulator j) and lane / 4 + 8 (entries 2, 3)
+  for (int i = threadIdx.x; i < SP * 16; i += SS_THREADS) {
+    const int k = i >> 4, c = i & 15;
+    const bool ok = k < p.S;
+    const size_t src = ok ? (((size_t)b * p.S + k) * p.Hkv + kvh) * SS_D + c * 8 : 0;
+    cp_async16(smem_u32(sK + k * SS_ROW_BYTES + c * 16), p.Kb + src, ok ? 16u : 0u);
+    cp_async16(smem_u32(sV + k * SS_ROW_BYTES + c * 16), p.Vb + src, ok ? 16u : 0u);
+  }
+  for (int i = threadIdx.x; i < SR_ROWS * 16; i += SS_THREADS) {
+    const int row = i >> 4, c = i & 15;
+    const int pr = pr0 + row;
+    const bool ok = pr < rows_unit;
+    const size_t q = ok ? ((size_t)b * p.S + pr / p.G) * p.Hq + kvh * p.G + pr % p.G : 0;
+    cp_async16(smem_u32(sQ + row * SS_ROW_BYTES + c * 16), p.Q + q * SS_D + c * 8, ok ? 16u : 0u);
+  }
+  cp_async_commit();
+  float lp2[2];
+  float oacc[SS_D / 8][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    lp2[i] = row_ok[i] ? __ldg(p.pre_lse + ((size_t)b * p.Hq + row_h[i]) * p.S + row_t[i]) * SS_LOG2E
+                       : -CUDART_INF_F;
+#pragma unroll
+    for (int j = 0; j < SS_D / 8; ++j) {
+      const float2 v = row_ok[i] ? __ldg(reinterpret_cast<const float2*>(p.pre_o + row_q[i] * SS_D + 8 * j + dl))
+                                 : make_float2(0.f, 0.f);
+      oacc[j][2 * i] = v.x;
+      oacc[j][2 * i + 1] = v.y;
+    }
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  if (pr0 + wr0 >= rows_unit) return;  // this warp has no rows (no barrier follows)
+
+  // ---- S = Q K^T for the warp's 16 rows
+  const uint32_t q_base = smem_u32(sQ) + wr0 * SS_ROW_BYTES, k_base = smem_u32(sK), v_base = smem_u32(sV);
+  float sacc[SP / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < SP / 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < SS_D / 16; ++kk) {
+    uint32_t qa[4];
+    ldmatrix_x4(qa, q_base + ((lane & 7) + 8 * ((lane >> 3) & 1)) * SS_ROW_BYTES + (16 * kk + 8 * (lane >> 4)) * 2);
+#pragma unroll
+    for (int np = 0; np < SP / 16; ++np) {
+      uint32_t bf[4];
+      ldmatrix_x4(bf, k_base + (16 * np + 8 * (lane >> 4) + (lane & 7)) * SS_ROW_BYTES +
+                          (16 * kk + 8 * ((lane >> 3) & 1)) * 2);
+      mma_bf16_16816(sacc[2 * np], qa, bf[0], bf[1]);
+      mma_bf16_16816(sacc[2 * np + 1], qa, bf[2], bf[3]);
+    }
+  }
+
+  // ---- softmax against M* = max(row max, L2_pre) of rows lane / 4
+  // (entries 0, 1) and lane / 4 + 8 (entries 2, 3)
+  float mx[2] = {-CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+  for (int nt = 0; nt < SP / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = 8 * nt + 2 * (lane & 3) + (e & 1);
+      sacc[nt][e] = key < p.S ? sacc[nt][e] * p.scale_log2 : -CUDART_INF_F;
+      mx[e >> 1] = fmaxf(mx[e >> 1], sacc[nt][e]);
+    }
+  float a[2], l[2] = {0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
+    mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
+    mx[i] = fmaxf(mx[i], lp2[i]);  // M* (finite: the block always has keys)
+    a[i] = exp2f(lp2[i] - mx[i]);  // 0 when the prefix is empty
+  }
+#pragma unroll
+  for (int nt = 0; nt < SP / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      sacc[nt][e] = exp2f(sacc[nt][e] - mx[e >> 1]);
+      l[e >> 1] += sacc[nt][e];
+    }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    l[i] += __shfl_xor_sync(0xffffffffu, l[i], 1);
+    l[i] += __shfl_xor_sync(0xffffffffu, l[i], 2);
+  }
+#pragma unroll
+  for (int j = 0; j < SS_D / 8; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) oacc[j][e] *= a[e >> 1];
+
+  // ---- O = a O_pre + P' V over all 128 dims
+#pragma unroll
+  for (int kk = 0; kk < SP / 16; ++kk) {
+    const uint32_t pa[4] = {pack_bf16x2(sacc[2 * kk][0], sacc[2 * kk][1]),
+                            pack_bf16x2(sacc[2 * kk][2], sacc[2 * kk][3]),
+                            pack_bf16x2(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]),
+                            pack_bf16x2(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3])};
+#pragma unroll
+    for (int jp = 0; jp < SS_D / 16; ++jp) {
+      uint32_t bf[4];
+      ldmatrix_x4_trans(bf, v_base + (16 * kk + 8 * ((lane >> 3) & 1) + (lane & 7)) * SS_ROW_BYTES +
+                                (16 * jp + 8 * (lane >> 4)) * 2);
+      mma_bf16_16816(oacc[2 * jp], pa, bf[0], bf[1]);
+      mma_bf16_16816(oacc[2 * jp + 1], pa, bf[2], bf[3]);
+    }
+  }
+
+  // ---- normalise and store
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    if (!row_ok[i]) continue;
+    const float den = a[i] + l[i];  // >= 1: one of the two weights is 2^0
+    const float inv = 1.f / den;
+    __nv_bfloat16* dst = p.out_o + row_q[i] * SS_D + dl;
+#pragma unroll
+    for (int j = 0; j < SS_D / 8; ++j)
+      *reinterpret_cast<uint32_t*>(dst + 8 * j) = pack_bf16x2(oacc[j][2 * i] * inv, oacc[j][2 * i + 1] * inv);
+    if ((lane & 3) == 0 && p.out_lse)
+      p.out_lse[((size_t)b * p.Hq + row_h[i]) * p.S + row_t[i]] = (mx[i] + log2f(den)) * SS_LN2;
+  }
+}
+
 }  // namespace
 
 bool small_step_fits(const fb_desc& d, int num_sms) {
@@ -248,6 +420,10 @@ bool small_step_fits(const fb_desc& d, int num_sms) {
   // short blocks whose tiles fit one wave of these CTAs
   return d.dtype == FB_BF16 && d.head_dim == SS_D && d.block_len <= SS_MAX_S && ctas > 0 &&
          ctas <= (long long)num_sms;
+}
+
+bool rows_step_fits(const fb_desc& d) {
+  return d.dtype == FB_BF16 && d.head_dim == SS_D && d.block_len <= SS_MAX_S && d.batch > 0 && d.block_len > 0;
 }
 
 cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
@@ -276,6 +452,49 @@ cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void*
     e = launch_pdl(block_step_small_kernel<32>, grid, dim3(SS_THREADS), 0, stream, p);
   else
     e = launch_pdl(block_step_small_kernel<64>, grid, dim3(SS_THREADS), 0, stream, p);
+  note_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+namespace {
+template <int SP>
+cudaError_t launch_rows(const SmallStepParams& p, dim3 grid, cudaStream_t stream) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !configured[dev]) {
+    e = cudaFuncSetAttribute(block_step_rows_kernel<SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)rows_smem_bytes<SP>());
+    if (e != cudaSuccess) return e;
+    if (dev < 64) configured[dev] = true;
+  }
+  return launch_pdl(block_step_rows_kernel<SP>, grid, dim3(SS_THREADS), rows_smem_bytes<SP>(), stream, p);
+}
+}  // namespace
+
+cudaError_t launch_block_step_rows(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
+                                   const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
+                                   cudaStream_t stream) {
+  SmallStepParams p;
+  p.B = d.batch;
+  p.Hq = d.num_q_heads;
+  p.Hkv = d.num_kv_heads;
+  p.G = d.num_q_heads / d.num_kv_heads;
+  p.S = d.block_len;
+  p.scale_log2 = d.softmax_scale * SS_LOG2E;
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.Kb = static_cast<const __nv_bfloat16*>(Kb);
+  p.Vb = static_cast<const __nv_bfloat16*>(Vb);
+  p.pre_o = O_pre;
+  p.pre_lse = LSE_pre;
+  p.out_o = static_cast<__nv_bfloat16*>(O);
+  p.out_lse = LSE_out;
+  const int cpu = (p.S * p.G + SR_ROWS - 1) / SR_ROWS;
+  const dim3 grid((unsigned)(p.B * p.Hkv * cpu));
+  cudaError_t e = p.S <= 16 ? launch_rows<16>(p, grid, stream)
+                  : p.S <= 32 ? launch_rows<32>(p, grid, stream)
+                              : launch_rows<64>(p, grid, stream);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

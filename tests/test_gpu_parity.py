@@ -72,14 +72,18 @@ def test_edge_lengths(L, S, G):
 
 
 def test_block_step_kernel_choice_both_paths():
-    # short blocks with few query rows run the warp-level MMA step kernel (16
-    # rows per CTA, all in registers); with many rows the tcgen05 kernel's 32-
-    # and 48-key instantiations run instead -- both against the oracle
+    # short blocks with few query rows run the warp-level MMA step kernel with
+    # 16 rows per CTA; with more rows than one wave of those CTAs, the one
+    # with 64 rows per CTA (16 per warp) -- both against the oracle, the
+    # latter also with units whose row count leaves warps without rows (7
+    # tokens x 4 heads = 28 rows) and with one-token blocks
     few = W["lm_gqa"].scaled(prefix_len=300, block_len=48, num_q_heads=16, num_kv_heads=2, blocks=1, steps=2)
     many32 = W["lm_gqa"].scaled(batch=12, prefix_len=300, block_len=32, blocks=1, steps=2)
     many48 = W["lm_gqa"].scaled(batch=10, prefix_len=300, block_len=48, num_q_heads=16, num_kv_heads=4,
                                 blocks=1, steps=2)
-    for w in (few, many32, many48):
+    ragged7 = W["lm_gqa"].scaled(batch=10, prefix_len=300, block_len=7, blocks=2, steps=2)
+    one = W["lm_gqa"].scaled(batch=40, prefix_len=129, block_len=1, blocks=2, steps=2)
+    for w in (few, many32, many48, ragged7, one):
         gpu_cases.run_workload(w)
 
 
