@@ -46,10 +46,7 @@ METRIC = "attention µs/denoise-step and tokens/s, cached vs uncached; prefix-pa
 # workload (dram__bytes_read.sum + dram__bytes_write.sum).  An entry holds only
 # for the kernel source it was captured with: re-capture, or drop it, when the
 # kernel changes.
-NCU_TRAFFIC = {
-    "long_ctx": 537217536 + 4151552,
-    "video": 719510272 + 89014528,
-}
+NCU_TRAFFIC = {}
 
 
 def parse():

@@ -14,15 +14,18 @@
 // pairs of one kv head, so each K/V tile that TMA brings in is used by all G
 // query heads of the group.
 //
-// Warp roles (192 threads):
+// Warp roles (224 threads):
 //   warps 0-3  softmax: thread r owns query row r (TMEM lane r); copies its Q
 //              row into tensor memory, then online softmax in fp32 with
 //              base-2 exponentials (a quarter of them on the FMA pipe), P
 //              written back into tensor memory as bf16 pairs, lazy rescaling
 //              of the accumulator, epilogue (output tile staged in shared
 //              memory, written by TMA stores);
-//   warp 4     TMA producer: Q once, then K and V tiles into a ring of six
-//              32 KB shared-memory slots (K and V of a tile take one slot each);
+//   warp 4     TMA producer of Q (once) and the K tiles, warp 6 of the V
+//              tiles, into a ring of six 32 KB shared-memory slots (tile j's
+//              K takes an even slot, its V an odd one): each producer refills
+//              its own slots as soon as they are consumed, so a K load never
+//              waits behind the release of a V slot;
 //   warp 5     TMEM owner; its lane 0 issues the tcgen05.mma: S = Q K^T (A = Q
 //              from tensor memory, B = K from shared memory) and O += P V (A =
 //              P from tensor memory, B = V from shared memory), M = 128,
@@ -363,15 +366,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (skip) {
     // nothing to load, multiply or write
-  } else if (warp == 4) {
-    // ------------------------------------------------------------ TMA producer
+  } else if (warp == 4 || warp == 6) {
+    // ----------------------------------------------------------- TMA producers
     if (lane == 0) {
+      const int kv = warp == 6 ? 1 : 0;  // this producer's items: 2 jj + kv
       const uint64_t policy = p.kv_stream_once ? l2_policy_evict_first() : l2_policy_evict_normal();
-      mbar_arrive_expect_tx(sh.q_full, Q_BYTES);
       const int t0 = rt * (BM / p.G);
-      tma_load_4d(sQ, &tmQ, sh.q_full, 0, kvh * p.G, t0, b);
-      tma_load_4d(sQ + BM * 128, &tmQ, sh.q_full, 64, kvh * p.G, t0, b);
-      if (pre_smem) {
+      if (kv == 0) {
+        mbar_arrive_expect_tx(sh.q_full, Q_BYTES);
+        tma_load_4d(sQ, &tmQ, sh.q_full, 0, kvh * p.G, t0, b);
+        tma_load_4d(sQ + BM * 128, &tmQ, sh.q_full, 64, kvh * p.G, t0, b);
+      }
+      if (kv == 0 && pre_smem) {
         // [4 column blocks of 32 floats][128 rows][128 B], 128-byte swizzle
         mbar_arrive_expect_tx(sh.pre_full, PRE_BYTES);
 #pragma unroll
@@ -379,28 +385,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           tma_load_4d(sRing + PRE_SLOT * SLOT_BYTES + c * (BM * 128), &tmPre, sh.pre_full, c * 32, kvh * p.G,
                       t0, b);
       }
-      int issued = 0;  // ring items issued
+      int issued = 0;  // tiles whose item this producer has issued
       for (int jj = 0; jj < nt; ++jj) {
         const Tile t = tile_at(p, u, b, kvh, j0 + jj);
-        bool ok = true;
-#pragma unroll
-        for (int kv = 0; kv < 2; ++kv) {
-          const int item = 2 * jj + kv;
-          const int sl = slot_of(item);
-          if (!(ok = wait_bar(&sh.empty[sl], (use_of(item) & 1) ^ 1, sh, status))) break;
-          mbar_arrive_expect_tx(&sh.full[sl], SLOT_BYTES);
-          load_kv_tile(sRing + sl * SLOT_BYTES, kv ? &tmVp : &tmKp, kv ? &tmVb : &tmKb, &sh.full[sl], p, u,
-                       t, b, kvh, policy);
-          issued = item + 1;
-        }
-        if (!ok) break;
+        const int item = 2 * jj + kv;
+        const int sl = slot_of(item);
+        if (!wait_bar(&sh.empty[sl], (use_of(item) & 1) ^ 1, sh, status)) break;
+        mbar_arrive_expect_tx(&sh.full[sl], SLOT_BYTES);
+        load_kv_tile(sRing + sl * SLOT_BYTES, kv ? &tmVp : &tmKp, kv ? &tmVb : &tmKb, &sh.full[sl], p, u, t, b,
+                     kvh, policy);
+        issued = jj + 1;
       }
-      // After an abort, let the copies in flight land before the CTA exits.
+      // After an abort, let the copies in flight land before the CTA exits
+      // (this producer's own: its last NSLOT / 2 items at most).
       if (*sh.abort_flag) {
-        wait_bar(sh.q_full, 0, sh, nullptr, false);
-        if (pre_smem) wait_bar(sh.pre_full, 0, sh, nullptr, false);
-        for (int item = max(0, issued - NSLOT); item < issued; ++item)
+        if (kv == 0) wait_bar(sh.q_full, 0, sh, nullptr, false);
+        if (kv == 0 && pre_smem) wait_bar(sh.pre_full, 0, sh, nullptr, false);
+        for (int jj = max(0, issued - NSLOT / 2); jj < issued; ++jj) {
+          const int item = 2 * jj + kv;
           wait_bar(&sh.full[slot_of(item)], use_of(item) & 1, sh, nullptr, false);
+        }
       }
     }
   } else if (warp == 5) {

@@ -76,7 +76,7 @@ constexpr int TC_BM = 128;      // query rows per tile (TMEM lanes)
 constexpr int TC_BN = 128;      // keys per tile
 constexpr int TC_D = 128;       // head dim
 constexpr int TC_SLOTS = 6;     // K/V ring: 32 KB slots (K and V of a tile take one each)
-constexpr int TC_THREADS = 192; // 4 softmax warps + TMA warp + MMA warp
+constexpr int TC_THREADS = 224; // 4 softmax warps, K/Q TMA warp, MMA warp, V TMA warp
 constexpr int TC_MAX_SPLITS = 128;  // key-range splits per work unit
 size_t tc_smem_bytes();
 // Launch with programmatic stream serialization: the kernel may start while

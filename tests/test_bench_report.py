@@ -55,7 +55,8 @@ def test_report_line_has_contract_keys(capsys, kw):
     if args.workload == "batched_sparse":
         assert line["chunk_select_us"] == pytest.approx(20.0)
     if args.workload == "long_ctx" and not args.residual:
-        assert roof["traffic"] == bench.NCU_TRAFFIC["long_ctx"]
+        # the recorded capture of the current kernel, or null when there is none
+        assert roof["traffic"] == bench.NCU_TRAFFIC.get("long_ctx")
 
 
 def test_report_without_e2e_phase(capsys):
