@@ -64,7 +64,7 @@ constexpr uint32_t HALF_BYTES = BN * 128;       // one 64-column half of a tile
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_RING = OFF_Q + Q_BYTES;
 constexpr uint32_t OFF_BAR = OFF_RING + NSLOT * SLOT_BYTES;
-constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 + 2 + 4;
+constexpr int NUM_BARS = 1 + 2 * NSLOT + 2 + 2 + 5;
 constexpr uint32_t PRE_BYTES = BM * HD * 4;      // 64 KB: O_pre rows of a tile (f32)
 constexpr int PRE_SLOT = NSLOT - 2;             // O_pre prefetch uses the last two ring slots
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
@@ -84,7 +84,7 @@ struct Shared {
   uint64_t* empty;   // [NSLOT] ring slot consumed
   uint64_t* s_full;  // [2] S buffer written by QK^T
   uint64_t* p_full;  // [2] P written into that S buffer (and O rescaled)
-  uint64_t* o_done;  // PV finished
+  uint64_t* o_done;  // [2] PV(j) finished: barrier j % 2
   uint64_t* drain;
   uint64_t* pre_full; // O_pre rows prefetched (merge epilogue of short units)
   uint64_t* q_tmem;   // Q copied into tensor memory by the softmax warps
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   sh.s_full = sh.empty + NSLOT;
   sh.p_full = sh.s_full + 2;
   sh.o_done = sh.p_full + 2;
-  sh.drain = sh.o_done + 1;
+  sh.drain = sh.o_done + 2;
   sh.pre_full = sh.drain + 1;
   sh.q_tmem = sh.pre_full + 1;
   sh.tmem_slot = reinterpret_cast<uint32_t*>(sh.q_tmem + 1);
@@ -286,7 +286,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&sh.s_full[i], 1);
       mbar_init(&sh.p_full[i], 4);
     }
-    mbar_init(sh.o_done, 1);
+    mbar_init(&sh.o_done[0], 1);
+    mbar_init(&sh.o_done[1], 1);
     mbar_init(sh.drain, 1);
     mbar_init(sh.pre_full, 1);
     mbar_init(sh.q_tmem, 4);
@@ -441,9 +442,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           umma_bf16_ts(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
     };
     // One thread (lane 0) runs the issue loop; the other lanes wait at the
-    // warp barrier below.  The loop keeps the work between "P of tile j is
-    // ready" and the PV(j) issue to one barrier test: V(j) is waited for, its
-    // tail rows cleared and tile j + 1 located before QK^T(j + 1) is issued.
+    // warp barrier below.  Per tile j: QK^T(j + 1) as soon as K(j + 1) has
+    // landed (the tensor pipe then works while the softmax of tile j runs),
+    // then V(j) is waited for and its tail rows cleared, so that the work
+    // between "P of tile j is ready" and the PV(j) issue is one barrier test.
     // (This warp shares its scheduler with a softmax warp, so every
     // instruction on that path delays the tensor pipe.)
     if (lane == 0) {
@@ -458,6 +460,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           tc_commit(&sh.empty[slot_of(0)]);
         }
         for (int jj = 0; ok && jj < nt; ++jj) {
+          Tile tn = tc;
+          if (jj + 1 < nt) {
+            tn = tile_at(p, u, b, kvh, j0 + jj + 1);
+            const int ik = 2 * (jj + 1);
+            if (!(ok = wait_bar(&sh.full[slot_of(ik)], use_of(ik) & 1, sh, status))) break;
+            tc_fence_after_sync();
+            issue_qk(jj + 1, tn.nvalid);
+            tc_commit(&sh.s_full[(jj + 1) & 1]);
+            tc_commit(&sh.empty[slot_of(ik)]);
+          }
           const int iv = 2 * jj + 1;
           if (!(ok = wait_bar(&sh.full[slot_of(iv)], use_of(iv) & 1, sh, status))) break;
           if (tc.seg == 0 && (tc.nvalid & 15)) {
@@ -474,20 +486,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             fence_proxy_async_smem();
           }
-          Tile tn = tc;
-          if (jj + 1 < nt) {
-            tn = tile_at(p, u, b, kvh, j0 + jj + 1);
-            const int ik = 2 * (jj + 1);
-            if (!(ok = wait_bar(&sh.full[slot_of(ik)], use_of(ik) & 1, sh, status))) break;
-            tc_fence_after_sync();
-            issue_qk(jj + 1, tn.nvalid);
-            tc_commit(&sh.s_full[(jj + 1) & 1]);
-            tc_commit(&sh.empty[slot_of(ik)]);
-          }
           if (!(ok = wait_bar(&sh.p_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
           tc_fence_after_sync();
           issue_pv(jj, tc.nvalid);
-          tc_commit(sh.o_done);
+          tc_commit(&sh.o_done[jj & 1]);
           tc_commit(&sh.empty[slot_of(iv)]);
           tc = tn;
         }
@@ -587,22 +589,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       l_run = l_run * alpha + ((l0 + l1) + (l2 + l3));
       m_run = m_new;
 
-      if (jj > 0) {
-        // Wait for the previous tile's PV before publishing this tile's P:
-        // o_done then never runs more than one phase ahead of this wait, and
-        // the accumulator is stable if rows whose max moved need rescaling.
-        if (!(ok = wait_bar_warp(sh.o_done, (jj - 1) & 1, sh, status))) break;
+      if (jj > 0 && __any_sync(0xffffffffu, need)) {
+        // Rows whose max moved rescale the accumulator once PV(j - 1) is
+        // done.  PV(j - 1) commits to o_done[(j - 1) % 2], whose next phase
+        // is PV(j + 1), behind this tile's P: the barrier is never two phases
+        // ahead of this wait even though tiles without a rescale skip it.
+        if (!(ok = wait_bar_warp(&sh.o_done[(jj - 1) & 1], ((jj - 1) >> 1) & 1, sh, status))) break;
         tc_fence_after_sync();
-        if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int c = 0; c < HD / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld_32x32(tO + c * 32, ov);
-            tmem_ld_wait();
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld_32x32(tO + c * 32, ov);
+          tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st_32x32(tO + c * 32, ov);
-          }
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st_32x32(tO + c * 32, ov);
         }
       }
       // P as bf16 pairs over the first 64 columns of this S buffer: the
@@ -620,7 +621,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (lane == 0) mbar_arrive(&sh.p_full[jj & 1]);
     }
     if (ok && nt > 0) {
-      ok = wait_bar_warp(sh.o_done, (nt - 1) & 1, sh, status);
+      ok = wait_bar_warp(&sh.o_done[(nt - 1) & 1], ((nt - 1) >> 1) & 1, sh, status);
       tc_fence_after_sync();
     }
     if (ok && pre_smem) ok = wait_bar_warp(sh.pre_full, 0, sh, status);
