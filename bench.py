@@ -46,7 +46,10 @@ METRIC = "attention µs/denoise-step and tokens/s, cached vs uncached; prefix-pa
 # workload (dram__bytes_read.sum + dram__bytes_write.sum).  An entry holds only
 # for the kernel source it was captured with: re-capture, or drop it, when the
 # kernel changes.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    "long_ctx": 537221376 + 3742464,
+    "video": 719319808 + 88570624,
+}
 
 
 def parse():
