@@ -417,6 +417,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // from its base is the base descriptor plus off >> 4 (start-address field).
     const uint64_t dK = sw128_desc(smem_u32(sRing), 16, 1024);
     const uint64_t dV = sw128_desc(smem_u32(sRing), HALF_BYTES, 1024);
+    // The whole warp runs the issue loop, so tile indices, descriptors and
+    // tensor-memory addresses are warp-uniform values; one elected lane issues
+    // each group of tcgen05.mma and its commits.
+    const bool leader = elect_one_sync();
     // A tile with fewer valid keys runs N = (valid keys rounded up to 16) for
     // QK^T and as many 16-key steps of PV: no work on empty columns.
     auto issue_qk = [&](int jj, int nvalid) {
@@ -426,77 +430,86 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t tS = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN;
       // A = Q from tensor memory (16 dims = 8 packed columns per step), B = K
       // from shared memory: only K crosses the shared-memory read port
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
-        umma_bf16_ts(tS, tmem + TMEM_Q + kk * 8, dk + off, idesc, kk > 0);
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+          umma_bf16_ts(tS, tmem + TMEM_Q + kk * 8, dk + off, idesc, kk > 0);
+        }
       }
     };
     auto issue_pv = [&](int jj, int nvalid) {
       const uint64_t dv = dV + ((slot_of(2 * jj + 1) * SLOT_BYTES) >> 4);
       const uint32_t tP = tmem + TMEM_S0 + (uint32_t)(jj & 1) * BN;  // P (bf16 pairs) over S
       const int ksteps = (nvalid + 15) >> 4;
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < NC / 16; ++kk)
-        if (kk < ksteps)
-          umma_bf16_ts(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < NC / 16; ++kk)
+          if (kk < ksteps)
+            umma_bf16_ts(tO, tP + kk * 8, dv + ((kk * 16 * 128) >> 4), IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+      }
     };
-    // One thread (lane 0) runs the issue loop; the other lanes wait at the
-    // warp barrier below.  Per tile j: QK^T(j + 1) as soon as K(j + 1) has
-    // landed (the tensor pipe then works while the softmax of tile j runs),
-    // then V(j) is waited for and its tail rows cleared, so that the work
-    // between "P of tile j is ready" and the PV(j) issue is one barrier test.
-    // (This warp shares its scheduler with a softmax warp, so every
-    // instruction on that path delays the tensor pipe.)
-    if (lane == 0) {
-      bool ok = wait_bar(sh.q_tmem, 0, sh, status);
-      if (ok && nt > 0) {
-        Tile tc = tile_at(p, u, b, kvh, j0);
-        ok = wait_bar(&sh.full[slot_of(0)], 0, sh, status);
-        if (ok) {
-          tc_fence_after_sync();
-          issue_qk(0, tc.nvalid);
+    // Per tile j: QK^T(j + 1) as soon as K(j + 1) has landed (the tensor pipe
+    // then works while the softmax of tile j runs), then V(j) is waited for
+    // and its tail rows cleared, so that the work between "P of tile j is
+    // ready" and the PV(j) issue is one barrier test.  (This warp shares its
+    // scheduler with a softmax warp, so every instruction on that path
+    // delays the tensor pipe.)
+    bool ok = wait_bar_warp(sh.q_tmem, 0, sh, status);
+    if (ok && nt > 0) {
+      Tile tc = tile_at(p, u, b, kvh, j0);
+      ok = wait_bar_warp(&sh.full[slot_of(0)], 0, sh, status);
+      if (ok) {
+        tc_fence_after_sync();
+        issue_qk(0, tc.nvalid);
+        if (leader) {
           tc_commit(&sh.s_full[0]);
           tc_commit(&sh.empty[slot_of(0)]);
         }
-        for (int jj = 0; ok && jj < nt; ++jj) {
-          Tile tn = tc;
-          if (jj + 1 < nt) {
-            tn = tile_at(p, u, b, kvh, j0 + jj + 1);
-            const int ik = 2 * (jj + 1);
-            if (!(ok = wait_bar(&sh.full[slot_of(ik)], use_of(ik) & 1, sh, status))) break;
-            tc_fence_after_sync();
-            issue_qk(jj + 1, tn.nvalid);
+      }
+      for (int jj = 0; ok && jj < nt; ++jj) {
+        Tile tn = tc;
+        if (jj + 1 < nt) {
+          tn = tile_at(p, u, b, kvh, j0 + jj + 1);
+          const int ik = 2 * (jj + 1);
+          if (!(ok = wait_bar_warp(&sh.full[slot_of(ik)], use_of(ik) & 1, sh, status))) break;
+          tc_fence_after_sync();
+          issue_qk(jj + 1, tn.nvalid);
+          if (leader) {
             tc_commit(&sh.s_full[(jj + 1) & 1]);
             tc_commit(&sh.empty[slot_of(ik)]);
           }
-          const int iv = 2 * jj + 1;
-          if (!(ok = wait_bar(&sh.full[slot_of(iv)], use_of(iv) & 1, sh, status))) break;
-          if (tc.seg == 0 && (tc.nvalid & 15)) {
-            // Cache rows past the prefix may hold anything (even NaN); P is 0
-            // there but 0 * NaN is not, so clear the V rows up to the next
-            // 16-key step that PV reads (at most 15 rows, once per unit).
-            uint8_t* dV = sRing + slot_of(iv) * SLOT_BYTES;
-            const int nrow = ((tc.nvalid + 15) & ~15) - tc.nvalid;
-            for (int i = 0; i < nrow * 16; ++i) {
-              const int r = tc.nvalid + (i >> 4);
-              const int h = (i >> 3) & 1;
-              const int c = i & 7;
-              *reinterpret_cast<uint4*>(dV + h * HALF_BYTES + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
+        }
+        const int iv = 2 * jj + 1;
+        if (!(ok = wait_bar_warp(&sh.full[slot_of(iv)], use_of(iv) & 1, sh, status))) break;
+        if (tc.seg == 0 && (tc.nvalid & 15)) {
+          // Cache rows past the prefix may hold anything (even NaN); P is 0
+          // there but 0 * NaN is not, so clear the V rows up to the next
+          // 16-key step that PV reads (at most 15 rows, once per unit), the
+          // warp's lanes sharing the 16-byte stores.
+          uint8_t* dVs = sRing + slot_of(iv) * SLOT_BYTES;
+          const int nrow = ((tc.nvalid + 15) & ~15) - tc.nvalid;
+          for (int i = lane; i < nrow * 16; i += 32) {
+            const int r = tc.nvalid + (i >> 4);
+            const int h = (i >> 3) & 1;
+            const int c = i & 7;
+            *reinterpret_cast<uint4*>(dVs + h * HALF_BYTES + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
           }
-          if (!(ok = wait_bar(&sh.p_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
-          tc_fence_after_sync();
-          issue_pv(jj, tc.nvalid);
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (!(ok = wait_bar_warp(&sh.p_full[jj & 1], (jj >> 1) & 1, sh, status))) break;
+        tc_fence_after_sync();
+        issue_pv(jj, tc.nvalid);
+        if (leader) {
           tc_commit(&sh.o_done[jj & 1]);
           tc_commit(&sh.empty[slot_of(iv)]);
-          tc = tn;
         }
+        tc = tn;
       }
-      // Drain every MMA this thread issued before TMEM can be released.
-      tc_commit(sh.drain);
     }
+    // Drain every MMA this warp issued before TMEM can be released.
+    if (leader) tc_commit(sh.drain);
     __syncwarp();
     wait_bar(sh.drain, 0, sh, nullptr, false);
   } else {
