@@ -26,10 +26,12 @@
 //              K takes an even slot, its V an odd one): each producer refills
 //              its own slots as soon as they are consumed, so a K load never
 //              waits behind the release of a V slot;
-//   warp 5     TMEM owner; its lane 0 issues the tcgen05.mma: S = Q K^T (A = Q
-//              from tensor memory, B = K from shared memory) and O += P V (A =
-//              P from tensor memory, B = V from shared memory), M = 128,
-//              N = 128, K = 16.
+//   warp 5     TMEM owner and MMA issuer: the whole warp runs the issue loop
+//              (warp-uniform tile indices and descriptors) and one elected
+//              lane issues the tcgen05.mma: S = Q K^T (A = Q from tensor
+//              memory, B = K from shared memory) and O += P V (A = P from
+//              tensor memory, B = V from shared memory), M = 128, N = 128,
+//              K = 16.
 //
 // TMEM (512 columns): S double-buffered at columns [0, 128) and [128, 256) --
 // tile j's P overwrites the first 64 columns of its own S buffer -- the O
