@@ -47,8 +47,7 @@ METRIC = "attention µs/denoise-step and tokens/s, cached vs uncached; prefix-pa
 # for the kernel source it was captured with: re-capture, or drop it, when the
 # kernel changes.
 NCU_TRAFFIC = {
-    "long_ctx": 537205248 + 3760128,
-    "video": 719354624 + 91463168,
+    "long_ctx": 537219072 + 3548160,
 }
 
 

@@ -510,10 +510,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tc = tn;
       }
     }
-    // Drain every MMA this warp issued before TMEM can be released.
+    // Drain every MMA this warp issued before TMEM can be released (a drain
+    // that runs out of time is recorded too, unless an error already is).
     if (leader) tc_commit(sh.drain);
     __syncwarp();
-    wait_bar(sh.drain, 0, sh, nullptr, false);
+    wait_bar(sh.drain, 0, sh, status, false);
   } else {
     // ------------------------------------------------------ softmax + epilogue
     const int r = warp * 32 + lane;  // query row of this thread = TMEM lane
