@@ -71,6 +71,17 @@ def test_edge_lengths(L, S, G):
     gpu_cases.run_workload(w)
 
 
+@pytest.mark.parametrize("B,L,S,G", [(1, 300, 32, 32), (1, 200, 16, 64), (1, 150, 130, 32), (3, 260, 64, 32)])
+def test_wide_groups(B, L, S, G):
+    # 32 and 64 query heads per kv head: a 128-row query tile holds 4 or 2
+    # tokens of one group in the prefix pass; the step runs the 16-row MMA
+    # kernel (the first two), the tcgen05 kernel (S > 64, ragged query tiles)
+    # and the 64-row MMA kernel (the last)
+    w = W["lm_gqa"].scaled(batch=B, prefix_len=L, block_len=S, num_q_heads=2 * G, num_kv_heads=2, blocks=2,
+                           steps=2)
+    gpu_cases.run_workload(w)
+
+
 def test_block_step_kernel_choice_both_paths():
     # short blocks with few query rows run the warp-level MMA step kernel with
     # 16 rows per CTA; with more rows than one wave of those CTAs, the one
