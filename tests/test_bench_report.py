@@ -65,3 +65,26 @@ def test_report_without_e2e_phase(capsys):
     bench.report(args, synth.WORKLOADS["long_ctx"], w, 1, _res(w, with_e2e=False, ms_unc=None))
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["e2e"] is None and line["uncached_us_per_denoise_step"] is None
+
+
+def test_reference_arm_line(capsys, monkeypatch):
+    # the reference arm times the oracle on the host: a real run on the tiny
+    # workload (seconds), its line carrying the contract's keys
+    monkeypatch.delenv("RANK", raising=False)
+    args = _args(workload="tiny_fp32", impl="reference", steps=1, warmup=0)
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["higher_is_better"] is True and line["steps"] == 1 and line["warmup"] == 0
+    assert line["config"]["workload"].startswith("tiny_fp32")
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_do_no_work(capsys, monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    args = _args(workload="tiny_fp32", impl="reference", steps=1, warmup=0)
+    assert bench.run_reference(args) == 0
+    assert capsys.readouterr().out.strip() == ""
