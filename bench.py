@@ -43,12 +43,32 @@ METRIC = "attention µs/denoise-step and tokens/s, cached vs uncached; prefix-pa
 
 # DRAM bytes read + written by one launch of the prefix-pass attention kernel,
 # from one `ncu --set full --clock-control none` capture of that launch on the
-# workload (dram__bytes_read.sum + dram__bytes_write.sum).  An entry holds only
-# for the kernel source it was captured with: re-capture, or drop it, when the
-# kernel changes.
-NCU_TRAFFIC = {
-    "long_ctx": 537219072 + 3548160,
-}
+# workload (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the
+# kernel sources it was captured on (see kernel_source_hash).  An entry whose
+# hash differs from the built sources is not reported: the kernel changed
+# since the counters were taken.
+NCU_TRAFFIC = {}
+KERNEL_SOURCES = ("fb_attn_tc.cu", "fb_ptx.cuh", "fb_internal.h", "fb_api.cu")
+
+
+def kernel_source_hash():
+    """sha256 (first 16 hex digits) over the sources that decide the prefix
+    pass's kernel code and launch plan."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "block_diffusion_attention_b200", "csrc", name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """Captured DRAM bytes per prefix-pass launch, or None when there is no
+    capture of the current kernel sources."""
+    e = NCU_TRAFFIC.get(workload)
+    if e is None or e["sources"] != kernel_source_hash():
+        return None
+    return e["bytes"]
 
 
 def parse():
@@ -211,7 +231,9 @@ def cpu_threads():
 def oracle_block_sample(w, K, V, lens, heads=1):
     """Time the oracle's cached block on the first `heads` kv heads of the
     workload (one block: refresh + every denoising step's in-block partial and
-    merge); returns seconds scaled to all kv heads."""
+    merge).  Returns the measured seconds of that sample; the sample does
+    heads / Hkv of the block's attention work (the kv heads are independent
+    and equal in size)."""
     import numpy as np
     from block_diffusion_attention_b200 import synth
     from oracle import flashblock_oracle as ora
@@ -234,8 +256,20 @@ def oracle_block_sample(w, K, V, lens, heads=1):
     t0 = time.perf_counter()
     ora.cached_block([x[0] for x in steps], [x[1] for x in steps], [x[2] for x in steps], Kc, Vc, lens64,
                      w.softmax_scale, w.refresh, chunk_fn, w.chunk_size)
-    dt = time.perf_counter() - t0
-    return dt * (w.num_kv_heads / heads)
+    return time.perf_counter() - t0
+
+
+def oracle_sample_record(w, seconds, heads=1):
+    """The oracle's measured sample as a rate: the sample finalizes
+    heads / Hkv of the attention of the block's B * S tokens, so its
+    throughput is B * S * heads / Hkv tokens over the measured seconds (no
+    time is extrapolated)."""
+    frac = heads / w.num_kv_heads
+    return {"value": w.batch * w.block_len * frac / seconds, "unit": "tokens/s",
+            "sample": f"the oracle's cached block (refresh + {w.steps} denoising steps) on {heads} of "
+                      f"{w.num_kv_heads} kv heads, i.e. {frac:g} of the block's attention work; the rate is "
+                      f"that work over its measured time",
+            "sample_seconds_measured": seconds, "sample_fraction_of_block": frac}
 
 
 def run_reference(args):
@@ -250,17 +284,19 @@ def run_reference(args):
         t = oracle_block_sample(w, K, V, lens, heads=1)
         if i >= args.warmup:
             times.append(t)
-    per_block = sum(times) / len(times)
-    tok_s = w.batch * w.block_len / per_block
+    per_step = sum(times) / len(times)  # measured seconds of one sample step
+    rec = oracle_sample_record(w, per_step, heads=1)
+    tok_s = rec["value"]
     line = {
         "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_block * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w),
-        "cached_us_per_denoise_step": per_block / w.steps * 1e6,
+        "step": "one bounded sample of the workload's block (see cpu_baseline.sample); ms_per_step is its "
+                "measured time",
         "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-                         "sample": f"each step: the oracle's cached block on 1 of {w.num_kv_heads} kv heads, "
-                                   f"time scaled x{w.num_kv_heads}"},
+                         "sample": rec["sample"], "sample_seconds_measured": per_step,
+                         "sample_fraction_of_block": rec["sample_fraction_of_block"]},
         "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -602,7 +638,7 @@ def report(args, w0, w, world, res):
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_source": f"{peak_kind} hbm_gbs",
                 "tensor_tflops": tflops, "tensor_frac": tflops / tc_peak}
-    traffic = None if args.residual else NCU_TRAFFIC.get(w.name)
+    traffic = None if args.residual else recorded_traffic(w.name)
     roof.update({"traffic": traffic,
                  "traffic_over_algorithmic": (traffic / abytes) if traffic else None,
                  "kernel": "prefix pass: attn_tc_kernel<EPI_PARTIAL> (+ combine_kernel when split)",
@@ -648,10 +684,7 @@ def report(args, w0, w, world, res):
     if not args.no_cpu_baseline and world == 1:
         K, V, lens_np = synth.prefix_kv(w0)
         t = oracle_block_sample(w0, K, V, lens_np, heads=1)
-        line["cpu_baseline"] = {
-            "value": w0.batch * w0.block_len / t, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"the oracle's cached block (refresh + {w0.steps} steps) on 1 of {w0.num_kv_heads} kv heads, "
-                      f"time scaled x{w0.num_kv_heads}"}
+        line["cpu_baseline"] = dict(oracle_sample_record(w0, t, heads=1), cores=cpu_threads(), kind="oracle")
     print(json.dumps(line), flush=True)
 
 

@@ -50,14 +50,19 @@ bool make_map(CUtensorMap* m, const void* base, const uint64_t dims[4], const ui
   return r == CUDA_SUCCESS;
 }
 
+// SM count of the current device, cached per device (host threads may call
+// concurrently: each entry is written once with the same value, atomically).
 int device_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  static int cache[64] = {0};
-  if (dev < 64 && cache[dev]) return cache[dev];
+  static std::atomic<int> cache[64];
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  if (dev < 64) cache[dev] = n;
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 

@@ -51,6 +51,8 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <atomic>
+
 #include "fb_internal.h"
 #include "fb_ptx.cuh"
 
@@ -924,11 +926,12 @@ cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CU
     kern = attn_tc_kernel<EPI_NORM>;
     which = 2;
   }
-  static bool configured[64][3] = {};
-  if (dev < 64 && !configured[dev][which]) {
+  // (set once per device and kernel; concurrent first calls both set it)
+  static std::atomic<bool> configured[64][3];
+  if (dev >= 64 || !configured[dev][which].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    configured[dev][which] = true;
+    if (dev < 64) configured[dev][which].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);

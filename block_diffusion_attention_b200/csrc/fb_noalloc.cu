@@ -1,16 +1,18 @@
 // fb_noalloc.cu -- the prefix pass for callers that cannot allocate device
 // memory.
 //
-// Some callers are not allowed to call cudaMalloc at all: a host program that
-// records its work into a CUDA graph (allocation is not a capturable
-// operation), an embedding that owns a fixed device-memory arena and forbids
-// allocator calls once it is running, or a serving loop that cannot afford
-// the device-wide synchronisation an allocation may cause.  For them the
-// split-key partials of the prefix pass live in a fixed scratch array that is
-// part of this library's device image instead of a caller-owned workspace.
+// Some callers are not allowed to call cudaMalloc at all: an embedding whose
+// memory planner hands out one fixed device arena at start-up and forbids
+// allocator calls once it is running, a plug-in host that gives its plug-ins
+// no allocator of their own, or a latency-critical serving loop that cannot
+// afford the device-wide synchronisation a cudaMalloc or cudaFree may cause.
+// For them the split-key partials of the prefix pass live in a fixed scratch
+// array that is part of this library's device image instead of a
+// caller-owned workspace.
 //
 // The array (FB_NOALLOC_SCRATCH_BYTES, 16 MiB) exists on every GPU that loads
 // the library, for as long as the process runs.  All calls share it.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -22,27 +24,74 @@ namespace {
 constexpr size_t kScratchBytes = FB_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_addr[64] = {};  // device address of the array, per device
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// On the host, g_noalloc_scratch names a host-side shadow, not device memory;
-// the kernels need the device address, looked up once per device with that
-// device current.
+struct DriverFns {
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+};
+
+DriverFns driver_fns() {
+  static DriverFns fns;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  return fns;
+}
+
+// Unique id of the calling thread's current context (0 if there is none yet
+// or the driver cannot say).  A device reset ends the context: the next one
+// gets a new id, and the library's device image (with the array) is loaded
+// into it again, possibly at another address.
+unsigned long long current_context_id() {
+  const DriverFns f = driver_fns();
+  if (!f.get_current || !f.get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  unsigned long long id = 0;
+  if (f.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+struct ScratchEntry {
+  unsigned long long ctx_id = 0;
+  void* addr = nullptr;
+};
+std::mutex g_scratch_mu;
+ScratchEntry g_scratch[64];  // per device
+
+// On the host, g_noalloc_scratch names a host-side stand-in, not device
+// memory: the kernels need the array's device address, looked up with the
+// device current, once per device and again whenever the device's context has
+// changed (after a device reset).
 fb_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FB_ERR_LAUNCH;
   if (dev < 0 || dev >= 64) return FB_ERR_UNSUPPORTED;
+  const unsigned long long id = current_context_id();
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  ScratchEntry& e = g_scratch[dev];
+  if (!e.addr || id == 0 || id != e.ctx_id) {
     void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr) {
+    const cudaError_t err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (err != cudaSuccess || p == nullptr) {
       cudaGetLastError();  // do not leave the error for the caller's next call
       return FB_ERR_LAUNCH;
     }
-    g_scratch_addr[dev] = p;
+    e.addr = p;
+    // the lookup above created the context if there was none
+    e.ctx_id = current_context_id();
   }
-  *out = g_scratch_addr[dev];
+  *out = e.addr;
   return FB_OK;
 }
 

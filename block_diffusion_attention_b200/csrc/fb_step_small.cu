@@ -25,6 +25,8 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <atomic>
+
 #include "fb_internal.h"
 #include "fb_ptx.cuh"
 
@@ -459,15 +461,15 @@ cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void*
 namespace {
 template <int SP>
 cudaError_t launch_rows(const SmallStepParams& p, dim3 grid, cudaStream_t stream) {
-  static bool configured[64] = {};
+  static std::atomic<bool> configured[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !configured[dev]) {
+  if (dev >= 64 || !configured[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(block_step_rows_kernel<SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)rows_smem_bytes<SP>());
     if (e != cudaSuccess) return e;
-    if (dev < 64) configured[dev] = true;
+    if (dev < 64) configured[dev].store(true, std::memory_order_release);
   }
   return launch_pdl(block_step_rows_kernel<SP>, grid, dim3(SS_THREADS), rows_smem_bytes<SP>(), stream, p);
 }

@@ -229,13 +229,16 @@ fb_status fb_kv_append(const fb_desc* d, const void* Kblk, const void* Vblk,
 /* Bytes of the static scratch array behind fb_prefix_partial_noalloc. */
 #define FB_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 
-/* fb_prefix_partial for callers that cannot allocate device memory (a graph
- * being captured, a fixed device-memory arena, a serving loop that must not
- * trigger allocator synchronisation).  No counterpart in the paper: it is a
- * deployment variant of the prefix pass.  Same arguments and results as
- * fb_prefix_partial without the workspace: the split-key partials go to a
- * FB_NOALLOC_SCRATCH_BYTES array inside the library's device image, present
- * on every GPU that loads the library until the process exits.
+/* fb_prefix_partial for callers that cannot allocate device memory: an
+ * embedding whose memory planner hands out one fixed device arena at start-up
+ * and forbids allocator calls afterwards, a plug-in host that gives its
+ * plug-ins no allocator, or a latency-critical serving loop that cannot afford
+ * the device-wide synchronisation a cudaMalloc or cudaFree may cause.  No
+ * counterpart in the paper: it is a deployment variant of the prefix pass.
+ * Same arguments and results as fb_prefix_partial without the workspace: the
+ * split-key partials go to a FB_NOALLOC_SCRATCH_BYTES array inside the
+ * library's device image, present on every GPU that loads the library until
+ * the process exits.
  *  - Allocates nothing and calls no allocating routine.
  *  - Returns FB_ERR_WORKSPACE (nothing launched) when this call's partials
  *    need more than FB_NOALLOC_SCRATCH_BYTES (fb_workspace_bytes() says how
@@ -243,6 +246,8 @@ fb_status fb_kv_append(const fb_desc* d, const void* Kblk, const void* Vblk,
  *    B = 1, S = 32, Hq = 32, 128K prefix).
  *  - The first call on each device looks up the array's device address with
  *    that device current; make that first call before any stream capture.
+ *    The lookup is repeated when the device's context has changed (after a
+ *    device reset), so the call after a reset is a first call again.
  *  - All calls share the one array, which keeps the last call's contents
  *    (nothing in it needs to start at zero).  Calls that can overlap on the
  *    GPU (other streams, other host threads) race on it: serialise them. */

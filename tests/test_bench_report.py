@@ -56,7 +56,17 @@ def test_report_line_has_contract_keys(capsys, kw):
         assert line["chunk_select_us"] == pytest.approx(20.0)
     if args.workload == "long_ctx" and not args.residual:
         # the recorded capture of the current kernel, or null when there is none
-        assert roof["traffic"] == bench.NCU_TRAFFIC.get("long_ctx")
+        assert roof["traffic"] == bench.recorded_traffic("long_ctx")
+
+
+def test_recorded_traffic_needs_the_captured_sources(monkeypatch):
+    # a capture is reported only while the kernel sources hash to the value
+    # recorded with it
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {"long_ctx": {"bytes": 123, "sources": bench.kernel_source_hash()}})
+    assert bench.recorded_traffic("long_ctx") == 123
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {"long_ctx": {"bytes": 123, "sources": "0" * 16}})
+    assert bench.recorded_traffic("long_ctx") is None
+    assert bench.recorded_traffic("video") is None
 
 
 def test_report_without_e2e_phase(capsys):
@@ -79,6 +89,9 @@ def test_reference_arm_line(capsys, monkeypatch):
     assert line["config"]["workload"].startswith("tiny_fp32")
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    # the step time is the measured sample's, not scaled up to the whole block
+    assert line["ms_per_step"] == pytest.approx(cb["sample_seconds_measured"] * 1e3)
+    assert line["value"] == pytest.approx(16 * cb["sample_fraction_of_block"] / cb["sample_seconds_measured"])
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
 

@@ -1,8 +1,10 @@
-"""fb_prefix_partial_noalloc: the prefix pass for callers that may not allocate
-device memory (graph capture, fixed arenas, serving loops that must not
-synchronise the device through the allocator).  Its split partials live in a
-static array of the library instead of a caller workspace; its results must
-match the regular entry point's, call after call.
+"""fb_prefix_partial_noalloc: the prefix pass for callers that may not
+allocate device memory (an embedding that owns one fixed device arena, a
+plug-in host that gives its plug-ins no allocator, a serving loop that cannot
+afford the device-wide synchronisation of cudaMalloc/cudaFree).  Its split
+partials live in a static array of the library instead of a caller
+workspace; its results must match the regular entry point's, call after
+call.
 
 Collected last on purpose (test_zz_*): if it fails, a run that stops at the
 first failure has already run every other test.  It builds its own inputs, so
@@ -39,6 +41,9 @@ def test_noalloc_matches_workspace_entry_point_two_calls_in_a_row():
         layer.check()
         gpu_cases.compare(f"noalloc O_pre, call {step}", O2.cpu().numpy(), layer.O_pre.cpu().numpy(), "bf16")
         gpu_cases.compare(f"noalloc LSE_pre, call {step}", L2.cpu().numpy(), layer.LSE_pre.cpu().numpy(), "bf16")
+        # the same kernels with the same split plan and merge order: the
+        # results are bit-identical, not just within tolerance
+        assert torch.equal(O2, layer.O_pre) and torch.equal(L2, layer.LSE_pre), f"call {step}: not bit-identical"
 
 
 def test_noalloc_rejects_partials_larger_than_the_scratch():
