@@ -505,7 +505,7 @@ def run_ours(args):
         unc = new_layer()
         if use_graph:
             g_unc = unc.capture_block(dev_in, outs, w.refresh, append_kv=(dev_in[-1][1], dev_in[-1][2]),
-                                      cached=False)
+                                      cached=False, advance=False)
             res["ms_unc"] = timed(lambda k: g_unc.replay(), unc)
             del g_unc
         else:

@@ -536,7 +536,20 @@ fb_status fb_chunk_means(const fb_desc* d, const void* Kc, int32_t c0, int32_t c
   const int64_t nch = (cache_rows(*d) + d->chunk_size - 1) / d->chunk_size;
   if (c0 < 0 || c1 < c0 || c1 > nch) return FB_ERR_INVALID_ARG;
   if (!aligned16(Kc) || !aligned16(Kmean)) return FB_ERR_ALIGNMENT;
-  return from_cuda(launch_chunk_means(*d, Kc, c0, c1, Kmean, dev_status,
+  return from_cuda(launch_chunk_means(*d, Kc, c0, c1, 0, Kmean, dev_status,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fb_status fb_chunk_means_tail(const fb_desc* d, const void* Kc, int32_t rows, float* Kmean,
+                              int32_t* dev_status, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if ((st = check_cache(d)) != FB_OK) return st;
+  if (!Kc || !Kmean || rows <= 0) return FB_ERR_INVALID_ARG;
+  if (d->chunk_size <= 0) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Kc) || !aligned16(Kmean)) return FB_ERR_ALIGNMENT;
+  const int64_t rows_cap = std::min<int64_t>(rows, cache_rows(*d));
+  return from_cuda(launch_chunk_means(*d, Kc, 0, 0, (int)std::max<int64_t>(rows_cap, 1), Kmean, dev_status,
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -64,14 +64,17 @@ template <>
 __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 // grid (chunks, Hkv, B), block D threads: thread d averages column d.
+// tail_rows == 0: chunk c0 + blockIdx.x of every sequence.  tail_rows > 0:
+// the chunks holding sequence b's last tail_rows valid rows, [L_b - tail_rows,
+// L_b), from its device length: chunk (max(L_b - tail_rows, 0) / chunk_size)
+// + blockIdx.x, skipped when it starts at or past L_b.
 template <typename T>
 __global__ void chunk_means_kernel(const CacheGeom g, const int32_t* lens, int chunk_size,
-                                   int c0, int nch_total, const T* __restrict__ K,
+                                   int c0, int tail_rows, int nch_total, const T* __restrict__ K,
                                    float* __restrict__ Kmean, int32_t* status) {
   // may start before the previous kernel in the stream has finished
   pdl_wait();
   pdl_launch_dependents();
-  const int c = c0 + blockIdx.x;
   const int kvh = blockIdx.y;
   const int b = blockIdx.z;
   const int d = threadIdx.x;
@@ -79,6 +82,11 @@ __global__ void chunk_means_kernel(const CacheGeom g, const int32_t* lens, int c
   if (L < 0 || L > g.cap) {
     if (d == 0) report(status, FB_ERR_BOUNDS);
     L = max(0, min(L, g.cap));
+  }
+  int c = c0 + blockIdx.x;
+  if (tail_rows > 0) {
+    c = max(L - tail_rows, 0) / chunk_size + blockIdx.x;
+    if (c * chunk_size >= L) return;  // (block-uniform)
   }
   const int lo = c * chunk_size;
   const int hi = min(lo + chunk_size, L);
@@ -355,19 +363,21 @@ __global__ void lens_advance_kernel(int32_t* lens, int B, int S, int cap) {
 
 }  // namespace
 
-cudaError_t launch_chunk_means(const fb_desc& d, const void* K, int c0, int c1, float* Kmean,
+cudaError_t launch_chunk_means(const fb_desc& d, const void* K, int c0, int c1, int tail_rows, float* Kmean,
                                int32_t* status, cudaStream_t stream) {
   const CacheGeom g = geom_of(d);
   const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
-  if (c1 <= c0) return cudaSuccess;
-  dim3 grid(c1 - c0, g.Hkv, g.B);
+  // tail mode: tail_rows rows straddle at most this many chunks
+  const int nblk = tail_rows > 0 ? (tail_rows + d.chunk_size - 1) / d.chunk_size + 1 : c1 - c0;
+  if (nblk <= 0) return cudaSuccess;
+  dim3 grid(nblk, g.Hkv, g.B);
   cudaError_t e;
   if (d.dtype == FB_BF16)
     e = launch_pdl(chunk_means_kernel<__nv_bfloat16>, grid, dim3(g.D), 0, stream, g, d.prefix_lens, d.chunk_size,
-                   c0, nch_total, static_cast<const __nv_bfloat16*>(K), Kmean, status);
+                   c0, tail_rows, nch_total, static_cast<const __nv_bfloat16*>(K), Kmean, status);
   else
     e = launch_pdl(chunk_means_kernel<float>, grid, dim3(g.D), 0, stream, g, d.prefix_lens, d.chunk_size, c0,
-                   nch_total, static_cast<const float*>(K), Kmean, status);
+                   tail_rows, nch_total, static_cast<const float*>(K), Kmean, status);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

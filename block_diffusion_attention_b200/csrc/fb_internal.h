@@ -161,7 +161,9 @@ cudaError_t launch_attn_simt(const AttnParams& p, const float* Q, const float* K
                              cudaStream_t stream);
 
 // Sparse prefix helpers and the cache append.
-cudaError_t launch_chunk_means(const fb_desc& d, const void* K, int chunk_begin, int chunk_end,
+// Chunks [chunk_begin, chunk_end) of every sequence, or (tail_rows > 0) the
+// chunks holding each sequence's last tail_rows valid rows by its device length.
+cudaError_t launch_chunk_means(const fb_desc& d, const void* K, int chunk_begin, int chunk_end, int tail_rows,
                                float* Kmean, int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* Kmean,
                                  int32_t* idx, int32_t* dev_status, cudaStream_t stream);

@@ -72,6 +72,7 @@ def load() -> ctypes.CDLL:
             "fb_block_step": (I32, [D, P, P, P, P, P, P, P, P, P]),
             "fb_full_reference_gpu": (I32, [D, P, P, P, P, P, P, P, P, SZ, P, P]),
             "fb_chunk_means": (I32, [D, P, I32, I32, P, P, P]),
+            "fb_chunk_means_tail": (I32, [D, P, I32, P, P, P]),
             "fb_select_chunks": (I32, [D, P, P, P, P, P]),
             "fb_kv_append": (I32, [D, P, P, P, P, P, P, P]),
             "fb_complement_chunks": (I32, [D, P, P, I32, P, P]),
@@ -171,6 +172,11 @@ def fb_full_reference_gpu(d, Q, Kcache, Vcache, Kblk, Vblk, O, LSE_out, workspac
 def fb_chunk_means(d, Kcache, chunk_begin, chunk_end, Kmean, dev_status, stream=None):
     _ok("fb_chunk_means", load().fb_chunk_means(
         ctypes.byref(d), _p(Kcache), int(chunk_begin), int(chunk_end), _p(Kmean), _p(dev_status), _s(stream)))
+
+
+def fb_chunk_means_tail(d, Kcache, rows, Kmean, dev_status, stream=None):
+    _ok("fb_chunk_means_tail", load().fb_chunk_means_tail(
+        ctypes.byref(d), _p(Kcache), int(rows), _p(Kmean), _p(dev_status), _s(stream)))
 
 
 def fb_select_chunks(d, Q, Kmean, chunk_idx, dev_status, stream=None):

@@ -51,7 +51,6 @@ class CachedBlockAttention:
         self.K = torch.zeros(cache_shape, dtype=self.tdtype, device=dev)
         self.V = torch.zeros(cache_shape, dtype=self.tdtype, device=dev)
         self.lens = torch.zeros(batch, dtype=torch.int32, device=dev)
-        self.lens_host = [0] * batch
         self.desc = fbl.make_desc(
             batch, num_q_heads, num_kv_heads, head_dim, block_len,
             dtype=fbl.FB_BF16 if dtype == "bf16" else fbl.FB_FP32, softmax_scale=softmax_scale,
@@ -120,7 +119,6 @@ class CachedBlockAttention:
                     self.K[pg, :hi - lo].copy_(K[b, lo:hi])
                     self.V[pg, :hi - lo].copy_(V[b, lo:hi])
         self.lens.copy_(torch.tensor(lens, dtype=torch.int32))
-        self.lens_host = lens
         if self.topk > 0:
             self.update_chunk_means(0, -(-self.capacity // self.chunk_size))
 
@@ -206,18 +204,15 @@ class CachedBlockAttention:
     def append(self, Kblk, Vblk, advance: bool = True) -> None:
         """Block end: write the finalized block's K/V after the prefix and grow it.
 
-        ``advance=False`` writes the rows but keeps the prefix length (a
-        benchmark holds its workload fixed this way)."""
+        The prefix lengths live on the device: the append reads them, writes
+        the rows and advances them, and (sparse prefix) the means of the
+        chunks it touched are recomputed from the advanced device lengths, so
+        no host round trip is needed and a recorded block replays correctly
+        block after block.  ``advance=False`` writes the rows but keeps the
+        prefix length (a benchmark holds its workload fixed this way)."""
         fbl.fb_kv_append(self.desc, Kblk, Vblk, self.K, self.V, self.lens if advance else None, self.status)
-        if not advance:
-            return
-        old = self.lens_host
-        self.lens_host = [min(L + self.S, self.capacity) if L + self.S <= self.capacity else L for L in old]
-        if self.topk > 0:
-            c0 = min(old) // self.chunk_size
-            c1 = -(-max(self.lens_host) // self.chunk_size)
-            if c1 > c0:
-                self.update_chunk_means(c0, c1)
+        if advance and self.topk > 0:
+            fbl.fb_chunk_means_tail(self.desc, self.K, self.S, self.Kmean, self.status)
 
     # ------------------------------------------------------------ graphs
     def run_block(self, steps, outs, refresh_steps, append_kv=None, advance=True, cached=True):
@@ -234,16 +229,20 @@ class CachedBlockAttention:
             self.append(append_kv[0], append_kv[1], advance=advance)
 
     def capture_block(self, steps, outs, refresh_steps, append_kv=None, cached=True, prologue=None,
-                      epilogue=None):
+                      epilogue=None, advance=True):
         """Record one block of calls (see ``run_block``) into a CUDA graph.
 
         The library's calls are capturable: they allocate nothing, never
         synchronise, and pass their TMA descriptors by value.  The block runs
-        once eagerly first, so one-time kernel attribute settings happen outside
-        the capture.  The append is recorded without advancing the prefix
-        length (a replayed graph cannot update the host-side bookkeeping).
-        ``prologue``/``epilogue`` (callables) are recorded before/after each
-        step, e.g. host<->device copies.  Returns the ``torch.cuda.CUDAGraph``.
+        once eagerly first, so one-time kernel attribute settings happen
+        outside the capture (that run is a real block: with ``advance`` it
+        appends, and the prefix grows by one block).  The append is recorded
+        with the device-side length update (``advance=True``): each replay
+        appends after the current prefix and grows it, and the graph can be
+        replayed for consecutive blocks once the next block's inputs are
+        copied into the tensors it was recorded with.  ``prologue``/
+        ``epilogue`` (callables) are recorded before/after each step, e.g.
+        host<->device copies.  Returns the ``torch.cuda.CUDAGraph``.
         """
         def body():
             for s, (Q, Kb, Vb) in enumerate(steps):
@@ -256,7 +255,7 @@ class CachedBlockAttention:
                 if epilogue is not None:
                     epilogue(s)
             if append_kv is not None:
-                self.append(append_kv[0], append_kv[1], advance=False)
+                self.append(append_kv[0], append_kv[1], advance=advance)
 
         body()
         torch.cuda.synchronize()

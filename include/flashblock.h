@@ -143,6 +143,17 @@ fb_status fb_chunk_means(const fb_desc* d, const void* Kcache, int32_t chunk_beg
                          int32_t chunk_end, float* Kmean, int32_t* dev_status,
                          fb_stream_t stream);
 
+/* Sparse prefix, step 1 after an append (Technical Summary §1: each finished
+ * block joins the cache that later blocks attend to): the same means for the
+ * chunks holding each sequence's last `rows` valid rows, j in
+ * [max(L_b - rows, 0), L_b), with L_b = prefix_lens[b] read on the device.
+ * Called with rows = S after fb_kv_append has advanced prefix_lens, it
+ * refreshes exactly the chunks the append touched, with no host-side length,
+ * so a block recorded once (in a CUDA graph, say) keeps the means current as
+ * the sequence grows.  rows > 0.  Kmean as for fb_chunk_means. */
+fb_status fb_chunk_means_tail(const fb_desc* d, const void* Kcache, int32_t rows, float* Kmean,
+                              int32_t* dev_status, fb_stream_t stream);
+
 /* Sparse prefix, step 2: per (b, kv head) score every valid chunk c by
  * qbar . Kmean[c], qbar the mean of Q over the S block tokens and the G query
  * heads of the group, and keep the top d->topk (ties to the lower index).

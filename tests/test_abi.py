@@ -70,6 +70,10 @@ def test_host_validation_codes(lib):
     assert blk == 1
     assert lib.fb_chunk_means(ctypes.byref(_desc(chunk_size=256)), FAKE, 0, 999, FAKE, None, None) == 1
     assert lib.fb_select_chunks(ctypes.byref(_desc(chunk_size=256, topk=0)), FAKE, FAKE, FAKE, None, None) == 1
+    tail = lib.fb_chunk_means_tail
+    assert tail(ctypes.byref(_desc(chunk_size=256)), FAKE, 0, FAKE, None, None) == 1     # rows > 0
+    assert tail(ctypes.byref(_desc(chunk_size=0)), FAKE, 32, FAKE, None, None) == 1
+    assert tail(ctypes.byref(_desc(chunk_size=256)), FAKE, 32, FAKE + 4, None, None) == 3
     assert lib.fb_kv_append(ctypes.byref(_desc(kv_capacity=0)), FAKE, FAKE, FAKE, FAKE, None, None, None) == 1
 
 

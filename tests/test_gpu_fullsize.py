@@ -5,8 +5,11 @@ The oracle cannot recompute every output of the large workloads in seconds,
 so it computes sampled query rows one by one from the definition (the LM
 workload is small enough to compare in full).  Samples cover every KV head,
 the first and last tokens, and -- for the video workload -- the ragged last
-query tile.  Tolerances are the bf16 ones of the method (max |diff| <= 2e-2,
-relative Frobenius error <= 1e-2)."""
+query tile.  Each workload is checked at a refresh step (the cached pair and
+the step's output), at reuse steps (the refresh step's pair merged with the
+step's own in-block partial) and on the uncached output.  Tolerances are the
+bf16 ones of the method (max |diff| <= 2e-2, relative Frobenius error <=
+1e-2)."""
 import numpy as np
 import pytest
 import gpu_cases
@@ -39,20 +42,31 @@ def _prefix_keys(Kc64, Vc64, lens, b, kvh, idx=None, chunk=256):
     return Kc64[b, pos, kvh, :], Vc64[b, pos, kvh, :]
 
 
-def _check_rows(w, rows, layer, Q64, Kb64, Vb64, Kc64, Vc64, lens, O_step, O_full, idx=None, pre_only=False):
+def _check_rows(w, rows, layer, Q64, Kb64, Vb64, Kc64, Vc64, lens, O_step, O_full, idx=None, pre_only=False,
+                Q_pre64=None, tag=""):
+    """Sampled rows against the oracle, each recomputed from the definition.
+
+    Q_pre64: the queries of the refresh step whose cached pair (O_pre,
+    LSE_pre) the step reuses (default: this step's Q64, i.e. a refresh step);
+    the cached pair is checked only then.  O_step is the cached step's output
+    (the refresh-step pair merged with this step's in-block partial), O_full
+    the uncached output over [dense prefix ; block] (or None)."""
+    refresh = Q_pre64 is None
+    Q_pre64 = Q64 if refresh else Q_pre64
     got_pre, ref_pre, got_lpre, ref_lpre = [], [], [], []
     got_o, ref_o, got_f, ref_f = [], [], [], []
     O_pre = layer.O_pre.cpu().numpy()
     L_pre = layer.LSE_pre.cpu().numpy()
     for (b, t, h) in rows:
         kvh = h // w.group
-        q = Q64[b, t, h][None, :]
         kp, vp = _prefix_keys(Kc64, Vc64, lens, b, kvh, idx, w.chunk_size)
-        op, lp = ora.attention_partial(q, kp, vp, w.softmax_scale)
-        got_pre.append(O_pre[b, t, h]); ref_pre.append(op[0])
-        got_lpre.append(L_pre[b, h, t]); ref_lpre.append(lp[0])
+        op, lp = ora.attention_partial(Q_pre64[b, t, h][None, :], kp, vp, w.softmax_scale)
+        if refresh:
+            got_pre.append(O_pre[b, t, h]); ref_pre.append(op[0])
+            got_lpre.append(L_pre[b, h, t]); ref_lpre.append(lp[0])
         if pre_only:
             continue
+        q = Q64[b, t, h][None, :]
         oi, li = ora.attention_partial(q, Kb64[b, :, kvh], Vb64[b, :, kvh], w.softmax_scale)
         om, _ = ora.merge_partials(op, lp, oi, li)
         got_o.append(O_step[b, t, h]); ref_o.append(om[0])
@@ -61,12 +75,14 @@ def _check_rows(w, rows, layer, Q64, Kb64, Vb64, Kc64, Vc64, lens, O_step, O_ful
                                           np.concatenate([Vc64[b, :int(lens[b]), kvh], Vb64[b, :, kvh]]),
                                           w.softmax_scale)
             got_f.append(O_full[b, t, h]); ref_f.append(of[0])
-    gpu_cases.compare(f"{w.name} O_pre rows", np.array(got_pre), np.array(ref_pre), "bf16")
-    gpu_cases.compare(f"{w.name} LSE_pre rows", np.array(got_lpre), np.array(ref_lpre), "bf16")
+    name = f"{w.name}{tag}"
+    if got_pre:
+        gpu_cases.compare(f"{name} O_pre rows", np.array(got_pre), np.array(ref_pre), "bf16")
+        gpu_cases.compare(f"{name} LSE_pre rows", np.array(got_lpre), np.array(ref_lpre), "bf16")
     if got_o:
-        gpu_cases.compare(f"{w.name} O rows", np.array(got_o), np.array(ref_o), "bf16")
+        gpu_cases.compare(f"{name} O rows", np.array(got_o), np.array(ref_o), "bf16")
     if got_f:
-        gpu_cases.compare(f"{w.name} O_full rows", np.array(got_f), np.array(ref_f), "bf16")
+        gpu_cases.compare(f"{name} O_full rows", np.array(got_f), np.array(ref_f), "bf16")
 
 
 def _setup(w):
@@ -122,46 +138,80 @@ def test_lm_gqa_full_size_every_output():
 
 
 def test_video_full_size_sampled():
+    # refresh at step 0 (cached pair, step output), then the reuse step 2: the
+    # step-0 pair merged with step 2's in-block partial, and the uncached
+    # output of step 2, on rows that include the ragged last query tile
     w = synth.WORKLOADS["video"]
     layer, Kc64, Vc64, lens = _setup(w)
     base = synth.block_base(w, 0)
-    Qt, Q64, Kbt, Kb64, Vbt, Vb64 = _step(w, layer, 0, base)
-    layer.refresh(Qt)
-    O = layer.step(Qt, Kbt, Vbt).float().cpu().numpy()
-    layer.check()
     rows = _sample_rows(w, 40, 2)
     # rows of the ragged last query tile (4680 = 36 * 128 + 72)
     rows += [(0, 4679, 3), (0, 4608, 17), (0, 4650, 39)]
-    _check_rows(w, rows, layer, Q64, Kb64, Vb64, Kc64, Vc64, lens, O, None)
+    Q0 = None
+    for s in range(3):
+        Qt, Q64, Kbt, Kb64, Vbt, Vb64 = _step(w, layer, s, base)
+        O = layer.cached_step(s, Qt, Kbt, Vbt, w.refresh).float().cpu().numpy()
+        Of = layer.full(Qt, Kbt, Vbt).float().cpu().numpy() if s == 2 else None
+        layer.check()
+        if s == 0:
+            Q0 = Q64
+            _check_rows(w, rows, layer, Q64, Kb64, Vb64, Kc64, Vc64, lens, O, None, tag=" step 0")
+        elif s == 2:
+            _check_rows(w, rows, layer, Q64, Kb64, Vb64, Kc64, Vc64, lens, O, Of, Q_pre64=Q0, tag=" step 2")
 
 
-def test_batched_sparse_full_size():
-    w = synth.WORKLOADS["batched_sparse"]
-    layer, Kc64, Vc64, lens = _setup(w)
-    base = synth.block_base(w, 0)
-    Qt, Q64, Kbt, Kb64, Vbt, Vb64 = _step(w, layer, 0, base)
-    layer.refresh(Qt)
-    O = layer.step(Qt, Kbt, Vbt).float().cpu().numpy()
-    layer.check()
+def _validated_selection(w, layer, Q64, Kc64, lens, step):
+    """The GPU's chunk lists, checked against the oracle's float64 scores.
+
+    Where the oracle's 16th and 17th scores of a unit are more than eps
+    apart the selection is unique and the lists must be equal; otherwise
+    (a near-tie, where fp32 and fp64 rounding may order the tied chunks
+    differently) every chunk the GPU chose must score within eps of the
+    16th-best, so the GPU's list is one of the correct top-k sets.  Returns
+    that list: the attention is then checked over the key set it names."""
     Km, valid = ora.chunk_means(Kc64, lens, w.chunk_size)
     idx = ora.select_chunks(Q64, Km, valid, w.topk)
     gidx = layer.chunk_idx.cpu().numpy()
     sc = ora.chunk_scores(Q64, Km, valid)
     srt = -np.sort(-sc, axis=2)
-    # fp32 (kernel) and fp64 (oracle) scores can order a near-tie differently;
     # eps is far above the fp32 rounding of these scores
     eps = 1e-5 * np.nanmax(np.abs(np.where(np.isfinite(srt), srt, 0.0)))
-    same = np.zeros((w.batch, w.num_kv_heads), dtype=bool)
+    ties = 0
     for b in range(w.batch):
         for kvh in range(w.num_kv_heads):
             g = [int(c) for c in gidx[b, kvh] if c >= 0]
             o = [int(c) for c in idx[b, kvh] if c >= 0]
-            assert len(g) == len(o) == len(set(g)), f"selection size b{b} kvh{kvh}"
+            assert len(g) == len(o) == len(set(g)), f"step {step}: selection size b{b} kvh{kvh}"
+            assert g == sorted(g), f"step {step}: list not ascending b{b} kvh{kvh}"
             kth = srt[b, kvh, w.topk - 1]
-            assert all(sc[b, kvh, c] >= kth - eps for c in g), f"invalid top-k b{b} kvh{kvh}"
-            same[b, kvh] = (g == o)
+            assert all(sc[b, kvh, c] >= kth - eps for c in g), f"step {step}: invalid top-k b{b} kvh{kvh}"
             if srt[b, kvh, w.topk - 1] - srt[b, kvh, w.topk] > eps:
-                assert same[b, kvh], f"selection differs beyond near-ties at b{b} kvh{kvh}"
-    assert same.mean() > 0.9
-    rows = [r for r in _sample_rows(w, 64, 3) if same[r[0], r[2] // w.group]]
-    _check_rows(w, rows, layer, Q64, Kb64, Vb64, Kc64, Vc64, lens, O, None, idx=idx)
+                assert g == o, f"step {step}: selection differs beyond near-ties at b{b} kvh{kvh}"
+            ties += g != o
+    assert ties <= 0.1 * w.batch * w.num_kv_heads, f"step {step}: {ties} near-tie units"
+    return gidx
+
+
+def test_batched_sparse_full_size():
+    # the whole 8-step block in the bench's launch configuration: refreshes at
+    # steps 0 and 4 (selection, cached pair, step output), reuse steps 1 and 5
+    # (the refresh pair merged with the step's in-block partial), and the
+    # uncached output of step 5 over the dense prefix; every sampled row is
+    # checked, near-tie units over their validated selection
+    w = synth.WORKLOADS["batched_sparse"]
+    layer, Kc64, Vc64, lens = _setup(w)
+    base = synth.block_base(w, 0)
+    rows = _sample_rows(w, 64, 3)
+    Q_ref, sel = None, None
+    for s in range(w.steps):
+        Qt, Q64, Kbt, Kb64, Vbt, Vb64 = _step(w, layer, s, base)
+        O = layer.cached_step(s, Qt, Kbt, Vbt, w.refresh).float().cpu().numpy()
+        Of = layer.full(Qt, Kbt, Vbt).float().cpu().numpy() if s == 5 else None
+        layer.check()
+        if s in w.refresh:
+            Q_ref = Q64
+            sel = _validated_selection(w, layer, Q64, Kc64, lens, s)
+            _check_rows(w, rows, layer, Q64, Kb64, Vb64, Kc64, Vc64, lens, O, None, idx=sel, tag=f" step {s}")
+        elif s in (1, 5):
+            _check_rows(w, rows, layer, Q64, Kb64, Vb64, Kc64, Vc64, lens, O, Of, idx=sel, Q_pre64=Q_ref,
+                        tag=f" step {s}")

@@ -167,6 +167,74 @@ def test_block_graph_replay_matches_eager():
         assert torch.equal(outs[s], eager[s]), f"step {s}"
 
 
+@pytest.mark.parametrize("name", ["lm_gqa", "batched_sparse"])
+def test_block_graph_advances_the_sequence(name):
+    # one block recorded once and replayed for consecutive blocks: each replay
+    # appends the finalized block after the current prefix, advances the
+    # device lengths and (sparse prefix) recomputes the touched chunk means,
+    # with no host bookkeeping; every step's output, the lengths and the
+    # chunk lists follow the oracle's run on its own appended cache
+    if name == "lm_gqa":
+        w = W["lm_gqa"].scaled(prefix_len=700, blocks=4, steps=3)
+    else:
+        w = W["batched_sparse"].scaled(batch=3, num_q_heads=8, num_kv_heads=2, prefix_len=1500,
+                                       prefix_min=600, topk=3, steps=5, blocks=3)
+    K, V, lens = synth.prefix_kv(w)
+    Kt, K64 = gpu_cases.tensors(w, K)
+    Vt, V64 = gpu_cases.tensors(w, V)
+    layer = gpu_cases.make_layer(w)
+    layer.load_prefix(Kt, Vt, lens)
+
+    def block_inputs(blk):
+        base = synth.block_base(w, blk)
+        return [tuple(gpu_cases.tensors(w, x) for x in synth.step_inputs(w, blk, s, base))
+                for s in range(w.steps)]
+
+    inp = block_inputs(0)
+    steps = [tuple(x[0] for x in t) for t in inp]  # the tensors the graph reads
+    outs = [torch.empty_like(steps[0][0]) for _ in range(w.steps)]
+    # block 0 runs eagerly inside capture_block, before the recording
+    g = layer.capture_block(steps, outs, w.refresh, append_kv=(steps[-1][1], steps[-1][2]))
+    Kc, Vc, lens_o = K64.copy(), V64.copy(), lens.astype(np.int64).copy()
+    S = w.block_len
+    for blk in range(w.blocks):
+        if blk > 0:
+            inp = block_inputs(blk)
+            for dst, src in zip(steps, inp):
+                for d_t, s_t in zip(dst, src):
+                    d_t.copy_(s_t[0])
+            for o in outs:
+                o.zero_()
+            g.replay()
+        layer.check()
+        got = [o.float().cpu().numpy() for o in outs]
+        pre, idx = None, None
+        for s in range(w.steps):
+            Q64, Kb64, Vb64 = (x[1] for x in inp[s])
+            if s in w.refresh or pre is None:
+                if w.topk:
+                    Km, valid = ora.chunk_means(Kc, lens_o, w.chunk_size)
+                    idx = ora.select_chunks(Q64, Km, valid, w.topk)
+                pre = ora.prefix_partial(Q64, Kc, Vc, lens_o, w.softmax_scale, idx, w.chunk_size)
+            o_ref, _ = ora.block_step(Q64, Kb64, Vb64, pre[0], pre[1], w.softmax_scale)
+            gpu_cases.compare(f"graph block {blk} step {s}", got[s], o_ref, w.dtype)
+        if w.topk:
+            assert np.array_equal(layer.chunk_idx.cpu().numpy(), idx), f"block {blk}: chunk lists"
+        # the oracle's own append of the block's last step
+        Kb64, Vb64 = inp[-1][1][1], inp[-1][2][1]
+        for b in range(w.batch):
+            L = int(lens_o[b])
+            if L + S <= Kc.shape[1]:
+                Kc[b, L:L + S] = Kb64[b]
+                Vc[b, L:L + S] = Vb64[b]
+                lens_o[b] = L + S
+        assert np.array_equal(layer.lens.cpu().numpy(), lens_o), f"block {blk}: prefix lengths"
+    if w.topk:
+        # the means kept current by the replays equal the means of the grown cache
+        Km, _ = ora.chunk_means(Kc, lens_o, w.chunk_size)
+        gpu_cases.compare("chunk means after the replays", layer.Kmean.cpu().numpy(), Km, "fp32")
+
+
 def test_residual_sparse_reuse():
     # residual reuse: cached unselected-chunk partial + fresh selected chunks + block
     w = W["batched_sparse"].scaled(batch=3, num_q_heads=8, num_kv_heads=2, prefix_len=1500,
