@@ -154,14 +154,29 @@ AttnParams base_params(const fb_desc& d) {
   return p;
 }
 
+// Query tiles (128 packed rows) of one (b, kv head) unit.
+int row_tiles(const fb_desc& d) {
+  const int G = d.num_q_heads / d.num_kv_heads;
+  return (d.block_len * G + TC_BM - 1) / TC_BM;
+}
+
+// Units of two or more query tiles run on the two-tile kernel: one CTA per
+// pair of tiles, each K/V tile loaded once for both.
+bool use_pairs(const fb_desc& d) { return d.dtype == FB_BF16 && row_tiles(d) >= 2; }
+
+// CTAs of one key split: (b, kv head, query tile) or (b, kv head, tile pair).
+long long cta_units(const fb_desc& d) {
+  const int rt = row_tiles(d);
+  return (long long)d.batch * d.num_kv_heads * (use_pairs(d) ? (rt + 1) / 2 : rt);
+}
+
 // Key-range splits of the prefix pass.  Cost model in key-tile times: every
 // wave of CTAs costs its longest split plus a fixed per-CTA overhead (set-up,
 // pipeline fill, epilogue ~ 3 tiles), and splitting adds a combine pass
 // (~ 2 tiles).  Splits keep at least 4 tiles each.
 int choose_splits(const fb_desc& d, long long est_tiles) {
   if (d.dtype != FB_BF16) return 1;
-  const int G = d.num_q_heads / d.num_kv_heads;
-  const long long units = (long long)d.batch * d.num_kv_heads * ((d.block_len * G + TC_BM - 1) / TC_BM);
+  const long long units = cta_units(d);
   long long max_ns = est_tiles / 4;
   if (max_ns < 1) max_ns = 1;
   if (max_ns > TC_MAX_SPLITS) max_ns = TC_MAX_SPLITS;
@@ -282,9 +297,9 @@ size_t fb_workspace_bytes(const fb_desc* d) {
   size_t need = split_bytes(*d, ns_pre);
   need = std::max(need, split_bytes(*d, ns_full));
   need = std::max(need, threshold_ws_bytes(*d));
-  if (d->dtype == FB_BF16) {
+  if (d->dtype == FB_BF16 && !use_pairs(*d)) {
     // the masked prefix pass's active-unit slots
-    const long long grid = (long long)d->batch * d->num_kv_heads * ((d->block_len * (d->num_q_heads / d->num_kv_heads) + TC_BM - 1) / TC_BM) * ns_pre;
+    const long long grid = cta_units(*d) * ns_pre;
     if (use_active_split(*d, grid)) need = std::max(need, active_split_bytes(grid));
   }
   return need;
@@ -318,8 +333,9 @@ fb_status prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const 
                                       static_cast<const float*>(Vc), nullptr, nullptr, s));
   }
   const int ns = choose_splits(*d, prefix_tiles_estimate(*d));
-  const long long grid = (long long)d->batch * d->num_kv_heads * p.n_rt * ns;
-  const bool active = unit_mask != nullptr && use_active_split(*d, grid);
+  const bool pairs = use_pairs(*d);
+  const long long grid = cta_units(*d) * ns;
+  const bool active = unit_mask != nullptr && !pairs && use_active_split(*d, grid);
   const size_t need = active ? active_split_bytes(grid) : split_bytes(*d, ns);
   if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return FB_ERR_WORKSPACE;
   Maps m;
@@ -364,7 +380,13 @@ fb_status prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const 
   p.out_lse = part_l;
   CUtensorMap tm_out;
   if (!pre_map(&tm_out, *d, part_o, d->batch * ns)) return FB_ERR_LAUNCH;
-  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kp, m.vp, m.q, tm_out, (int)grid, s);
+  cudaError_t e;
+  if (pairs) {
+    p.kv_stream_once = (p.n_rt <= 2);  // one tile pair per unit: each K/V byte is read once
+    e = launch_attn_tc2(p, m.q, m.kp, m.vp, m.kp, m.vp, tm_out, (int)grid, s);
+  } else {
+    e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kp, m.vp, m.q, tm_out, (int)grid, s);
+  }
   if (e != cudaSuccess || ns == 1) return from_cuda(e);
   CombineParams c;
   std::memset(&c, 0, sizeof(c));
@@ -457,7 +479,11 @@ fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const v
   if (!q_map(&m.q, *d, Q) || !block_map(&m.kb, *d, Kb) || !block_map(&m.vb, *d, Vb) ||
       !pre_map(&tm_pre, *d, O_pre) || !q_map(&tm_out, *d, O))
     return FB_ERR_LAUNCH;
-  const long long grid = (long long)d->batch * d->num_kv_heads * p.n_rt;
+  const long long grid = cta_units(*d);
+  if (use_pairs(*d)) {
+    p.kv_stream_once = (p.n_rt <= 2);
+    return from_cuda(launch_attn_tc2(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_out, (int)grid, s));
+  }
   return from_cuda(launch_attn_tc(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_pre, tm_out, (int)grid, s));
 }
 
@@ -492,13 +518,16 @@ fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc,
   if (!q_map(&m.q, dense, Q) || !cache_map(&m.kp, dense, Kc) || !cache_map(&m.vp, dense, Vc) ||
       !block_map(&m.kb, dense, Kb) || !block_map(&m.vb, dense, Vb))
     return FB_ERR_LAUNCH;
-  const long long units = (long long)d->batch * d->num_kv_heads * p.n_rt;
+  const long long units = cta_units(dense);
+  const bool pairs = use_pairs(dense);
+  if (pairs) p.kv_stream_once = (p.n_rt <= 2);
   if (ns == 1) {
     p.epi = EPI_NORM;
     p.out_o = O;
     p.out_lse = LSE_out;
     CUtensorMap tm_out;
     if (!q_map(&tm_out, dense, O)) return FB_ERR_LAUNCH;
+    if (pairs) return from_cuda(launch_attn_tc2(p, m.q, m.kp, m.vp, m.kb, m.vb, tm_out, (int)units, s));
     return from_cuda(launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, tm_out, (int)units, s));
   }
   p.epi = EPI_PARTIAL;
@@ -509,7 +538,8 @@ fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc,
   p.out_lse = part_l;
   CUtensorMap tm_out;
   if (!pre_map(&tm_out, dense, part_o, d->batch * ns)) return FB_ERR_LAUNCH;
-  cudaError_t e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, tm_out, (int)(units * ns), s);
+  cudaError_t e = pairs ? launch_attn_tc2(p, m.q, m.kp, m.vp, m.kb, m.vb, tm_out, (int)(units * ns), s)
+                        : launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, tm_out, (int)(units * ns), s);
   if (e != cudaSuccess) return from_cuda(e);
   CombineParams c;
   std::memset(&c, 0, sizeof(c));

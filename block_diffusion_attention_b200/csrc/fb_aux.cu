@@ -11,11 +11,14 @@
 // Append (Technical Summary §1: block diffusion keeps a KV cache of the blocks
 // already generated, each block causal with respect to the earlier ones):
 // a finalized block's K/V joins the prefix.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
 #include "fb_internal.h"
 #include "fb_ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace fb {
 
@@ -103,10 +106,28 @@ __global__ void chunk_means_kernel(const CacheGeom g, const int32_t* lens, int c
   Kmean[(((size_t)b * g.Hkv + kvh) * nch_total + c) * g.D + d] = mean;
 }
 
-// grid (Hkv, B), block SEL_THREADS.  Dynamic shared memory:
-// SEL_PART_FLOATS + D floats for the query mean, nch scores, nch flags.
-constexpr int SEL_WARPS = 8, SEL_THREADS = SEL_WARPS * 32;
+// One 8-CTA thread-block cluster per (b, kv head); grid (SEL_CLUSTER, Hkv, B).
+// CTA k of the cluster
+//   1. sums its slice of the unit's S x G query rows per column (the
+//      partials are added in rank order by every CTA: one qbar for all),
+//   2. scores its slice of the chunks (its Kmean rows are loaded before the
+//      first cluster barrier, while the query loads are in flight),
+//   3. ranks its chunks against every score (a chunk's rank = chunks with a
+//      higher score, or an equal score and a lower index); the chunk of rank
+//      topk - 1 is the k-th best key,
+//   4. knowing that key, marks every chunk at or above it and writes its own
+//      selected chunks at their ascending-order positions (a block scan).
+// Dynamic shared memory: see sel_smem_bytes.
+constexpr int SEL_CLUSTER = 8;
+constexpr int SEL_THREADS = 256;
 constexpr int SEL_PART_FLOATS = SEL_THREADS * 8;  // row-group sums of the query mean (16-bit inputs)
+
+size_t sel_smem_bytes(int D, int nch_total) {
+  // row-group sums, the CTA's column partial, qbar, the k-th key, every
+  // score, one flag (then scan offset) per chunk, warp totals
+  return (size_t)(SEL_PART_FLOATS + 2 * D + 4 + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int) +
+         (SEL_THREADS / 32 + 1) * sizeof(int);
+}
 
 // Adds the eight bf16 or four f32 values of a 16-byte vector to acc.
 template <typename T>
@@ -129,8 +150,13 @@ __device__ __forceinline__ void add_vec16<float>(const uint4& v, float* acc) {
   acc[3] += __uint_as_float(v.w);
 }
 
+// Does chunk a (score sa) rank above chunk b (score sb)?
+__device__ __forceinline__ bool ranks_above(float sa, int a, float sb, int b) {
+  return sa > sb || (sa == sb && a < b);
+}
+
 template <typename T>
-__global__ void __launch_bounds__(SEL_THREADS)
+__global__ void __cluster_dims__(SEL_CLUSTER, 1, 1) __launch_bounds__(SEL_THREADS)
     select_chunks_kernel(const CacheGeom g, const int32_t* lens, int chunk_size, int nch_total, int S, int Hq,
                          int topk, const T* __restrict__ Q, const float* __restrict__ Kmean,
                          int32_t* __restrict__ idx, int32_t* status) {
@@ -138,102 +164,173 @@ __global__ void __launch_bounds__(SEL_THREADS)
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ float sm[];
-  const int kvh = blockIdx.x;
-  const int b = blockIdx.y;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
   const int G = Hq / g.Hkv;
-  // query mean over the S block tokens and the G heads of the group: the
-  // unit's S x G rows of D values are read as 16-byte vectors, thread i taking
-  // vector i % vpr of rows i / vpr, i / vpr + rpi, ...; the rpi row sums of
-  // each column are then added in a fixed order
-  constexpr int VEC = 16 / sizeof(T);
-  const int vpr = g.D / VEC;                // vectors per row
-  const int rpi = SEL_THREADS / vpr;        // rows per iteration
-  float* part = sm;                         // [rpi][D] row-group sums
-  float* qbar = sm + SEL_PART_FLOATS;       // [D]
-  float* score = qbar + g.D;                // [nch_total]
-  int* sel = reinterpret_cast<int*>(score + nch_total);
+  const int D = g.D;
+  float* rowsum = sm;                       // [rpi][D] row-group sums
+  float* part = rowsum + SEL_PART_FLOATS;   // [D] this CTA's column sums
+  float* qbar = part + D;                   // [D]
+  float* kth = qbar + D;                    // {score, index as float bits, found}
+  float* score = kth + 4;                   // [nch_total] every chunk's score
+  int* flag = reinterpret_cast<int*>(score + nch_total);  // [nch_total]
+  int* wsum = flag + nch_total;             // [warps + 1]
   int L = lens[b];
   if (L < 0 || L > g.cap) {
-    if (threadIdx.x == 0) report(status, FB_ERR_BOUNDS);
+    if (threadIdx.x == 0 && rank == 0) report(status, FB_ERR_BOUNDS);
     L = max(0, min(L, g.cap));
   }
   const int nch = (L + chunk_size - 1) / chunk_size;
-  const int rows = S * G;
+  const int c_lo = (int)((long long)nch * rank / SEL_CLUSTER);
+  const int c_hi = (int)((long long)nch * (rank + 1) / SEL_CLUSTER);
+  // this CTA's Kmean rows (first pass: 64 chunks, 4 lanes per chunk, each a
+  // quarter of D), loaded now so they are in flight with the query loads
+  const float* km = Kmean + ((size_t)b * g.Hkv + kvh) * nch_total * D;
+  const int q4 = threadIdx.x & 3, dq = D / 4;
+  constexpr int CPP = SEL_THREADS / 4;  // chunks per pass
+  float4 kr[8];
   {
-    const int vi = threadIdx.x % vpr, r0 = threadIdx.x / vpr;
-    if (r0 < rpi) {
+    const int c = c_lo + (threadIdx.x >> 2);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      kr[i] = (c < c_hi && i < dq / 4) ? reinterpret_cast<const float4*>(km + (size_t)c * D + q4 * dq)[i]
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // 1. column sums of this CTA's rows of the unit (16-byte vectors: thread i
+  // takes vector i % vpr of rows r0 + i / vpr, + rpi, ...; the rpi row-group
+  // sums of each column are then added in a fixed order)
+  constexpr int VEC = 16 / sizeof(T);
+  const int vpr = D / VEC;                // vectors per row
+  const int rpi = SEL_THREADS / vpr;      // rows per iteration
+  const int rows = S * G;
+  const int r_lo = (int)((long long)rows * rank / SEL_CLUSTER);
+  const int r_hi = (int)((long long)rows * (rank + 1) / SEL_CLUSTER);
+  {
+    const int vi = threadIdx.x % vpr, rg = threadIdx.x / vpr;
+    if (rg < rpi) {
       float acc[VEC];
 #pragma unroll
       for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
-#pragma unroll 16
-      for (int rr = r0; rr < rows; rr += rpi) {
+#pragma unroll 4
+      for (int rr = r_lo + rg; rr < r_hi; rr += rpi) {
         const int t = rr / G, gg = rr - t * G;
-        const uint4 v =
-            *reinterpret_cast<const uint4*>(Q + (((size_t)b * S + t) * Hq + kvh * G + gg) * g.D + vi * VEC);
+        const uint4 v = *reinterpret_cast<const uint4*>(Q + (((size_t)b * S + t) * Hq + kvh * G + gg) * D + vi * VEC);
         add_vec16<T>(v, acc);
       }
 #pragma unroll
-      for (int k = 0; k < VEC; ++k) part[r0 * g.D + vi * VEC + k] = acc[k];
+      for (int k = 0; k < VEC; ++k) rowsum[rg * D + vi * VEC + k] = acc[k];
     }
   }
   __syncthreads();
-  for (int d = threadIdx.x; d < g.D; d += SEL_THREADS) {
+  for (int d = threadIdx.x; d < D; d += SEL_THREADS) {
     float acc = 0.f;
-    for (int w2 = 0; w2 < rpi; ++w2) acc += part[w2 * g.D + d];
+    for (int w2 = 0; w2 < rpi; ++w2) acc += rowsum[w2 * D + d];
+    part[d] = acc;
+  }
+  if (threadIdx.x == 0) kth[2] = 0.f;  // no k-th key found here yet
+  cluster.sync();
+  // qbar: the cluster's partials in rank order (the same value in every CTA)
+  for (int d = threadIdx.x; d < D; d += SEL_THREADS) {
+    float acc = 0.f;
+    for (int r = 0; r < SEL_CLUSTER; ++r) acc += cluster.map_shared_rank(part, r)[d];
     qbar[d] = acc / (float)rows;
   }
   __syncthreads();
-  // score of chunk c: four lanes per chunk, each over a quarter of D with
-  // 16-byte loads (all independent), then two shuffles
-  const float* km = Kmean + ((size_t)b * g.Hkv + kvh) * nch_total * g.D;
-  // two chunks per lane group per pass, so a 128-chunk prefix needs one pass
-  // with all of its loads in flight
-  const int q4 = threadIdx.x & 3, dq = g.D / 4;
-  constexpr int CPP = SEL_THREADS / 4;  // chunks per half-pass
-  for (int base = 0; base < nch; base += 2 * CPP) {
-    const int c0 = base + (threadIdx.x >> 2), c1 = c0 + CPP;
-    float acc0 = 0.f, acc1 = 0.f;
+  // 2. scores of this CTA's chunks: four lanes per chunk, then two shuffles
+  for (int base = c_lo; base < c_hi; base += CPP) {
+    const int c = base + (threadIdx.x >> 2);
     const float4* qr = reinterpret_cast<const float4*>(qbar + q4 * dq);
-    const float4* kr0 = reinterpret_cast<const float4*>(km + (size_t)c0 * g.D + q4 * dq);
-    const float4* kr1 = reinterpret_cast<const float4*>(km + (size_t)c1 * g.D + q4 * dq);
-#pragma unroll 8
-    for (int i = 0; i < dq / 4; ++i) {
-      const float4 q = qr[i];
-      const float4 k0 = c0 < nch ? kr0[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 k1 = c1 < nch ? kr1[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-      acc0 = fmaf(q.x, k0.x, fmaf(q.y, k0.y, fmaf(q.z, k0.z, fmaf(q.w, k0.w, acc0))));
-      acc1 = fmaf(q.x, k1.x, fmaf(q.y, k1.y, fmaf(q.z, k1.z, fmaf(q.w, k1.w, acc1))));
+    const float4* kp = reinterpret_cast<const float4*>(km + (size_t)c * D + q4 * dq);
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i < dq / 4) {
+        const float4 q = qr[i];
+        const float4 k = base == c_lo ? kr[i] : (c < c_hi ? kp[i] : make_float4(0.f, 0.f, 0.f, 0.f));
+        acc = fmaf(q.x, k.x, fmaf(q.y, k.y, fmaf(q.z, k.z, fmaf(q.w, k.w, acc))));
+      }
     }
-    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
-    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
-    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
-    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
-    if (q4 == 0 && c0 < nch) score[c0] = acc0;
-    if (q4 == 0 && c1 < nch) score[c1] = acc1;
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (q4 == 0 && c < c_hi) score[c] = acc;
+  }
+  cluster.sync();
+  // every score, from the CTAs that computed them
+  for (int r = 0; r < SEL_CLUSTER; ++r) {
+    if (r == rank) continue;
+    const int lo = (int)((long long)nch * r / SEL_CLUSTER), hi = (int)((long long)nch * (r + 1) / SEL_CLUSTER);
+    const float* rs = cluster.map_shared_rank(score, r);
+    for (int c = lo + threadIdx.x; c < hi; c += SEL_THREADS) score[c] = rs[c];
   }
   __syncthreads();
-  // rank = chunks that beat c (higher score, or equal score and lower index)
-  for (int c = threadIdx.x; c < nch; c += SEL_THREADS) {
+  // 3. rank of each own chunk; the one of rank topk - 1 is the k-th best key
+  for (int c = c_lo + threadIdx.x; c < c_hi; c += SEL_THREADS) {
     const float sc = score[c];
     int better = 0;
-    for (int c2 = 0; c2 < nch; ++c2) {
-      const float s2 = score[c2];
-      better += (s2 > sc) || (s2 == sc && c2 < c);
+    for (int c2 = 0; c2 < nch; ++c2) better += ranks_above(score[c2], c2, sc, c);
+    if (better == topk - 1) {
+      kth[0] = sc;
+      kth[1] = __int_as_float(c);
+      kth[2] = 1.f;
     }
-    sel[c] = better < topk;
+  }
+  cluster.sync();
+  // 4. the k-th key (fewer valid chunks than topk: every chunk is selected)
+  float ks = -CUDART_INF_F;
+  int kc = nch;  // selects all
+  if (nch > topk) {
+    for (int r = 0; r < SEL_CLUSTER; ++r) {
+      const float* rk = cluster.map_shared_rank(kth, r);
+      if (rk[2] != 0.f) {
+        ks = rk[0];
+        kc = __float_as_int(rk[1]);
+      }
+    }
+  }
+  cluster.sync();  // no CTA leaves while another still reads its shared memory
+  // flags of all chunks, then a block scan: the ascending-order position of
+  // each selected chunk
+  const int per = (nch + SEL_THREADS - 1) / SEL_THREADS;
+  const int f0 = min(nch, threadIdx.x * per), f1 = min(nch, f0 + per);
+  int cnt = 0;
+  for (int c = f0; c < f1; ++c) {
+    const int f = (nch <= topk) || !ranks_above(ks, kc, score[c], c);  // c at or above the k-th key
+    flag[c] = f;
+    cnt += f;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int w2 = 0; w2 < SEL_THREADS / 32; ++w2) {
+      const int v = wsum[w2];
+      wsum[w2] = acc;
+      acc += v;
+    }
+    wsum[SEL_THREADS / 32] = acc;
   }
   __syncthreads();
-  // ascending chunk order: output slot = selected chunks before c
+  int pos = wsum[warp] + incl - cnt;  // selected chunks before f0
   int32_t* out = idx + ((size_t)b * g.Hkv + kvh) * topk;
-  for (int c = threadIdx.x; c < nch; c += SEL_THREADS) {
-    if (sel[c]) {
-      int before = 0;
-      for (int c2 = 0; c2 < c; ++c2) before += sel[c2];
-      out[before] = c;
+  for (int c = f0; c < f1; ++c) {
+    if (flag[c]) {
+      if (c >= c_lo && c < c_hi && pos < topk) out[pos] = c;
+      ++pos;
     }
   }
-  const int nsel = min(topk, nch);
-  for (int i = nsel + threadIdx.x; i < topk; i += SEL_THREADS) out[i] = -1;
+  if (rank == 0) {
+    const int nsel = min(wsum[SEL_THREADS / 32], topk);
+    for (int i = nsel + threadIdx.x; i < topk; i += SEL_THREADS) out[i] = -1;
+  }
 }
 
 // One thread per 16-byte vector of the block's K and V.
@@ -386,8 +483,8 @@ cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* K
                                  int32_t* status, cudaStream_t stream) {
   const CacheGeom g = geom_of(d);
   const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
-  const size_t smem = (size_t)(SEL_PART_FLOATS + g.D + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int);
-  dim3 grid(g.Hkv, g.B);
+  const size_t smem = sel_smem_bytes(g.D, nch_total);
+  dim3 grid(SEL_CLUSTER, g.Hkv, g.B);
   cudaError_t e;
   if (d.dtype == FB_BF16) {
     auto k = select_chunks_kernel<__nv_bfloat16>;

@@ -154,6 +154,12 @@ cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CU
                            const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
                            const CUtensorMap& tmPre, const CUtensorMap& tmO, int grid, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& c, cudaStream_t stream);
+// Two 128-row query tiles per CTA (tiles 2i and 2i + 1 of a unit; the grid is
+// (b, kv head, tile pair, split) with the split fastest): for units of two or
+// more query tiles.  No active-unit split (AttnParams::dyn must be 0).
+cudaError_t launch_attn_tc2(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
+                            const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
+                            const CUtensorMap& tmO, int grid, cudaStream_t stream);
 
 // CUDA-core (fp32) path.
 cudaError_t launch_attn_simt(const AttnParams& p, const float* Q, const float* Kp,

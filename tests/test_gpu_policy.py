@@ -49,8 +49,19 @@ def test_threshold_extremes_bf16():
     assert not any(m.any() for m in masks[1:])
 
 
-@pytest.mark.parametrize("num_splits,page_size", [(0, 0), (5, 0), (0, 128), (3, 64)])
-def test_masked_prefix_pass_random_masks(num_splits, page_size):
+MASKED_SHAPES = {
+    # one query tile per unit (the grid may be shared out among the selected units)
+    "lm": dict(batch=2, prefix_len=5000, blocks=1),
+    # two and three query tiles per unit: the two-tile kernel, masked units skipped
+    "pair": dict(batch=2, block_len=64, prefix_len=3000, blocks=1),
+    "mha": dict(batch=1, num_q_heads=4, num_kv_heads=4, block_len=300, prefix_len=2000, blocks=1),
+}
+
+
+@pytest.mark.parametrize("shape,num_splits,page_size", [("lm", 0, 0), ("lm", 5, 0), ("lm", 0, 128), ("lm", 3, 64),
+                                                        ("pair", 0, 0), ("pair", 3, 128), ("mha", 0, 0),
+                                                        ("mha", 2, 0)])
+def test_masked_prefix_pass_random_masks(shape, num_splits, page_size):
     """fb_prefix_partial_masked against the oracle's prefix partial: the rows
     of selected units are recomputed, the others are left untouched (also
     when the grid is shared out among the selected units only)."""
@@ -59,7 +70,7 @@ def test_masked_prefix_pass_random_masks(num_splits, page_size):
     from gpu_cases import compare, make_layer, tensors
     from oracle import flashblock_oracle as ora
 
-    w = synth.WORKLOADS["lm_gqa"].scaled(batch=2, prefix_len=5000, blocks=1)
+    w = synth.WORKLOADS["lm_gqa"].scaled(**MASKED_SHAPES[shape])
     K, V, lens = synth.prefix_kv(w)
     Kt, K64 = tensors(w, K)
     Vt, V64 = tensors(w, V)
@@ -72,7 +83,7 @@ def test_masked_prefix_pass_random_masks(num_splits, page_size):
     masks = [np.ones((w.batch, w.num_kv_heads), np.int32), np.zeros((w.batch, w.num_kv_heads), np.int32),
              (rng.random((w.batch, w.num_kv_heads)) < 0.3).astype(np.int32)]
     one = np.zeros((w.batch, w.num_kv_heads), np.int32)
-    one[1, 5] = 1
+    one[w.batch - 1, w.num_kv_heads - 1] = 1
     masks.append(one)
     G = w.group
     for mk in masks:
