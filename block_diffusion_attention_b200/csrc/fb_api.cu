@@ -18,6 +18,10 @@ namespace fb {
 static std::atomic<uint64_t> g_launches{0};
 void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
+#ifdef FB_TEST_HOOKS
+static std::atomic<int> g_test_skip_k1{0};
+#endif
+
 namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -151,6 +155,9 @@ AttnParams base_params(const fb_desc& d) {
   p.scale = d.softmax_scale;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
   p.kv_stream_once = (p.n_rt == 1);  // one query tile per unit: each K/V byte is read once
+#ifdef FB_TEST_HOOKS
+  p.test_skip_k1 = g_test_skip_k1.load(std::memory_order_relaxed);
+#endif
   return p;
 }
 
@@ -487,6 +494,39 @@ fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const v
   return from_cuda(launch_attn_tc(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_pre, tm_out, (int)grid, s));
 }
 
+fb_status fb_block_step_append(const fb_desc* d, const void* Q, const void* Kb, const void* Vb,
+                               const float* O_pre, const float* LSE_pre, void* O, float* LSE_out, void* Kc,
+                               void* Vc, int32_t* lens_inout, int32_t* dev_status, fb_stream_t stream) {
+  fb_status st = check_desc(d);
+  if (st != FB_OK) return st;
+  if (!Q || !Kb || !Vb || !O_pre || !LSE_pre || !O || !Kc || !Vc) return FB_ERR_INVALID_ARG;
+  if (!d->prefix_lens && !lens_inout) return FB_ERR_INVALID_ARG;
+  if (d->page_size > 0) {
+    if (!pow2(d->page_size) || !d->block_table || d->max_pages <= 0 || d->num_pages <= 0)
+      return FB_ERR_INVALID_ARG;
+  } else if (d->kv_capacity <= 0) {
+    return FB_ERR_INVALID_ARG;
+  }
+  if (!aligned16(Q) || !aligned16(Kb) || !aligned16(Vb) || !aligned16(O_pre) || !aligned16(O) ||
+      !aligned16(Kc) || !aligned16(Vc) || (reinterpret_cast<uintptr_t>(LSE_pre) & 3u) ||
+      (reinterpret_cast<uintptr_t>(LSE_out) & 3u))
+    return FB_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool small = small_step_fits(*d, device_sms());
+  if (small || rows_step_fits(*d)) {
+    // one kernel: the step, and the unit's first CTA writes the block's rows
+    const StepAppend app{lens_inout ? lens_inout : d->prefix_lens, Kc, Vc, dev_status};
+    cudaError_t e = small ? launch_block_step_small(*d, Q, Kb, Vb, O_pre, LSE_pre, O, LSE_out, s, &app)
+                          : launch_block_step_rows(*d, Q, Kb, Vb, O_pre, LSE_pre, O, LSE_out, s, &app);
+    if (e != cudaSuccess || !lens_inout) return from_cuda(e);
+    return from_cuda(launch_lens_advance(*d, lens_inout, s));
+  }
+  // other shapes: the step, then the append
+  st = fb_block_step(d, Q, Kb, Vb, O_pre, LSE_pre, O, LSE_out, dev_status, stream);
+  if (st != FB_OK) return st;
+  return fb_kv_append(d, Kb, Vb, Kc, Vc, lens_inout, dev_status, stream);
+}
+
 fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc, const void* Vc,
                                 const void* Kb, const void* Vb, void* O, float* LSE_out, void* ws,
                                 size_t ws_bytes, int32_t* dev_status, fb_stream_t stream) {
@@ -659,5 +699,12 @@ const char* fb_status_string(fb_status s) {
 uint64_t fb_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int32_t fb_abi_version(void) { return FB_ABI_VERSION; }
+
+#ifdef FB_TEST_HOOKS
+// Test builds only (libflashblock_testhooks.so): 1 = the attention kernels'
+// K producers leave the load of their second key tile out, so the wait for it
+// runs out (these builds bound every wait by a short FB_WAIT_LIMIT_NS).
+void fb_test_set_skip_k1(int32_t on) { g_test_skip_k1.store(on ? 1 : 0, std::memory_order_relaxed); }
+#endif
 
 }  // extern "C"

@@ -256,10 +256,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int item = 2 * jj + kv;
         const int sl = slot_of(item);
         if (!wait_bar(&sh.empty[sl], (use_of(item) & 1) ^ 1, sh, status)) break;
+        issued = jj + 1;
+#ifdef FB_TEST_HOOKS
+        if (p.test_skip_k1 && kv == 0 && jj == 1) continue;  // never loaded: its wait runs out
+#endif
         mbar_arrive_expect_tx(&sh.full[sl], SLOT_BYTES);
         load_kv_tile(sRing + sl * SLOT_BYTES, kv ? &tmVp : &tmKp, kv ? &tmVb : &tmKb, &sh.full[sl], p, u, t, b,
                      kvh, policy);
-        issued = jj + 1;
       }
       // After an abort, let the copies in flight land before the CTA exits
       // (this producer's own: its last NSLOT / 2 items at most).
@@ -267,6 +270,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (kv == 0) wait_bar(sh.q_full, 0, sh, nullptr, false);
         if (kv == 0 && pre_smem) wait_bar(sh.pre_full, 0, sh, nullptr, false);
         for (int jj = max(0, issued - NSLOT / 2); jj < issued; ++jj) {
+#ifdef FB_TEST_HOOKS
+          if (p.test_skip_k1 && kv == 0 && jj == 1) continue;
+#endif
           const int item = 2 * jj + kv;
           wait_bar(&sh.full[slot_of(item)], use_of(item) & 1, sh, nullptr, false);
         }

@@ -191,16 +191,22 @@ __device__ __forceinline__ void producer_role(const CUtensorMap* tmQ, const CUte
     const int item = 2 * jj + kv;
     const int sl = slot2(item);
     if (!wait2(&sh.empty[sl], (use2(item) & 1) ^ 1, sh, status)) break;
+    issued = jj + 1;
+#ifdef FB_TEST_HOOKS
+    if (p.test_skip_k1 && kv == 0 && jj == 1) continue;  // never loaded: its wait runs out
+#endif
     mbar_arrive_expect_tx(&sh.full[sl], SLOT_BYTES);
     load_kv_tile(sRing + sl * SLOT_BYTES, kv ? tmVp : tmKp, kv ? tmVb : tmKb, &sh.full[sl], p, u, t, w.b, w.kvh,
                  policy);
-    issued = jj + 1;
   }
   // After an abort, let the copies in flight land before the CTA exits (this
   // producer's own: its last three items at most).
   if (*sh.abort_flag) {
     if (kv == 0) wait2(sh.q_full, 0, sh, nullptr, false);
     for (int jj = max(0, issued - (NSLOT2 + 1) / 2); jj < issued; ++jj) {
+#ifdef FB_TEST_HOOKS
+      if (p.test_skip_k1 && kv == 0 && jj == 1) continue;
+#endif
       const int item = 2 * jj + kv;
       wait2(&sh.full[slot2(item)], use2(item) & 1, sh, nullptr, false);
     }

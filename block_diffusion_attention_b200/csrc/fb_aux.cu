@@ -11,53 +11,15 @@
 // Append (Technical Summary §1: block diffusion keeps a KV cache of the blocks
 // already generated, each block causal with respect to the earlier ones):
 // a finalized block's K/V joins the prefix.
-#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
 #include "fb_internal.h"
 #include "fb_ptx.cuh"
 
-namespace cg = cooperative_groups;
-
 namespace fb {
 
 namespace {
-
-struct CacheGeom {
-  int B, Hkv, D, cap, paged, page_shift, max_pages, num_pages;
-  const int32_t* block_table;
-};
-
-CacheGeom geom_of(const fb_desc& d) {
-  CacheGeom g;
-  g.B = d.batch;
-  g.Hkv = d.num_kv_heads;
-  g.D = d.head_dim;
-  g.paged = d.page_size > 0;
-  g.page_shift = 0;
-  if (g.paged)
-    while ((1 << g.page_shift) < d.page_size) ++g.page_shift;
-  g.max_pages = d.max_pages;
-  g.num_pages = d.num_pages;
-  g.cap = g.paged ? d.max_pages * d.page_size : d.kv_capacity;
-  g.block_table = d.block_table;
-  return g;
-}
-
-// Element offset of cache row `pos` of sequence b, kv head kvh; -1 if the row
-// has no valid page.
-__device__ __forceinline__ long long cache_offset(const CacheGeom& g, int b, int pos, int kvh) {
-  if (g.paged) {
-    const int pi = pos >> g.page_shift;
-    if (pi >= g.max_pages) return -1;
-    const int pg = g.block_table[(size_t)b * g.max_pages + pi];
-    if (pg < 0 || pg >= g.num_pages) return -1;
-    const int prow = pos & ((1 << g.page_shift) - 1);
-    return (((long long)pg << g.page_shift) + prow) * g.Hkv * g.D + (long long)kvh * g.D;
-  }
-  return ((long long)b * g.cap + pos) * g.Hkv * g.D + (long long)kvh * g.D;
-}
 
 template <typename T>
 __device__ __forceinline__ float to_f(T v);
@@ -106,26 +68,25 @@ __global__ void chunk_means_kernel(const CacheGeom g, const int32_t* lens, int c
   Kmean[(((size_t)b * g.Hkv + kvh) * nch_total + c) * g.D + d] = mean;
 }
 
-// One 8-CTA thread-block cluster per (b, kv head); grid (SEL_CLUSTER, Hkv, B).
-// CTA k of the cluster
-//   1. sums its slice of the unit's S x G query rows per column (the
-//      partials are added in rank order by every CTA: one qbar for all),
-//   2. scores its slice of the chunks (its Kmean rows are loaded before the
-//      first cluster barrier, while the query loads are in flight),
-//   3. ranks its chunks against every score (a chunk's rank = chunks with a
-//      higher score, or an equal score and a lower index); the chunk of rank
-//      topk - 1 is the k-th best key,
-//   4. knowing that key, marks every chunk at or above it and writes its own
-//      selected chunks at their ascending-order positions (a block scan).
+// One CTA of SEL_THREADS per (b, kv head); grid (Hkv, B).  The CTA
+//   1. issues the loads of the first SEL_THREADS / 4 chunk means (four lanes
+//      per chunk, a quarter of D each) into registers, so they are in flight
+//      with the query loads,
+//   2. sums the unit's S x G query rows per column (16-byte vectors, the row
+//      groups added in a fixed order) into qbar,
+//   3. scores every chunk, then ranks each chunk against all scores (rank =
+//      chunks with a higher score, or an equal score and a lower index); the
+//      chunk of rank topk - 1 is the k-th best key,
+//   4. marks every chunk at or above that key and writes the selected chunks
+//      at their ascending-order positions (a block scan of the marks).
 // Dynamic shared memory: see sel_smem_bytes.
-constexpr int SEL_CLUSTER = 8;
-constexpr int SEL_THREADS = 256;
+constexpr int SEL_THREADS = 512;
 constexpr int SEL_PART_FLOATS = SEL_THREADS * 8;  // row-group sums of the query mean (16-bit inputs)
 
 size_t sel_smem_bytes(int D, int nch_total) {
-  // row-group sums, the CTA's column partial, qbar, the k-th key, every
-  // score, one flag (then scan offset) per chunk, warp totals
-  return (size_t)(SEL_PART_FLOATS + 2 * D + 4 + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int) +
+  // row-group sums, qbar, the k-th key, every score, one mark per chunk,
+  // warp totals
+  return (size_t)(SEL_PART_FLOATS + D + 4 + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int) +
          (SEL_THREADS / 32 + 1) * sizeof(int);
 }
 
@@ -156,7 +117,7 @@ __device__ __forceinline__ bool ranks_above(float sa, int a, float sb, int b) {
 }
 
 template <typename T>
-__global__ void __cluster_dims__(SEL_CLUSTER, 1, 1) __launch_bounds__(SEL_THREADS)
+__global__ void __launch_bounds__(SEL_THREADS)
     select_chunks_kernel(const CacheGeom g, const int32_t* lens, int chunk_size, int nch_total, int S, int Hq,
                          int topk, const T* __restrict__ Q, const float* __restrict__ Kmean,
                          int32_t* __restrict__ idx, int32_t* status) {
@@ -164,57 +125,49 @@ __global__ void __cluster_dims__(SEL_CLUSTER, 1, 1) __launch_bounds__(SEL_THREAD
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ float sm[];
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = (int)cluster.block_rank();
-  const int kvh = blockIdx.y;
-  const int b = blockIdx.z;
+  const int kvh = blockIdx.x;
+  const int b = blockIdx.y;
   const int G = Hq / g.Hkv;
   const int D = g.D;
   float* rowsum = sm;                       // [rpi][D] row-group sums
-  float* part = rowsum + SEL_PART_FLOATS;   // [D] this CTA's column sums
-  float* qbar = part + D;                   // [D]
-  float* kth = qbar + D;                    // {score, index as float bits, found}
-  float* score = kth + 4;                   // [nch_total] every chunk's score
-  int* flag = reinterpret_cast<int*>(score + nch_total);  // [nch_total]
-  int* wsum = flag + nch_total;             // [warps + 1]
+  float* qbar = rowsum + SEL_PART_FLOATS;   // [D]
+  float* kth = qbar + D;                    // {score, index as float bits}
+  float* score = kth + 4;                   // [nch_total]
+  int* mark = reinterpret_cast<int*>(score + nch_total);  // [nch_total]
+  int* wsum = mark + nch_total;             // [warps + 1]
   int L = lens[b];
   if (L < 0 || L > g.cap) {
-    if (threadIdx.x == 0 && rank == 0) report(status, FB_ERR_BOUNDS);
+    if (threadIdx.x == 0) report(status, FB_ERR_BOUNDS);
     L = max(0, min(L, g.cap));
   }
   const int nch = (L + chunk_size - 1) / chunk_size;
-  const int c_lo = (int)((long long)nch * rank / SEL_CLUSTER);
-  const int c_hi = (int)((long long)nch * (rank + 1) / SEL_CLUSTER);
-  // this CTA's Kmean rows (first pass: 64 chunks, 4 lanes per chunk, each a
-  // quarter of D), loaded now so they are in flight with the query loads
+  // 1. the first pass's chunk means, in flight with the query loads
   const float* km = Kmean + ((size_t)b * g.Hkv + kvh) * nch_total * D;
   const int q4 = threadIdx.x & 3, dq = D / 4;
   constexpr int CPP = SEL_THREADS / 4;  // chunks per pass
   float4 kr[8];
   {
-    const int c = c_lo + (threadIdx.x >> 2);
+    const int c = threadIdx.x >> 2;
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      kr[i] = (c < c_hi && i < dq / 4) ? reinterpret_cast<const float4*>(km + (size_t)c * D + q4 * dq)[i]
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      kr[i] = (c < nch && i < dq / 4) ? reinterpret_cast<const float4*>(km + (size_t)c * D + q4 * dq)[i]
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  // 1. column sums of this CTA's rows of the unit (16-byte vectors: thread i
-  // takes vector i % vpr of rows r0 + i / vpr, + rpi, ...; the rpi row-group
-  // sums of each column are then added in a fixed order)
+  // 2. query mean over the S block tokens and the G heads of the group:
+  // thread i takes vector i % vpr of rows i / vpr, + rpi, ...; the rpi
+  // row-group sums of each column are then added in a fixed order
   constexpr int VEC = 16 / sizeof(T);
   const int vpr = D / VEC;                // vectors per row
   const int rpi = SEL_THREADS / vpr;      // rows per iteration
   const int rows = S * G;
-  const int r_lo = (int)((long long)rows * rank / SEL_CLUSTER);
-  const int r_hi = (int)((long long)rows * (rank + 1) / SEL_CLUSTER);
   {
     const int vi = threadIdx.x % vpr, rg = threadIdx.x / vpr;
     if (rg < rpi) {
       float acc[VEC];
 #pragma unroll
       for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
-#pragma unroll 4
-      for (int rr = r_lo + rg; rr < r_hi; rr += rpi) {
+#pragma unroll 8
+      for (int rr = rg; rr < rows; rr += rpi) {
         const int t = rr / G, gg = rr - t * G;
         const uint4 v = *reinterpret_cast<const uint4*>(Q + (((size_t)b * S + t) * Hq + kvh * G + gg) * D + vi * VEC);
         add_vec16<T>(v, acc);
@@ -227,19 +180,11 @@ __global__ void __cluster_dims__(SEL_CLUSTER, 1, 1) __launch_bounds__(SEL_THREAD
   for (int d = threadIdx.x; d < D; d += SEL_THREADS) {
     float acc = 0.f;
     for (int w2 = 0; w2 < rpi; ++w2) acc += rowsum[w2 * D + d];
-    part[d] = acc;
-  }
-  if (threadIdx.x == 0) kth[2] = 0.f;  // no k-th key found here yet
-  cluster.sync();
-  // qbar: the cluster's partials in rank order (the same value in every CTA)
-  for (int d = threadIdx.x; d < D; d += SEL_THREADS) {
-    float acc = 0.f;
-    for (int r = 0; r < SEL_CLUSTER; ++r) acc += cluster.map_shared_rank(part, r)[d];
     qbar[d] = acc / (float)rows;
   }
   __syncthreads();
-  // 2. scores of this CTA's chunks: four lanes per chunk, then two shuffles
-  for (int base = c_lo; base < c_hi; base += CPP) {
+  // 3a. scores: four lanes per chunk, then two shuffles
+  for (int base = 0; base < nch; base += CPP) {
     const int c = base + (threadIdx.x >> 2);
     const float4* qr = reinterpret_cast<const float4*>(qbar + q4 * dq);
     const float4* kp = reinterpret_cast<const float4*>(km + (size_t)c * D + q4 * dq);
@@ -248,56 +193,40 @@ __global__ void __cluster_dims__(SEL_CLUSTER, 1, 1) __launch_bounds__(SEL_THREAD
     for (int i = 0; i < 8; ++i) {
       if (i < dq / 4) {
         const float4 q = qr[i];
-        const float4 k = base == c_lo ? kr[i] : (c < c_hi ? kp[i] : make_float4(0.f, 0.f, 0.f, 0.f));
+        const float4 k = base == 0 ? kr[i] : (c < nch ? kp[i] : make_float4(0.f, 0.f, 0.f, 0.f));
         acc = fmaf(q.x, k.x, fmaf(q.y, k.y, fmaf(q.z, k.z, fmaf(q.w, k.w, acc))));
       }
     }
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (q4 == 0 && c < c_hi) score[c] = acc;
-  }
-  cluster.sync();
-  // every score, from the CTAs that computed them
-  for (int r = 0; r < SEL_CLUSTER; ++r) {
-    if (r == rank) continue;
-    const int lo = (int)((long long)nch * r / SEL_CLUSTER), hi = (int)((long long)nch * (r + 1) / SEL_CLUSTER);
-    const float* rs = cluster.map_shared_rank(score, r);
-    for (int c = lo + threadIdx.x; c < hi; c += SEL_THREADS) score[c] = rs[c];
+    if (q4 == 0 && c < nch) score[c] = acc;
   }
   __syncthreads();
-  // 3. rank of each own chunk; the one of rank topk - 1 is the k-th best key
-  for (int c = c_lo + threadIdx.x; c < c_hi; c += SEL_THREADS) {
-    const float sc = score[c];
-    int better = 0;
-    for (int c2 = 0; c2 < nch; ++c2) better += ranks_above(score[c2], c2, sc, c);
-    if (better == topk - 1) {
-      kth[0] = sc;
-      kth[1] = __int_as_float(c);
-      kth[2] = 1.f;
-    }
-  }
-  cluster.sync();
-  // 4. the k-th key (fewer valid chunks than topk: every chunk is selected)
-  float ks = -CUDART_INF_F;
-  int kc = nch;  // selects all
+  // 3b. ranks; the chunk of rank topk - 1 is the k-th best key (with at most
+  // topk valid chunks every chunk is selected)
   if (nch > topk) {
-    for (int r = 0; r < SEL_CLUSTER; ++r) {
-      const float* rk = cluster.map_shared_rank(kth, r);
-      if (rk[2] != 0.f) {
-        ks = rk[0];
-        kc = __float_as_int(rk[1]);
+    for (int c = threadIdx.x; c < nch; c += SEL_THREADS) {
+      const float sc = score[c];
+      int better = 0;
+#pragma unroll 8
+      for (int c2 = 0; c2 < nch; ++c2) better += ranks_above(score[c2], c2, sc, c);
+      if (better == topk - 1) {
+        kth[0] = sc;
+        kth[1] = __int_as_float(c);
       }
     }
   }
-  cluster.sync();  // no CTA leaves while another still reads its shared memory
-  // flags of all chunks, then a block scan: the ascending-order position of
-  // each selected chunk
+  __syncthreads();
+  const float ks = nch > topk ? kth[0] : CUDART_INF_F;
+  const int kc = nch > topk ? __float_as_int(kth[1]) : -1;
+  // 4. marks (chunk at or above the k-th key), then a block scan: the
+  // ascending-order position of each selected chunk
   const int per = (nch + SEL_THREADS - 1) / SEL_THREADS;
   const int f0 = min(nch, threadIdx.x * per), f1 = min(nch, f0 + per);
   int cnt = 0;
   for (int c = f0; c < f1; ++c) {
-    const int f = (nch <= topk) || !ranks_above(ks, kc, score[c], c);  // c at or above the k-th key
-    flag[c] = f;
+    const int f = (nch <= topk) || !ranks_above(ks, kc, score[c], c);
+    mark[c] = f;
     cnt += f;
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -322,15 +251,13 @@ __global__ void __cluster_dims__(SEL_CLUSTER, 1, 1) __launch_bounds__(SEL_THREAD
   int pos = wsum[warp] + incl - cnt;  // selected chunks before f0
   int32_t* out = idx + ((size_t)b * g.Hkv + kvh) * topk;
   for (int c = f0; c < f1; ++c) {
-    if (flag[c]) {
-      if (c >= c_lo && c < c_hi && pos < topk) out[pos] = c;
+    if (mark[c]) {
+      if (pos < topk) out[pos] = c;
       ++pos;
     }
   }
-  if (rank == 0) {
-    const int nsel = min(wsum[SEL_THREADS / 32], topk);
-    for (int i = nsel + threadIdx.x; i < topk; i += SEL_THREADS) out[i] = -1;
-  }
+  const int nsel = min(wsum[SEL_THREADS / 32], topk);
+  for (int i = nsel + threadIdx.x; i < topk; i += SEL_THREADS) out[i] = -1;
 }
 
 // One thread per 16-byte vector of the block's K and V.
@@ -484,7 +411,7 @@ cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* K
   const CacheGeom g = geom_of(d);
   const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
   const size_t smem = sel_smem_bytes(g.D, nch_total);
-  dim3 grid(SEL_CLUSTER, g.Hkv, g.B);
+  dim3 grid(g.Hkv, g.B);
   cudaError_t e;
   if (d.dtype == FB_BF16) {
     auto k = select_chunks_kernel<__nv_bfloat16>;
@@ -547,8 +474,13 @@ cudaError_t launch_kv_append(const fb_desc& d, const void* Kb, const void* Vb, v
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || !lens_inout) return e;
   // (waits for the append above to complete before it moves the lengths)
-  e = launch_pdl(lens_advance_kernel, dim3((g.B + 127) / 128), dim3(128), 0, stream, lens_inout, g.B, d.block_len,
-                 g.cap);
+  return launch_lens_advance(d, lens_inout, stream);
+}
+
+cudaError_t launch_lens_advance(const fb_desc& d, int32_t* lens, cudaStream_t stream) {
+  const CacheGeom g = geom_of(d);
+  cudaError_t e = launch_pdl(lens_advance_kernel, dim3((g.B + 127) / 128), dim3(128), 0, stream, lens, g.B,
+                             d.block_len, g.cap);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -48,6 +48,10 @@ struct AttnParams {
   // slot i of out_o32 ([grid][128][D]) and out_lse ([grid][128])
   int dyn;
   KeySource src;
+  // Test builds only (FB_TEST_HOOKS): 1 = every CTA's K producer leaves the
+  // load of its second key tile out, so the pipeline wait for it runs out
+  // (the time-out path is then exercised).  Always 0 in the library proper.
+  int test_skip_k1;
   // outputs
   float* out_o32;         // EPI_PARTIAL: [nsplit][B][S][Hq][D]
   float* out_lse;         // EPI_PARTIAL: [nsplit][B][Hq][S]; others: [B][Hq][S] or null
@@ -137,18 +141,65 @@ __device__ __forceinline__ int active_splits(int grid, int n_active, int n_rt) {
   return ns < 1 ? 1 : (ns > TC_MAX_SPLITS ? TC_MAX_SPLITS : ns);
 }
 
+// Geometry of a K/V cache (contiguous [B, cap, Hkv, D] or a page pool
+// [num_pages, page, Hkv, D] addressed through block_table).
+struct CacheGeom {
+  int B, Hkv, D, cap, paged, page_shift, max_pages, num_pages;
+  const int32_t* block_table;
+};
+
+inline CacheGeom geom_of(const fb_desc& d) {
+  CacheGeom g;
+  g.B = d.batch;
+  g.Hkv = d.num_kv_heads;
+  g.D = d.head_dim;
+  g.paged = d.page_size > 0;
+  g.page_shift = 0;
+  if (g.paged)
+    while ((1 << g.page_shift) < d.page_size) ++g.page_shift;
+  g.max_pages = d.max_pages;
+  g.num_pages = d.num_pages;
+  g.cap = g.paged ? d.max_pages * d.page_size : d.kv_capacity;
+  g.block_table = d.block_table;
+  return g;
+}
+
+// Element offset of cache row `pos` of sequence b, kv head kvh; -1 if the row
+// has no valid page.
+__device__ __forceinline__ long long cache_offset(const CacheGeom& g, int b, int pos, int kvh) {
+  if (g.paged) {
+    const int pi = pos >> g.page_shift;
+    if (pi >= g.max_pages) return -1;
+    const int pg = g.block_table[(size_t)b * g.max_pages + pi];
+    if (pg < 0 || pg >= g.num_pages) return -1;
+    const int prow = pos & ((1 << g.page_shift) - 1);
+    return (((long long)pg << g.page_shift) + prow) * g.Hkv * g.D + (long long)kvh * g.D;
+  }
+  return ((long long)b * g.cap + pos) * g.Hkv * g.D + (long long)kvh * g.D;
+}
+
 // Block step of a short block on warp-level MMA (16 query rows per CTA, the
 // tile in registers): usable when small_step_fits().
+// With `app`, the step also writes the block's K/V into the cache rows
+// [L_b, L_b + S) (the append of a block's last step; lens is not advanced).
+struct StepAppend {
+  const int32_t* lens;
+  void* Kc;
+  void* Vc;
+  int32_t* status;
+};
 bool small_step_fits(const fb_desc& d, int num_sms);
 cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
                                     const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
-                                    cudaStream_t stream);
+                                    cudaStream_t stream, const StepAppend* app = nullptr);
 // The same on 64 query rows per CTA (16 per warp), for short blocks with more
 // rows than small_step_fits() takes: usable when rows_step_fits().
 bool rows_step_fits(const fb_desc& d);
 cudaError_t launch_block_step_rows(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
                                    const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
-                                   cudaStream_t stream);
+                                   cudaStream_t stream, const StepAppend* app = nullptr);
+// Advances lens[b] by S where the block fitted (after the append).
+cudaError_t launch_lens_advance(const fb_desc& d, int32_t* lens, cudaStream_t stream);
 
 cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
                            const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,

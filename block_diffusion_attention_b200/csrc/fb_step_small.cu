@@ -26,6 +26,7 @@
 #include <math_constants.h>
 
 #include <atomic>
+#include <cstring>
 
 #include "fb_internal.h"
 #include "fb_ptx.cuh"
@@ -54,7 +55,37 @@ struct SmallStepParams {
   const float* pre_lse;     // [B, Hq, S] natural log
   __nv_bfloat16* out_o;     // [B, S, Hq, D]
   float* out_lse;           // [B, Hq, S] or null
+  // The block append fused into the last step of a block (append != 0): the
+  // first CTA of each (b, kv head) writes the block's K/V rows into the cache
+  // rows [L_b, L_b + S), L_b = lens[b] read after the dependency wait; a
+  // block that does not fit is reported and not written.
+  int append;
+  CacheGeom cache;
+  const int32_t* lens;
+  __nv_bfloat16* Kc;
+  __nv_bfloat16* Vc;
+  int32_t* status;
 };
+
+// 16-byte chunk c of block row k into the cache (the append of the block's
+// K or V); returns false when the row has no cache row to go to.
+__device__ __forceinline__ bool append_chunk(const SmallStepParams& p, __nv_bfloat16* cache, int b, int kvh, int L,
+                                             int k, int c, const uint4& v) {
+  const long long off = cache_offset(p.cache, b, L + k, kvh);
+  if (off < 0) return false;
+  *reinterpret_cast<uint4*>(cache + off + c * 8) = v;
+  return true;
+}
+
+// L_b of the append, or -1 (reported) when the block does not fit.
+__device__ __forceinline__ int append_start(const SmallStepParams& p, int b) {
+  const int L = p.lens[b];
+  if (L < 0 || L + p.S > p.cache.cap) {
+    if (threadIdx.x == 0) report(p.status, FB_ERR_BOUNDS);
+    return -1;
+  }
+  return L;
+}
 
 // SP: keys padded to a multiple of 16 (16, 32 or 64); keys S .. SP - 1 are
 // zero rows in shared memory and masked out of the softmax.
@@ -111,6 +142,19 @@ __global__ void __launch_bounds__(SS_THREADS) block_step_small_kernel(const Smal
       const size_t q = ((size_t)b * p.S + pr / p.G) * p.Hq + kvh * p.G + pr % p.G;
       qr[j] = __ldg(reinterpret_cast<const uint4*>(p.Q + q * SS_D + c * 8));
     }
+  }
+  if (p.append && blockIdx.x % cpu == 0) {
+    // the last step of a block: this unit's K/V rows join the cache
+    const int L = append_start(p, b);
+    bool ok = true;
+#pragma unroll
+    for (int j = 0; j < KCH; ++j) {
+      const int i = threadIdx.x + j * SS_THREADS;
+      const int k = i >> 4, c = i & 15;
+      if (L >= 0 && k < p.S)
+        ok = append_chunk(p, p.Kc, b, kvh, L, k, c, kr[j]) && append_chunk(p, p.Vc, b, kvh, L, k, c, vr[j]) && ok;
+    }
+    if (!ok) report(p.status, FB_ERR_BOUNDS);
   }
   // cached pair of this lane's entries: dims 32 warp + 8 j + 2 (lane % 4) + {0, 1}
   float2 op[2][4];
@@ -325,6 +369,18 @@ __global__ void __launch_bounds__(SS_THREADS, 4) block_step_rows_kernel(const Sm
   }
   cp_async_wait_all();
   __syncthreads();
+  if (p.append && blockIdx.x % cpu == 0) {
+    // the last step of a block: this unit's K/V rows join the cache
+    const int L = append_start(p, b);
+    bool ok = true;
+    for (int i = threadIdx.x; L >= 0 && i < p.S * 16; i += SS_THREADS) {
+      const int k = i >> 4, c = i & 15;
+      ok = append_chunk(p, p.Kc, b, kvh, L, k, c, *reinterpret_cast<const uint4*>(sK + k * SS_ROW_BYTES + c * 16)) &&
+           append_chunk(p, p.Vc, b, kvh, L, k, c, *reinterpret_cast<const uint4*>(sV + k * SS_ROW_BYTES + c * 16)) &&
+           ok;
+    }
+    if (!ok) report(p.status, FB_ERR_BOUNDS);
+  }
   if (pr0 + wr0 >= rows_unit) return;  // this warp has no rows (no barrier follows)
 
   // ---- S = Q K^T for the warp's 16 rows
@@ -428,10 +484,11 @@ bool rows_step_fits(const fb_desc& d) {
   return d.dtype == FB_BF16 && d.head_dim == SS_D && d.block_len <= SS_MAX_S && d.batch > 0 && d.block_len > 0;
 }
 
-cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
-                                    const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
-                                    cudaStream_t stream) {
+namespace {
+SmallStepParams step_params(const fb_desc& d, const void* Q, const void* Kb, const void* Vb, const float* O_pre,
+                            const float* LSE_pre, void* O, float* LSE_out, const StepAppend* app) {
   SmallStepParams p;
+  std::memset(&p, 0, sizeof(p));
   p.B = d.batch;
   p.Hq = d.num_q_heads;
   p.Hkv = d.num_kv_heads;
@@ -445,6 +502,22 @@ cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void*
   p.pre_lse = LSE_pre;
   p.out_o = static_cast<__nv_bfloat16*>(O);
   p.out_lse = LSE_out;
+  if (app) {
+    p.append = 1;
+    p.cache = geom_of(d);
+    p.lens = app->lens;
+    p.Kc = static_cast<__nv_bfloat16*>(app->Kc);
+    p.Vc = static_cast<__nv_bfloat16*>(app->Vc);
+    p.status = app->status;
+  }
+  return p;
+}
+}  // namespace
+
+cudaError_t launch_block_step_small(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
+                                    const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
+                                    cudaStream_t stream, const StepAppend* app) {
+  const SmallStepParams p = step_params(d, Q, Kb, Vb, O_pre, LSE_pre, O, LSE_out, app);
   const int cpu = (p.S * p.G + SS_ROWS - 1) / SS_ROWS;
   const dim3 grid((unsigned)(p.B * p.Hkv * cpu));
   cudaError_t e;
@@ -477,21 +550,8 @@ cudaError_t launch_rows(const SmallStepParams& p, dim3 grid, cudaStream_t stream
 
 cudaError_t launch_block_step_rows(const fb_desc& d, const void* Q, const void* Kb, const void* Vb,
                                    const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
-                                   cudaStream_t stream) {
-  SmallStepParams p;
-  p.B = d.batch;
-  p.Hq = d.num_q_heads;
-  p.Hkv = d.num_kv_heads;
-  p.G = d.num_q_heads / d.num_kv_heads;
-  p.S = d.block_len;
-  p.scale_log2 = d.softmax_scale * SS_LOG2E;
-  p.Q = static_cast<const __nv_bfloat16*>(Q);
-  p.Kb = static_cast<const __nv_bfloat16*>(Kb);
-  p.Vb = static_cast<const __nv_bfloat16*>(Vb);
-  p.pre_o = O_pre;
-  p.pre_lse = LSE_pre;
-  p.out_o = static_cast<__nv_bfloat16*>(O);
-  p.out_lse = LSE_out;
+                                   cudaStream_t stream, const StepAppend* app) {
+  const SmallStepParams p = step_params(d, Q, Kb, Vb, O_pre, LSE_pre, O, LSE_out, app);
   const int cpu = (p.S * p.G + SR_ROWS - 1) / SR_ROWS;
   const dim3 grid((unsigned)(p.B * p.Hkv * cpu));
   cudaError_t e = p.S <= 16 ? launch_rows<16>(p, grid, stream)

@@ -70,6 +70,7 @@ def load() -> ctypes.CDLL:
             "fb_prefix_partial": (I32, [D, P, P, P, P, P, P, P, SZ, P, P]),
             "fb_prefix_partial_noalloc": (I32, [D, P, P, P, P, P, P, P, P]),
             "fb_block_step": (I32, [D, P, P, P, P, P, P, P, P, P]),
+            "fb_block_step_append": (I32, [D, P, P, P, P, P, P, P, P, P, P, P, P]),
             "fb_full_reference_gpu": (I32, [D, P, P, P, P, P, P, P, P, SZ, P, P]),
             "fb_chunk_means": (I32, [D, P, I32, I32, P, P, P]),
             "fb_chunk_means_tail": (I32, [D, P, I32, P, P, P]),
@@ -161,6 +162,13 @@ def fb_block_step(d, Q, Kblk, Vblk, O_pre, LSE_pre, O, LSE_out, dev_status, stre
     _ok("fb_block_step", load().fb_block_step(
         ctypes.byref(d), _p(Q), _p(Kblk), _p(Vblk), _p(O_pre), _p(LSE_pre), _p(O), _p(LSE_out),
         _p(dev_status), _s(stream)))
+
+
+def fb_block_step_append(d, Q, Kblk, Vblk, O_pre, LSE_pre, O, LSE_out, Kcache, Vcache, lens_inout, dev_status,
+                         stream=None):
+    _ok("fb_block_step_append", load().fb_block_step_append(
+        ctypes.byref(d), _p(Q), _p(Kblk), _p(Vblk), _p(O_pre), _p(LSE_pre), _p(O), _p(LSE_out), _p(Kcache),
+        _p(Vcache), _p(lens_inout), _p(dev_status), _s(stream)))
 
 
 def fb_full_reference_gpu(d, Q, Kcache, Vcache, Kblk, Vblk, O, LSE_out, workspace, dev_status, stream=None):

@@ -8,6 +8,7 @@ chunk list -- and exposes the calls of one block of denoising steps:
     refresh(Q)            prefix partial with this step's queries (refresh step)
     adapt(Q, Kblk, Vblk)  policy mode: refresh mask, then the masked prefix partial
     step(Q, Kblk, Vblk)   in-block partial merged with the cached pair -> O
+    step_append(...)      the block's last step and its append in one call
     full(Q, Kblk, Vblk)   uncached attention over [prefix ; block] -> O
     append(Kblk, Vblk)    finalized block joins the cache
 
@@ -168,14 +169,25 @@ class CachedBlockAttention:
                                      self.LSE_pre, self.workspace, self.status)
 
     def cached_step(self, s: int, Q, Kblk, Vblk, refresh_steps=(0,), out: Optional[torch.Tensor] = None,
-                    lse: bool = False):
+                    lse: bool = False, append: bool = False, advance: bool = True):
         """Step s of a block: the refresh its schedule (or policy) asks for,
-        then the fused step."""
+        then the fused step (with ``append``: the block's last step, which
+        also appends this step's K/V -- see ``step_append``)."""
         if self.policy is not None:
             self.adapt(Q, Kblk, Vblk, first=(s == 0))
         elif s in refresh_steps:
             self.refresh(Q)
+        if append:
+            return self.step_append(Q, Kblk, Vblk, out=out, lse=lse, advance=advance)
         return self.step(Q, Kblk, Vblk, out=out, lse=lse)
+
+    def _residual_merge(self, Q) -> None:
+        # residual mode: the cached residual merged with a fresh partial over
+        # the selected chunks (three partials in all, with the step's own)
+        fbl.fb_prefix_partial(self.desc, Q, self.K, self.V, self.chunk_idx, self.O_sel, self.LSE_sel,
+                              self.workspace, self.status)
+        fbl.fb_merge_partials(self.desc, self.O_res, self.LSE_res, self.O_sel, self.LSE_sel,
+                              self.O_pre, self.LSE_pre)
 
     def step(self, Q, Kblk, Vblk, out: Optional[torch.Tensor] = None, lse: bool = False):
         """Cached denoising step: O = merge(cached pair, in-block partial).
@@ -185,12 +197,25 @@ class CachedBlockAttention:
         if out is None:
             out = torch.empty_like(Q)
         if self.residual:
-            fbl.fb_prefix_partial(self.desc, Q, self.K, self.V, self.chunk_idx, self.O_sel, self.LSE_sel,
-                                  self.workspace, self.status)
-            fbl.fb_merge_partials(self.desc, self.O_res, self.LSE_res, self.O_sel, self.LSE_sel,
-                                  self.O_pre, self.LSE_pre)
+            self._residual_merge(Q)
         fbl.fb_block_step(self.desc, Q, Kblk, Vblk, self.O_pre, self.LSE_pre, out,
                           self.LSE if lse else None, self.status)
+        return out
+
+    def step_append(self, Q, Kblk, Vblk, out: Optional[torch.Tensor] = None, lse: bool = False,
+                    advance: bool = True):
+        """The last denoising step of a block together with the block's
+        append (one kernel for short blocks): the same as ``step`` then
+        ``append(Kblk, Vblk, advance)``."""
+        if out is None:
+            out = torch.empty_like(Q)
+        if self.residual:
+            self._residual_merge(Q)
+        fbl.fb_block_step_append(self.desc, Q, Kblk, Vblk, self.O_pre, self.LSE_pre, out,
+                                 self.LSE if lse else None, self.K, self.V, self.lens if advance else None,
+                                 self.status)
+        if advance and self.topk > 0:
+            fbl.fb_chunk_means_tail(self.desc, self.K, self.S, self.Kmean, self.status)
         return out
 
     def full(self, Q, Kblk, Vblk, out: Optional[torch.Tensor] = None, lse: bool = False):
@@ -215,18 +240,32 @@ class CachedBlockAttention:
             fbl.fb_chunk_means_tail(self.desc, self.K, self.S, self.Kmean, self.status)
 
     # ------------------------------------------------------------ graphs
+    def _issue_block(self, steps, outs, refresh_steps, append_kv, advance, cached, prologue=None, epilogue=None):
+        # the block's append rides on its last cached step when it appends
+        # that step's own K/V
+        last = len(steps) - 1
+        fuse = (cached and append_kv is not None and last >= 0 and append_kv[0] is steps[last][1]
+                and append_kv[1] is steps[last][2])
+        for s, (Q, Kb, Vb) in enumerate(steps):
+            if prologue is not None:
+                prologue(s)
+            if cached:
+                self.cached_step(s, Q, Kb, Vb, refresh_steps, out=outs[s], append=fuse and s == last,
+                                 advance=advance)
+            else:
+                self.full(Q, Kb, Vb, out=outs[s])
+            if epilogue is not None:
+                epilogue(s)
+        if append_kv is not None and not fuse:
+            self.append(append_kv[0], append_kv[1], advance=advance)
+
     def run_block(self, steps, outs, refresh_steps, append_kv=None, advance=True, cached=True):
         """Issue one block of denoising steps: ``steps`` is a list of (Q, Kblk,
         Vblk) device tensors, ``outs`` the per-step outputs.  Cached: refresh at
         ``refresh_steps``, fused step everywhere; uncached: full attention at
-        every step.  Ends with the append of ``append_kv`` when given."""
-        for s, (Q, Kb, Vb) in enumerate(steps):
-            if cached:
-                self.cached_step(s, Q, Kb, Vb, refresh_steps, out=outs[s])
-            else:
-                self.full(Q, Kb, Vb, out=outs[s])
-        if append_kv is not None:
-            self.append(append_kv[0], append_kv[1], advance=advance)
+        every step.  Ends with the append of ``append_kv`` when given (fused
+        into the last cached step when it is that step's K/V)."""
+        self._issue_block(steps, outs, refresh_steps, append_kv, advance, cached)
 
     def capture_block(self, steps, outs, refresh_steps, append_kv=None, cached=True, prologue=None,
                       epilogue=None, advance=True):
@@ -245,17 +284,7 @@ class CachedBlockAttention:
         host<->device copies.  Returns the ``torch.cuda.CUDAGraph``.
         """
         def body():
-            for s, (Q, Kb, Vb) in enumerate(steps):
-                if prologue is not None:
-                    prologue(s)
-                if cached:
-                    self.cached_step(s, Q, Kb, Vb, refresh_steps, out=outs[s])
-                else:
-                    self.full(Q, Kb, Vb, out=outs[s])
-                if epilogue is not None:
-                    epilogue(s)
-            if append_kv is not None:
-                self.append(append_kv[0], append_kv[1], advance=advance)
+            self._issue_block(steps, outs, refresh_steps, append_kv, advance, cached, prologue, epilogue)
 
         body()
         torch.cuda.synchronize()

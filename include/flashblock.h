@@ -237,6 +237,19 @@ fb_status fb_kv_append(const fb_desc* d, const void* Kblk, const void* Vblk,
                        void* Kcache, void* Vcache, int32_t* lens_inout,
                        int32_t* dev_status, fb_stream_t stream);
 
+/* The last denoising step of a block, with the block's append: the same
+ * results as fb_block_step followed by fb_kv_append(d, Kblk, Vblk, Kcache,
+ * Vcache, lens_inout, ...) (Core Mechanism: the step's output; Technical
+ * Summary §1: the finished block joins the cache).  For short blocks (S <= 64,
+ * bf16) it is one kernel -- the step kernel also writes the block's K/V rows
+ * into the cache rows [L_b, L_b + S) -- plus the length update when
+ * lens_inout is not NULL; other shapes run the two calls.  Arguments, layouts
+ * and errors as for those two calls. */
+fb_status fb_block_step_append(const fb_desc* d, const void* Q, const void* Kblk, const void* Vblk,
+                               const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
+                               void* Kcache, void* Vcache, int32_t* lens_inout, int32_t* dev_status,
+                               fb_stream_t stream);
+
 /* Bytes of the static scratch array behind fb_prefix_partial_noalloc. */
 #define FB_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 

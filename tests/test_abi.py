@@ -20,6 +20,18 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), f"{n} declared in flashblock.h but not exported"
 
 
+def test_test_hooks_only_in_the_test_library(lib):
+    # the hook that leaves a K load out lives only in the test-only build
+    import os
+    from block_diffusion_attention_b200.build import TEST_LIB
+    assert not hasattr(lib, "fb_test_set_skip_k1")
+    assert os.path.exists(TEST_LIB)
+    tl = ctypes.CDLL(TEST_LIB)
+    assert hasattr(tl, "fb_test_set_skip_k1")
+    for n in fbl.header_functions():
+        assert hasattr(tl, n), n
+
+
 def test_version_and_status_strings(lib):
     assert fbl.fb_abi_version() == 1
     for code, name in fbl.STATUS.items():

@@ -235,6 +235,40 @@ def test_block_graph_advances_the_sequence(name):
         gpu_cases.compare("chunk means after the replays", layer.Kmean.cpu().numpy(), Km, "fp32")
 
 
+@pytest.mark.parametrize("batch,page_size", [(1, 0), (1, 64), (12, 0), (12, 128)])
+def test_step_append_equals_step_then_append(batch, page_size):
+    # the block's last step with its append fused into the step kernel (the
+    # 16-row kernel at batch 1, the 64-row kernel at batch 12): the same
+    # output, cache rows and lengths as fb_block_step then fb_kv_append
+    w = W["lm_gqa"].scaled(batch=batch, prefix_len=600, prefix_min=300, blocks=2, steps=1)
+    K, V, lens = synth.prefix_kv(w)
+    Kt, Vt = gpu_cases.tensors(w, K)[0], gpu_cases.tensors(w, V)[0]
+    ref = gpu_cases.make_layer(w, page_size=page_size)
+    fused = gpu_cases.make_layer(w, page_size=page_size)
+    for layer in (ref, fused):
+        layer.load_prefix(Kt, Vt, lens)
+    base = synth.block_base(w, 0)
+    Q, Kb, Vb = (gpu_cases.tensors(w, x)[0] for x in synth.step_inputs(w, 0, 0, base))
+    for layer in (ref, fused):
+        layer.refresh(Q)
+    o_ref = ref.step(Q, Kb, Vb)
+    ref.append(Kb, Vb)
+    o_fused = fused.step_append(Q, Kb, Vb)
+    ref.check()
+    fused.check()
+    assert torch.equal(o_fused, o_ref)
+    assert torch.equal(fused.lens, ref.lens)
+    assert torch.equal(fused.K, ref.K) and torch.equal(fused.V, ref.V)
+    # a block that does not fit is reported and not written
+    fused.lens.fill_(fbl.fb_cache_rows(fused.desc) - w.block_len + 1)
+    before = fused.K.clone()
+    fused.step_append(Q, Kb, Vb)
+    with pytest.raises(fbl.FlashBlockError) as e:
+        fused.check()
+    assert e.value.status == 7
+    assert torch.equal(fused.K, before)
+
+
 def test_residual_sparse_reuse():
     # residual reuse: cached unselected-chunk partial + fresh selected chunks + block
     w = W["batched_sparse"].scaled(batch=3, num_q_heads=8, num_kv_heads=2, prefix_len=1500,
