@@ -143,19 +143,6 @@ __global__ void __launch_bounds__(SS_THREADS) block_step_small_kernel(const Smal
       qr[j] = __ldg(reinterpret_cast<const uint4*>(p.Q + q * SS_D + c * 8));
     }
   }
-  if (p.append && blockIdx.x % cpu == 0) {
-    // the last step of a block: this unit's K/V rows join the cache
-    const int L = append_start(p, b);
-    bool ok = true;
-#pragma unroll
-    for (int j = 0; j < KCH; ++j) {
-      const int i = threadIdx.x + j * SS_THREADS;
-      const int k = i >> 4, c = i & 15;
-      if (L >= 0 && k < p.S)
-        ok = append_chunk(p, p.Kc, b, kvh, L, k, c, kr[j]) && append_chunk(p, p.Vc, b, kvh, L, k, c, vr[j]) && ok;
-    }
-    if (!ok) report(p.status, FB_ERR_BOUNDS);
-  }
   // cached pair of this lane's entries: dims 32 warp + 8 j + 2 (lane % 4) + {0, 1}
   float2 op[2][4];
   float lp[2];
@@ -178,6 +165,21 @@ __global__ void __launch_bounds__(SS_THREADS) block_step_small_kernel(const Smal
     *reinterpret_cast<uint4*>(sK + k * SS_ROW_BYTES + c * 16) = kr[j];
     *reinterpret_cast<uint4*>(sV + k * SS_ROW_BYTES + c * 16) = vr[j];
   }
+  // (after every load of the CTA is in flight)
+  if (p.append && blockIdx.x % cpu == 0) {
+    // the last step of a block: this unit's K/V rows join the cache
+    const int L = append_start(p, b);
+    bool ok = true;
+#pragma unroll
+    for (int j = 0; j < KCH; ++j) {
+      const int i = threadIdx.x + j * SS_THREADS;
+      const int k = i >> 4, c = i & 15;
+      if (L >= 0 && k < p.S)
+        ok = append_chunk(p, p.Kc, b, kvh, L, k, c, kr[j]) && append_chunk(p, p.Vc, b, kvh, L, k, c, vr[j]) && ok;
+    }
+    if (!ok) report(p.status, FB_ERR_BOUNDS);
+  }
+
 #pragma unroll
   for (int j = 0; j < QCH; ++j) {
     const int i = threadIdx.x + j * SS_THREADS;
