@@ -180,11 +180,11 @@ long long cta_units(const fb_desc& d) {
 // Key-range splits of the prefix pass.  Cost model in key-tile times: every
 // wave of CTAs costs its longest split plus a fixed per-CTA overhead (set-up,
 // pipeline fill, epilogue ~ 3 tiles), and splitting adds a combine pass
-// (~ 2 tiles).  Splits keep at least 4 tiles each.
+// (~ 2 tiles).  Splits keep at least 3 tiles each.
 int choose_splits(const fb_desc& d, long long est_tiles) {
   if (d.dtype != FB_BF16) return 1;
   const long long units = cta_units(d);
-  long long max_ns = est_tiles / 4;
+  long long max_ns = est_tiles / 3;
   if (max_ns < 1) max_ns = 1;
   if (max_ns > TC_MAX_SPLITS) max_ns = TC_MAX_SPLITS;
   if (d.num_splits > 0)

@@ -86,8 +86,8 @@ constexpr int SEL_PART_FLOATS = SEL_THREADS * 8;  // row-group sums of the query
 size_t sel_smem_bytes(int D, int nch_total) {
   // row-group sums, qbar, the k-th key, every score, one mark per chunk,
   // warp totals
-  return (size_t)(SEL_PART_FLOATS + D + 4 + nch_total) * sizeof(float) + (size_t)nch_total * sizeof(int) +
-         (SEL_THREADS / 32 + 1) * sizeof(int);
+  return (size_t)(SEL_PART_FLOATS + D + 4 + ((nch_total + 3) & ~3)) * sizeof(float) +
+         (size_t)nch_total * sizeof(int) + (SEL_THREADS / 32 + 1) * sizeof(int);
 }
 
 // Adds the eight bf16 or four f32 values of a 16-byte vector to acc.
@@ -132,16 +132,13 @@ __global__ void __launch_bounds__(SEL_THREADS)
   float* rowsum = sm;                       // [rpi][D] row-group sums
   float* qbar = rowsum + SEL_PART_FLOATS;   // [D]
   float* kth = qbar + D;                    // {score, index as float bits}
-  float* score = kth + 4;                   // [nch_total]
-  int* mark = reinterpret_cast<int*>(score + nch_total);  // [nch_total]
+  float* score = kth + 4;                   // [nch_total rounded up to 4], 16-byte aligned
+  int* mark = reinterpret_cast<int*>(score + ((nch_total + 3) & ~3));  // [nch_total]
   int* wsum = mark + nch_total;             // [warps + 1]
-  int L = lens[b];
-  if (L < 0 || L > g.cap) {
-    if (threadIdx.x == 0) report(status, FB_ERR_BOUNDS);
-    L = max(0, min(L, g.cap));
-  }
-  const int nch = (L + chunk_size - 1) / chunk_size;
-  // 1. the first pass's chunk means, in flight with the query loads
+  // 1. the first pass's chunk means, loaded before anything else (rows below
+  // nch_total always exist, whatever the prefix length), in flight with the
+  // query loads.  Lane q4 of a chunk's four takes the float4s q4, q4 + 4, ...
+  // of its mean row, so the four lanes read 64 contiguous bytes per step.
   const float* km = Kmean + ((size_t)b * g.Hkv + kvh) * nch_total * D;
   const int q4 = threadIdx.x & 3, dq = D / 4;
   constexpr int CPP = SEL_THREADS / 4;  // chunks per pass
@@ -150,9 +147,15 @@ __global__ void __launch_bounds__(SEL_THREADS)
     const int c = threadIdx.x >> 2;
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      kr[i] = (c < nch && i < dq / 4) ? reinterpret_cast<const float4*>(km + (size_t)c * D + q4 * dq)[i]
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      kr[i] = (c < nch_total && i < dq / 4) ? reinterpret_cast<const float4*>(km + (size_t)c * D)[4 * i + q4]
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  int L = lens[b];
+  if (L < 0 || L > g.cap) {
+    if (threadIdx.x == 0) report(status, FB_ERR_BOUNDS);
+    L = max(0, min(L, g.cap));
+  }
+  const int nch = (L + chunk_size - 1) / chunk_size;
   // 2. query mean over the S block tokens and the G heads of the group:
   // thread i takes vector i % vpr of rows i / vpr, + rpi, ...; the rpi
   // row-group sums of each column are then added in a fixed order
@@ -186,14 +189,14 @@ __global__ void __launch_bounds__(SEL_THREADS)
   // 3a. scores: four lanes per chunk, then two shuffles
   for (int base = 0; base < nch; base += CPP) {
     const int c = base + (threadIdx.x >> 2);
-    const float4* qr = reinterpret_cast<const float4*>(qbar + q4 * dq);
-    const float4* kp = reinterpret_cast<const float4*>(km + (size_t)c * D + q4 * dq);
+    const float4* qr = reinterpret_cast<const float4*>(qbar);
+    const float4* kp = reinterpret_cast<const float4*>(km + (size_t)c * D);
     float acc = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if (i < dq / 4) {
-        const float4 q = qr[i];
-        const float4 k = base == 0 ? kr[i] : (c < nch ? kp[i] : make_float4(0.f, 0.f, 0.f, 0.f));
+        const float4 q = qr[4 * i + q4];
+        const float4 k = base == 0 ? kr[i] : (c < nch ? kp[4 * i + q4] : make_float4(0.f, 0.f, 0.f, 0.f));
         acc = fmaf(q.x, k.x, fmaf(q.y, k.y, fmaf(q.z, k.z, fmaf(q.w, k.w, acc))));
       }
     }
@@ -205,12 +208,20 @@ __global__ void __launch_bounds__(SEL_THREADS)
   // 3b. ranks; the chunk of rank topk - 1 is the k-th best key (with at most
   // topk valid chunks every chunk is selected)
   if (nch > topk) {
-    for (int c = threadIdx.x; c < nch; c += SEL_THREADS) {
-      const float sc = score[c];
+    // four lanes per chunk, each counting a quarter of the others (four
+    // scores per shared-memory read), then two shuffles
+    for (int base = 0; base < nch; base += CPP) {
+      const int c = base + (threadIdx.x >> 2);
+      const float sc = c < nch ? score[c] : 0.f;
       int better = 0;
-#pragma unroll 8
-      for (int c2 = 0; c2 < nch; ++c2) better += ranks_above(score[c2], c2, sc, c);
-      if (better == topk - 1) {
+      for (int c0 = 4 * q4; c0 < nch; c0 += 16) {
+        const float4 s4 = *reinterpret_cast<const float4*>(score + c0);  // (padded: see below)
+        better += (c0 < nch && ranks_above(s4.x, c0, sc, c)) + (c0 + 1 < nch && ranks_above(s4.y, c0 + 1, sc, c)) +
+                  (c0 + 2 < nch && ranks_above(s4.z, c0 + 2, sc, c)) + (c0 + 3 < nch && ranks_above(s4.w, c0 + 3, sc, c));
+      }
+      better += __shfl_xor_sync(0xffffffffu, better, 1);
+      better += __shfl_xor_sync(0xffffffffu, better, 2);
+      if (q4 == 0 && c < nch && better == topk - 1) {
         kth[0] = sc;
         kth[1] = __int_as_float(c);
       }
