@@ -51,9 +51,13 @@ def make_layer(w, page_size=0, num_splits=0, topk=None, residual=False):
         chunk_size=w.chunk_size if topk else 0, topk=topk, num_splits=num_splits, residual=residual)
 
 
-def run_workload(w, page_size=0, num_splits=0, check_full=True, steps=None, blocks=None):
-    """Runs the workload on GPU and oracle; returns per-step error records."""
+def run_workload(w, page_size=0, num_splits=0, check_full=True, steps=None, blocks=None, v_scale=1.0):
+    """Runs the workload on GPU and oracle; returns per-step error records.
+
+    v_scale (a power of two, so the scaled values round to bf16 exactly as
+    the unscaled ones do) multiplies every value row, prefix and block."""
     K, V, lens = synth.prefix_kv(w)
+    V = V * np.float32(v_scale)
     Kt, K64 = tensors(w, K)
     Vt, V64 = tensors(w, V)
     layer = make_layer(w, page_size, num_splits)
@@ -68,6 +72,7 @@ def run_workload(w, page_size=0, num_splits=0, check_full=True, steps=None, bloc
         pre = None
         for s in range(nsteps):
             Q, Kb, Vb = synth.step_inputs(w, blk, s, base)
+            Vb = Vb * np.float32(v_scale)
             Qt, Q64 = tensors(w, Q)
             Kbt, Kb64 = tensors(w, Kb)
             Vbt, Vb64 = tensors(w, Vb)

@@ -28,7 +28,7 @@ def _res(w, with_e2e=True, **kw):
            "lens1": [w.prefix_len] * w.batch, "ms_cached": 0.6, "ms_cached_eager": 0.7, "ms_unc": 3.0,
            "graph": True, "launches": 44, "clocks": {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}}
     if with_e2e:
-        res.update({"ms_e2e": 1.2, "h2d": 1000, "d2h": 500})
+        res.update({"ms_e2e": 1.2, "h2d": 1000, "d2h": 500, "h2d_ms": 0.1, "d2h_ms": 0.05})
     res.update(kw)
     return res
 
@@ -49,6 +49,7 @@ def test_report_line_has_contract_keys(capsys, kw):
     roof = line["roofline"]
     assert roof["bound"] in ("hbm", "tensor") and roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"])
     assert line["e2e"]["h2d_bytes_per_step"] == 1000 and line["e2e"]["d2h_bytes_per_step"] == 500
+    assert line["e2e"]["h2d_gbs"] == pytest.approx(1000 / 0.1e-3 / 1e9)
     if args.policy:
         assert line["config"]["policy"]["name"] == args.policy
         assert line["refresh_fraction"] == 0.25

@@ -111,9 +111,14 @@ def test_other_softmax_scale():
 
 def test_large_logits_rescale_path():
     # Q ~ N(0, 4): logits with std ~ 22, so the running row max keeps growing
-    # and the lazy rescale of the accumulator fires.
+    # and the lazy rescale of the accumulator fires.  Such a peaked softmax
+    # returns single value rows, so the values are scaled by 1/4 (exact in
+    # bf16): with |O| up to ~1.2 half an ulp of the bf16 output (2^-9 |O|)
+    # stays well below the 2e-2 bound, as it does on the workloads' own
+    # distributions (at |O| ~ 4-5 the output's rounding alone would be
+    # 1.6e-2).
     w = W["lm_gqa"].scaled(prefix_len=1200, blocks=1, steps=2, q_std=2.0, softmax_scale=1.0)
-    gpu_cases.run_workload(w)
+    gpu_cases.run_workload(w, v_scale=0.25)
 
 
 def test_refresh_determinism_bitwise():
