@@ -16,8 +16,11 @@ the configured prefix.
 
 By default each block is recorded once as a CUDA graph and replayed (the
 library's calls are capturable); ``--no-graph`` issues every call from the
-host.  The eager cached block is always timed too: CUDA events around its
-prefix pass give the roofline figures of the dominant kernel.
+host.  The eager cached block is always timed too.  CUDA events around the
+prefix pass inside the timed blocks give the roofline figures of the dominant
+kernel; the line also gives the pass timed 16 times back to back in a graph
+(no event nodes next to it) and, where the KV cache fits in L2, after an L2
+flush.
 
 ``value`` is cached attention tokens/s over all ranks (B * S tokens finalized
 per block per rank).  Under torchrun each rank runs an independent replica
@@ -47,7 +50,10 @@ METRIC = "attention µs/denoise-step and tokens/s, cached vs uncached; prefix-pa
 # kernel sources it was captured on (see kernel_source_hash).  An entry whose
 # hash differs from the built sources is not reported: the kernel changed
 # since the counters were taken.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/prefix_pass_long_ctx.md, capture b12_prof_lc
+    "long_ctx": {"bytes": 537204480 + 5754624, "sources": "08128c1f3bfb20b5"},
+}
 KERNEL_SOURCES = ("fb_attn_tc.cu", "fb_ptx.cuh", "fb_internal.h", "fb_api.cu")
 
 
@@ -509,6 +515,28 @@ def run_ours(args):
     torch.cuda.synchronize()
     res["blk_ms"] = [e0.elapsed_time(e1) / reps]
     del g_steps
+    if not policy:
+        # the prefix pass on its own: 16 passes back to back in one graph,
+        # CUDA events around the replay (each pass's start overlaps its
+        # predecessor's end, as inside a block without event nodes)
+        Q0 = dev_in[0][0]
+        cached.select(Q0)
+        for _ in range(3):
+            cached.prefix(Q0)
+        torch.cuda.synchronize()
+        g_pre = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_pre):
+            for _ in range(16):
+                cached.prefix(Q0)
+        g_pre.replay()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g_pre.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res["pre_b2b_ms"] = e0.elapsed_time(e1) / 16
+        del g_pre
     if not policy and kv_cache_bytes(w) < L2_BYTES:
         # The KV cache fits in L2, so the replayed blocks time the prefix pass
         # L2-warm.  Cold figure: before each pass a 256 MB scratch buffer is
@@ -724,6 +752,8 @@ def report(args, w0, w, world, res):
         "block_step_us": blk_avg * 1e3,
         "refresh_fraction": res.get("refresh_fraction"),
         "prefix_gbs": achieved,
+        "prefix_pass_back_to_back_us": (res["pre_b2b_ms"] * 1e3) if res.get("pre_b2b_ms") else None,
+        "prefix_gbs_back_to_back": (abytes / (res["pre_b2b_ms"] * 1e-3) / 1e9) if res.get("pre_b2b_ms") else None,
         "prefix_pass_l2_cold_us": cold_us,
         "prefix_gbs_l2_cold": (abytes / (cold_us * 1e-6) / 1e9) if cold_us else None,
         "prefix_hbm_frac_l2_cold": (abytes / (cold_us * 1e-6) / 1e9 / hbm_peak) if cold_us else None,
