@@ -82,6 +82,16 @@ def test_wide_groups(B, L, S, G):
     gpu_cases.run_workload(w)
 
 
+@pytest.mark.parametrize("page_size,num_splits", [(64, 0), (128, 3), (0, 5)])
+def test_two_tile_kernel_paged_and_split(page_size, num_splits):
+    # units of three query tiles (G = 1, 300 tokens = 2 x 128 + 44): a tile
+    # pair plus a lone ragged tile on the two-tile kernel, with paged caches
+    # and explicit key splits (prefix pass and uncached pass), two blocks with
+    # the append in between
+    w = W["video"].scaled(num_q_heads=2, num_kv_heads=2, block_len=300, prefix_len=1500, steps=2, blocks=2)
+    gpu_cases.run_workload(w, page_size=page_size, num_splits=num_splits)
+
+
 def test_block_step_kernel_choice_both_paths():
     # short blocks with few query rows run the warp-level MMA step kernel with
     # 16 rows per CTA; with more rows than one wave of those CTAs, the one
