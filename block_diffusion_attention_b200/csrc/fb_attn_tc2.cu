@@ -409,6 +409,14 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tmO, const AttnP
       s[c + 4] = x2.x; s[c + 5] = x2.y; s[c + 6] = x3.x; s[c + 7] = x3.y;
       la = fadd2(la, fadd2(x0, x1));
       lb = fadd2(lb, fadd2(x2, x3));
+      if (c == NC / 2 - 8) {
+        // P of the first 64 keys (bf16 pairs over the first 32 columns of
+        // S_X) stored while the second half's exponentials run
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
+        tmem_st_32x32(tS, pk);
+      }
     }
     l_run = l_run * alpha + ((la.x + la.y) + (lb.x + lb.y));
     m_run = m_new;
@@ -426,12 +434,12 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tmO, const AttnP
       }
     }
     // P as bf16 pairs over the first 64 columns of S_X: the A operand of PV
-#pragma unroll
-    for (int c = 0; c < NC / 64; ++c) {
+    {
+      // P of the last 64 keys: the A operand of PV is the first 64 columns of S_X
       uint32_t pk[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[c * 64 + 2 * i], s[c * 64 + 2 * i + 1]);
-      tmem_st_32x32(tS + c * 32, pk);
+      for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s[NC / 2 + 2 * i], s[NC / 2 + 2 * i + 1]);
+      tmem_st_32x32(tS + 32, pk);
     }
     tmem_st_wait();
     tc_fence_before_sync();
