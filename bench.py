@@ -51,8 +51,8 @@ METRIC = "attention µs/denoise-step and tokens/s, cached vs uncached; prefix-pa
 # hash differs from the built sources is not reported: the kernel changed
 # since the counters were taken.
 NCU_TRAFFIC = {
-    # profiles/prefix_pass_long_ctx.md, capture b12_prof_lc
-    "long_ctx": {"bytes": 537204480 + 5754624, "sources": "08128c1f3bfb20b5"},
+    # profiles/prefix_pass_long_ctx.md, capture b16_prof_lc
+    "long_ctx": {"bytes": 537205760 + 3928320, "sources": "3d596fe3a1abc379"},
 }
 KERNEL_SOURCES = ("fb_attn_tc.cu", "fb_ptx.cuh", "fb_internal.h", "fb_api.cu")
 
