@@ -182,8 +182,8 @@ def test_block_graph_replay_matches_eager():
         assert torch.equal(outs[s], eager[s]), f"step {s}"
 
 
-@pytest.mark.parametrize("name", ["lm_gqa", "batched_sparse"])
-def test_block_graph_advances_the_sequence(name):
+@pytest.mark.parametrize("name,page_size", [("lm_gqa", 0), ("batched_sparse", 0), ("batched_sparse", 128)])
+def test_block_graph_advances_the_sequence(name, page_size):
     # one block recorded once and replayed for consecutive blocks: each replay
     # appends the finalized block after the current prefix, advances the
     # device lengths and (sparse prefix) recomputes the touched chunk means,
@@ -197,7 +197,7 @@ def test_block_graph_advances_the_sequence(name):
     K, V, lens = synth.prefix_kv(w)
     Kt, K64 = gpu_cases.tensors(w, K)
     Vt, V64 = gpu_cases.tensors(w, V)
-    layer = gpu_cases.make_layer(w)
+    layer = gpu_cases.make_layer(w, page_size=page_size)
     layer.load_prefix(Kt, Vt, lens)
 
     def block_inputs(blk):
@@ -250,12 +250,16 @@ def test_block_graph_advances_the_sequence(name):
         gpu_cases.compare("chunk means after the replays", layer.Kmean.cpu().numpy(), Km, "fp32")
 
 
-@pytest.mark.parametrize("batch,page_size", [(1, 0), (1, 64), (12, 0), (12, 128)])
-def test_step_append_equals_step_then_append(batch, page_size):
+@pytest.mark.parametrize("batch,page_size,block_len,wl", [(1, 0, 32, "lm_gqa"), (1, 64, 32, "lm_gqa"),
+                                                          (12, 0, 32, "lm_gqa"), (12, 128, 32, "lm_gqa"),
+                                                          (2, 0, 100, "lm_gqa"), (2, 0, 16, "tiny_fp32")])
+def test_step_append_equals_step_then_append(batch, page_size, block_len, wl):
     # the block's last step with its append fused into the step kernel (the
-    # 16-row kernel at batch 1, the 64-row kernel at batch 12): the same
-    # output, cache rows and lengths as fb_block_step then fb_kv_append
-    w = W["lm_gqa"].scaled(batch=batch, prefix_len=600, prefix_min=300, blocks=2, steps=1)
+    # 16-row kernel at batch 1, the 64-row kernel at batch 12; a 100-token
+    # block and the fp32 path run the step and the append one after the
+    # other): the same output, cache rows and lengths as fb_block_step then
+    # fb_kv_append
+    w = W[wl].scaled(batch=batch, prefix_len=600, prefix_min=300, blocks=2, steps=1, block_len=block_len)
     K, V, lens = synth.prefix_kv(w)
     Kt, Vt = gpu_cases.tensors(w, K)[0], gpu_cases.tensors(w, V)[0]
     ref = gpu_cases.make_layer(w, page_size=page_size)
