@@ -14,6 +14,7 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include "fb_attn_common.cuh"
 #include "fb_internal.h"
 #include "fb_ptx.cuh"
 
@@ -76,18 +77,18 @@ __global__ void chunk_means_kernel(const CacheGeom g, const int32_t* lens, int c
 //      groups added in a fixed order) into qbar,
 //   3. scores every chunk, then ranks each chunk against all scores (rank =
 //      chunks with a higher score, or an equal score and a lower index); the
-//      chunk of rank topk - 1 is the k-th best key,
-//   4. marks every chunk at or above that key and writes the selected chunks
-//      at their ascending-order positions (a block scan of the marks).
+//      chunks of rank below topk are the selected ones,
+//   4. writes the selected chunks at their ascending-order positions
+//      (select_from_scores).
 // Dynamic shared memory: see sel_smem_bytes.
 constexpr int SEL_THREADS = 512;
 constexpr int SEL_PART_FLOATS = SEL_THREADS * 8;  // row-group sums of the query mean (16-bit inputs)
 
 size_t sel_smem_bytes(int D, int nch_total) {
-  // row-group sums, qbar, the k-th key, every score, one mark per chunk,
-  // warp totals
-  return (size_t)(SEL_PART_FLOATS + D + 4 + ((nch_total + 3) & ~3)) * sizeof(float) +
-         (size_t)nch_total * sizeof(int) + (SEL_THREADS / 32 + 1) * sizeof(int);
+  // row-group sums, qbar, every score (padded to 4), every key (padded to
+  // 2), one rank per chunk, warp totals
+  return (size_t)(SEL_PART_FLOATS + D + ((nch_total + 3) & ~3)) * sizeof(float) +
+         (size_t)((nch_total + 1) & ~1) * 8 + (size_t)nch_total * sizeof(int) + (SEL_THREADS / 32) * sizeof(int);
 }
 
 // Adds the eight bf16 or four f32 values of a 16-byte vector to acc.
@@ -111,9 +112,71 @@ __device__ __forceinline__ void add_vec16<float>(const uint4& v, float* acc) {
   acc[3] += __uint_as_float(v.w);
 }
 
-// Does chunk a (score sa) rank above chunk b (score sb)?
-__device__ __forceinline__ bool ranks_above(float sa, int a, float sb, int b) {
-  return sa > sb || (sa == sb && a < b);
+// The selection order -- chunk a ranks above chunk b iff its score is higher,
+// or equal with a lower index -- as one unsigned 64-bit key: the score's bits
+// made monotonic (-0 taken as +0, so that equal scores compare equal), then
+// the chunk index inverted; a chunk ranks above another iff its key is larger.
+__device__ __forceinline__ unsigned long long rank_key(float sc, int c) {
+  uint32_t u = __float_as_uint(sc + 0.f);
+  u ^= (u >> 31) ? 0xffffffffu : 0x80000000u;
+  return ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)c);
+}
+
+// Steps 3b and 4 of the selection, from the scores of the nch valid chunks in
+// shared memory (key: nch 64-bit keys rounded up to an even count, rank: nch
+// ints and wsum: SEL_THREADS / 32 ints of shared memory); writes the unit's
+// topk list to out.
+//   3b. rank of each chunk = the chunks that rank above it, counted by 1, 2
+//       or 4 lanes per chunk (as many as keep all chunks in one pass of the
+//       CTA where they can), two keys per shared-memory read; a chunk is
+//       selected iff its rank is below topk (every chunk when there are at
+//       most topk);
+//   4.  the selected chunks at their ascending-order positions: within a warp
+//       from a ballot, across warps from the warps' counts.
+__device__ __forceinline__ void select_from_scores(const float* score, unsigned long long* key, int* rank, int* wsum,
+                                                   int nch, int topk, int32_t* out) {
+  if (nch > topk) {
+    for (int c = threadIdx.x; c < ((nch + 1) & ~1); c += SEL_THREADS)
+      key[c] = c < nch ? rank_key(score[c], c) : 0ull;  // the padding key ranks above nothing
+    __syncthreads();
+    const int lpc = nch <= SEL_THREADS / 4 ? 4 : (nch <= SEL_THREADS / 2 ? 2 : 1);  // lanes per chunk
+    const int sub = threadIdx.x & (lpc - 1);
+    const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(key);
+    for (int base = 0; base < nch; base += SEL_THREADS / lpc) {
+      const int c = base + threadIdx.x / lpc;
+      const unsigned long long kc = key[min(c, nch - 1)];
+      int better = 0;
+      for (int o = sub; 2 * o < nch; o += lpc) {
+        const ulonglong2 v = k2[o];
+        better += (v.x > kc) + (v.y > kc);
+      }
+      if (lpc >= 2) better += __shfl_xor_sync(0xffffffffu, better, 1);
+      if (lpc == 4) better += __shfl_xor_sync(0xffffffffu, better, 2);
+      if (sub == 0 && c < nch) rank[c] = better;
+    }
+  } else {
+    for (int c = threadIdx.x; c < nch; c += SEL_THREADS) rank[c] = 0;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int carry = 0;  // chunks selected in earlier passes
+  for (int base = 0; base < nch; base += SEL_THREADS) {
+    const int c = base + threadIdx.x;
+    const bool sel = c < nch && rank[c] < topk;
+    const unsigned bal = __ballot_sync(0xffffffffu, sel);
+    if (lane == 0) wsum[warp] = __popc(bal);
+    __syncthreads();
+    int before = carry + __popc(bal & ((1u << lane) - 1u)), total = carry;
+    for (int w2 = 0; w2 < SEL_THREADS / 32; ++w2) {
+      const int v = wsum[w2];
+      before += w2 < warp ? v : 0;
+      total += v;
+    }
+    if (sel && before < topk) out[before] = c;
+    carry = total;
+    __syncthreads();  // wsum is written again by the next pass
+  }
+  for (int i = min(carry, topk) + threadIdx.x; i < topk; i += SEL_THREADS) out[i] = -1;
 }
 
 template <typename T>
@@ -131,10 +194,11 @@ __global__ void __launch_bounds__(SEL_THREADS)
   const int D = g.D;
   float* rowsum = sm;                       // [rpi][D] row-group sums
   float* qbar = rowsum + SEL_PART_FLOATS;   // [D]
-  float* kth = qbar + D;                    // {score, index as float bits}
-  float* score = kth + 4;                   // [nch_total rounded up to 4], 16-byte aligned
-  int* mark = reinterpret_cast<int*>(score + ((nch_total + 3) & ~3));  // [nch_total]
-  int* wsum = mark + nch_total;             // [warps + 1]
+  float* score = qbar + D;                  // [nch_total rounded up to 4]
+  unsigned long long* key =                 // [nch_total rounded up to 2], 16-byte aligned
+      reinterpret_cast<unsigned long long*>(score + ((nch_total + 3) & ~3));
+  int* rank = reinterpret_cast<int*>(key + ((nch_total + 1) & ~1));  // [nch_total]
+  int* wsum = rank + nch_total;             // [warps]
   // 1. the first pass's chunk means, loaded before anything else (rows below
   // nch_total always exist, whatever the prefix length), in flight with the
   // query loads.  Lane q4 of a chunk's four takes the float4s q4, q4 + 4, ...
@@ -205,70 +269,152 @@ __global__ void __launch_bounds__(SEL_THREADS)
     if (q4 == 0 && c < nch) score[c] = acc;
   }
   __syncthreads();
-  // 3b. ranks; the chunk of rank topk - 1 is the k-th best key (with at most
-  // topk valid chunks every chunk is selected)
-  if (nch > topk) {
-    // four lanes per chunk, each counting a quarter of the others (four
-    // scores per shared-memory read), then two shuffles
-    for (int base = 0; base < nch; base += CPP) {
-      const int c = base + (threadIdx.x >> 2);
-      const float sc = c < nch ? score[c] : 0.f;
-      int better = 0;
-      for (int c0 = 4 * q4; c0 < nch; c0 += 16) {
-        const float4 s4 = *reinterpret_cast<const float4*>(score + c0);  // (padded: see below)
-        better += (c0 < nch && ranks_above(s4.x, c0, sc, c)) + (c0 + 1 < nch && ranks_above(s4.y, c0 + 1, sc, c)) +
-                  (c0 + 2 < nch && ranks_above(s4.z, c0 + 2, sc, c)) + (c0 + 3 < nch && ranks_above(s4.w, c0 + 3, sc, c));
-      }
-      better += __shfl_xor_sync(0xffffffffu, better, 1);
-      better += __shfl_xor_sync(0xffffffffu, better, 2);
-      if (q4 == 0 && c < nch && better == topk - 1) {
-        kth[0] = sc;
-        kth[1] = __int_as_float(c);
-      }
-    }
-  }
-  __syncthreads();
-  const float ks = nch > topk ? kth[0] : CUDART_INF_F;
-  const int kc = nch > topk ? __float_as_int(kth[1]) : -1;
-  // 4. marks (chunk at or above the k-th key), then a block scan: the
-  // ascending-order position of each selected chunk
-  const int per = (nch + SEL_THREADS - 1) / SEL_THREADS;
-  const int f0 = min(nch, threadIdx.x * per), f1 = min(nch, f0 + per);
-  int cnt = 0;
-  for (int c = f0; c < f1; ++c) {
-    const int f = (nch <= topk) || !ranks_above(ks, kc, score[c], c);
-    mark[c] = f;
-    cnt += f;
-  }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) wsum[warp] = incl;
-  __syncthreads();
+  select_from_scores(score, key, rank, wsum, nch, topk, idx + ((size_t)b * g.Hkv + kvh) * topk);
+}
+
+// The same selection with every input of the unit in shared memory first:
+// warp 0 issues plain bulk copies of the unit's chunk means (one contiguous
+// nch_total x D block) and of its S x G query rows (one copy of G contiguous
+// heads per token), all completing on one mbarrier, so the unit's inputs
+// (2 x 64 KB in the batched sparse workload) cross HBM in one round trip
+// without the load/store unit.  Then
+//   2. column sums of the query rows (16-byte vectors in up to 32 row
+//      groups, added in a fixed order) into qbar,
+//   3a. scores, eight lanes per chunk (four chunks per warp and step),
+//   3b, 4. as in select_chunks_kernel.
+// D = 128.  Used when sel_bulk_smem_bytes fits and both sources are 16-byte
+// aligned.
+constexpr int SELB_D = 128;
+constexpr int SELB_GROUPS = 32;  // row groups of the column sums (at most)
+
+size_t sel_bulk_smem_bytes(int rows, int nch_total, size_t esz) {
+  // barrier (16), chunk means, query rows, row-group sums, qbar, every
+  // score (padded to 4), every key (padded to 2), one rank per chunk, warp
+  // totals
+  return 16 + (size_t)nch_total * SELB_D * 4 + (size_t)rows * SELB_D * esz +
+         (size_t)(SELB_GROUPS * SELB_D + SELB_D + ((nch_total + 3) & ~3)) * sizeof(float) +
+         (size_t)((nch_total + 1) & ~1) * 8 + (size_t)nch_total * sizeof(int) + (SEL_THREADS / 32) * sizeof(int);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(SEL_THREADS)
+    select_chunks_bulk_kernel(const CacheGeom g, const int32_t* lens, int chunk_size, int nch_total, int S, int Hq,
+                              int topk, const T* __restrict__ Q, const float* __restrict__ Kmean,
+                              int32_t* __restrict__ idx, int32_t* status) {
+  constexpr int D = SELB_D;
+  extern __shared__ __align__(16) uint8_t selb_raw[];
+  const int kvh = blockIdx.x;
+  const int b = blockIdx.y;
+  const int G = Hq / g.Hkv;
+  const int rows = S * G;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(selb_raw);
+  float* skm = reinterpret_cast<float*>(selb_raw + 16);      // [nch_total][D]
+  T* sq = reinterpret_cast<T*>(skm + (size_t)nch_total * D);  // [rows][D]
+  float* part = reinterpret_cast<float*>(sq + (size_t)rows * D);  // [SELB_GROUPS][D]
+  float* qbar = part + SELB_GROUPS * D;                       // [D]
+  float* score = qbar + D;                                    // [nch_total rounded up to 4]
+  unsigned long long* key =                                   // [nch_total rounded up to 2]
+      reinterpret_cast<unsigned long long*>(score + ((nch_total + 3) & ~3));
+  int* rank = reinterpret_cast<int*>(key + ((nch_total + 1) & ~1));  // [nch_total]
+  int* wsum = rank + nch_total;                               // [warps]
+  __shared__ int abort_flag;
   if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int w2 = 0; w2 < SEL_THREADS / 32; ++w2) {
-      const int v = wsum[w2];
-      wsum[w2] = acc;
-      acc += v;
-    }
-    wsum[SEL_THREADS / 32] = acc;
+    mbar_init(bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
   }
   __syncthreads();
-  int pos = wsum[warp] + incl - cnt;  // selected chunks before f0
-  int32_t* out = idx + ((size_t)b * g.Hkv + kvh) * topk;
-  for (int c = f0; c < f1; ++c) {
-    if (mark[c]) {
-      if (pos < topk) out[pos] = c;
-      ++pos;
+  // may start before the previous kernel in the stream has finished
+  pdl_wait();
+  pdl_launch_dependents();
+  const uint32_t qpiece = (uint32_t)(G * D * sizeof(T));
+  if (threadIdx.x < 32) {
+    // warp 0 issues the copies, the byte count first
+    const uint32_t kbytes = (uint32_t)nch_total * D * 4;
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(bar, kbytes + (uint32_t)S * qpiece);
+      bulk_load(skm, Kmean + ((size_t)b * g.Hkv + kvh) * nch_total * D, kbytes, bar);
+    }
+    __syncwarp();
+    for (int t = threadIdx.x; t < S; t += 32)
+      bulk_load(sq + (size_t)t * G * D, Q + (((size_t)b * S + t) * Hq + (size_t)kvh * G) * D, qpiece, bar);
+  }
+  int L = lens[b];
+  if (L < 0 || L > g.cap) {
+    if (threadIdx.x == 0) report(status, FB_ERR_BOUNDS);
+    L = max(0, min(L, g.cap));
+  }
+  const int nch = (L + chunk_size - 1) / chunk_size;
+  if (!bounded_wait(bar, 0, &abort_flag, status, false)) {
+    // the copies did not land in time (reported): wait once more, also
+    // bounded, before the CTA's shared memory is given up
+    bounded_wait(bar, 0, &abort_flag, nullptr, false);
+    return;
+  }
+  // 2. query mean: thread i sums the 16-byte vector i % VPR of rows i / VPR,
+  // + SEL_THREADS / VPR, ... (pairs of columns added as f32x2), then the row
+  // groups are added in a fixed order
+  {
+    constexpr int VEC = 16 / sizeof(T);  // columns per vector
+    constexpr int VPR = D / VEC;         // vectors per row
+    static_assert(SEL_THREADS / VPR <= SELB_GROUPS, "row groups");
+    const int vi = threadIdx.x % VPR;
+    const int rg = threadIdx.x / VPR;
+    float2 acc[VEC / 2];
+#pragma unroll
+    for (int k = 0; k < VEC / 2; ++k) acc[k] = make_float2(0.f, 0.f);
+#pragma unroll 4
+    for (int r = rg; r < rows; r += SEL_THREADS / VPR) {
+      const uint4 v = *reinterpret_cast<const uint4*>(sq + (size_t)r * D + vi * VEC);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      if constexpr (VEC == 8) {
+        // bf16 pair -> two floats: the low half shifted up, the high half masked
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          acc[k] = fadd2(acc[k], make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u)));
+      } else {
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          acc[k] = fadd2(acc[k], make_float2(__uint_as_float(w[2 * k]), __uint_as_float(w[2 * k + 1])));
+      }
+    }
+    float* dst = part + rg * D + vi * VEC;
+#pragma unroll
+    for (int k = 0; k < VEC / 2; ++k) *reinterpret_cast<float2*>(dst + 2 * k) = acc[k];
+  }
+  __syncthreads();
+  if (threadIdx.x < D) {
+    constexpr int NG = SEL_THREADS / (D / (16 / sizeof(T)));  // row groups written
+    float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int w2 = 0; w2 < NG; ++w2) a4[w2 & 3] += part[w2 * D + threadIdx.x];
+    qbar[threadIdx.x] = ((a4[0] + a4[1]) + (a4[2] + a4[3])) / (float)rows;
+  }
+  __syncthreads();
+  // 3a. scores: eight lanes per chunk, each a quarter-stride of float4s
+  {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int l8 = lane & 7;
+    const float4* q4p = reinterpret_cast<const float4*>(qbar);
+#pragma unroll 2
+    for (int base = 0; base < nch; base += SEL_THREADS / 8) {
+      const int c = base + warp * 4 + (lane >> 3);
+      const float4* kp = reinterpret_cast<const float4*>(skm + (size_t)min(c, nch_total - 1) * D);
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) {
+        const float4 q = q4p[l8 + 8 * i];
+        const float4 k = kp[l8 + 8 * i];
+        acc = fmaf(q.x, k.x, fmaf(q.y, k.y, fmaf(q.z, k.z, fmaf(q.w, k.w, acc))));
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      if (l8 == 0 && c < nch) score[c] = acc;
     }
   }
-  const int nsel = min(wsum[SEL_THREADS / 32], topk);
-  for (int i = nsel + threadIdx.x; i < topk; i += SEL_THREADS) out[i] = -1;
+  __syncthreads();
+  select_from_scores(score, key, rank, wsum, nch, topk, idx + ((size_t)b * g.Hkv + kvh) * topk);
 }
 
 // One thread per 16-byte vector of the block's K and V.
@@ -421,9 +567,33 @@ cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* K
                                  int32_t* status, cudaStream_t stream) {
   const CacheGeom g = geom_of(d);
   const int nch_total = (g.cap + d.chunk_size - 1) / d.chunk_size;
-  const size_t smem = sel_smem_bytes(g.D, nch_total);
   dim3 grid(g.Hkv, g.B);
   cudaError_t e;
+  // every input of a unit in shared memory, when it fits and the bulk copies'
+  // 16-byte alignment holds
+  const size_t esz = d.dtype == FB_BF16 ? 2 : 4;
+  const int rows = d.block_len * (d.num_q_heads / g.Hkv);
+  const size_t bulk_smem = sel_bulk_smem_bytes(rows, nch_total, esz);
+  const size_t bulk_tx = (size_t)nch_total * SELB_D * 4 + (size_t)rows * SELB_D * esz;
+  if (g.D == SELB_D && bulk_smem <= 220 * 1024 && bulk_tx < (1u << 20) &&
+      (reinterpret_cast<uintptr_t>(Q) & 15) == 0 && (reinterpret_cast<uintptr_t>(Kmean) & 15) == 0) {
+    if (d.dtype == FB_BF16) {
+      auto k = select_chunks_bulk_kernel<__nv_bfloat16>;
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bulk_smem);
+      if (e == cudaSuccess)
+        e = launch_pdl(k, grid, dim3(SEL_THREADS), bulk_smem, stream, g, d.prefix_lens, d.chunk_size, nch_total,
+                       d.block_len, d.num_q_heads, d.topk, static_cast<const __nv_bfloat16*>(Q), Kmean, idx, status);
+    } else {
+      auto k = select_chunks_bulk_kernel<float>;
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bulk_smem);
+      if (e == cudaSuccess)
+        e = launch_pdl(k, grid, dim3(SEL_THREADS), bulk_smem, stream, g, d.prefix_lens, d.chunk_size, nch_total,
+                       d.block_len, d.num_q_heads, d.topk, static_cast<const float*>(Q), Kmean, idx, status);
+    }
+    note_launch();
+    return e != cudaSuccess ? e : cudaGetLastError();
+  }
+  const size_t smem = sel_smem_bytes(g.D, nch_total);
   if (d.dtype == FB_BF16) {
     auto k = select_chunks_kernel<__nv_bfloat16>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -325,6 +325,57 @@ def _sparse_layer(prefix_len, chunk_size, topk, batch=2):
     return w, layer, Qt, Q64, K64, V64, lens.astype(np.int64)
 
 
+@pytest.mark.parametrize("dtype,cap,chunk_size,block,G,ties", [
+    ("bf16", 3000, 256, 32, 4, False),    # 12 chunk means and 128 query rows: staged in shared memory
+    ("fp32", 3000, 256, 32, 4, False),    # the same with fp32 queries
+    ("bf16", 2048, 128, 64, 8, False),    # 512 query rows (128 KB) beside the chunk means
+    ("bf16", 9000, 128, 32, 4, True),     # 71 chunks, 30 of them with one mean: the tie goes to lower indices
+    ("bf16", 33000, 128, 32, 4, True),    # 258 chunks: two lanes per chunk in the rank count
+    ("bf16", 70000, 128, 32, 4, False),   # 547 chunk means (274 KB) do not fit: the kernel that streams them
+    ("bf16", 70000, 128, 32, 4, True),
+])
+def test_chunk_selection_kernels(dtype, cap, chunk_size, block, G, ties):
+    # fb_select_chunks on given chunk means (no cache needed) against the
+    # oracle's top-k of qbar . kbar_c; two lengths per batch leave chunks past
+    # the prefix that must not be chosen
+    rng = np.random.default_rng(cap + block)
+    B, Hkv, D, topk = 2, 2, 128, 16
+    Hq = Hkv * G
+    nch_total = -(-cap // chunk_size)
+    lens = np.array([cap - 5, cap // 2 + 7], np.int32)
+    valid = np.arange(nch_total)[None, :] * chunk_size < lens[:, None]
+    Km = rng.standard_normal((B, Hkv, nch_total, D)).astype(np.float32)
+    if ties:
+        # every second of the first 40 chunks carries the same mean, well
+        # above the others: equal scores in both float32 and float64, more
+        # of them (inside both prefixes) than topk, so the top-k boundary
+        # falls inside the tie
+        Km *= np.float32(0.01)
+        Km[:, :, 0:40:2, :] = rng.standard_normal((B, Hkv, 1, D)).astype(np.float32)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    Qm = rng.standard_normal((B, block, Hq, D)).astype(np.float32)
+    if ties:
+        Qm += 2 * Km[:, :, :1, :].repeat(G, axis=1).transpose(0, 2, 1, 3)  # qbar along the tied mean: a high score
+    Qt = torch.from_numpy(Qm).to(tdt).cuda()
+    lens_t = torch.from_numpy(lens).cuda()
+    d = fbl.make_desc(B, Hq, Hkv, D, block, fbl.FB_BF16 if dtype == "bf16" else fbl.FB_FP32, kv_capacity=cap,
+                      prefix_lens=lens_t, chunk_size=chunk_size, topk=topk)
+    idx = torch.full((B, Hkv, topk), -7, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fbl.fb_select_chunks(d, Qt, torch.from_numpy(Km).cuda(), idx, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    Q64 = Qt.float().cpu().numpy().astype(np.float64)
+    ref = ora.select_chunks(Q64, Km.astype(np.float64), valid, topk)
+    if ties:
+        # the tie decides: all of the oracle's picks come from the tied chunks
+        sc = ora.chunk_scores(Q64, Km.astype(np.float64), valid)
+        for b in range(B):
+            for h in range(Hkv):
+                assert len(set(sc[b, h, ref[b, h]].tolist())) == 1
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
 def test_sparse_chunk_lists_longer_than_a_warp():
     # 40-entry chunk lists (two 32-entry steps of the list scan), hand-made
     # with gaps, against the oracle's prefix partial over the same chunks
