@@ -45,16 +45,16 @@ sys.path.insert(0, ROOT)
 METRIC = "attention µs/denoise-step and tokens/s, cached vs uncached; prefix-pass HBM GB/s"
 
 # DRAM bytes read + written by one launch of the prefix-pass attention kernel,
-# from one `ncu --set full --clock-control none` capture of that launch on the
-# workload (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the
+# from one `ncu --clock-control none` capture of that launch on the workload
+# (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the
 # kernel sources it was captured on (see kernel_source_hash).  An entry whose
 # hash differs from the built sources is not reported: the kernel changed
 # since the counters were taken.
 NCU_TRAFFIC = {
-    # profiles/prefix_pass_long_ctx.md, capture b16_prof_lc
-    "long_ctx": {"bytes": 537205760 + 3928320, "sources": "3d596fe3a1abc379"},
+    # profiles/prefix_pass_long_ctx.md, capture b30_traffic_lc
+    "long_ctx": {"bytes": 537209600 + 3059712, "sources": "141a69f6f5809b93"},
 }
-KERNEL_SOURCES = ("fb_attn_tc.cu", "fb_ptx.cuh", "fb_internal.h", "fb_api.cu")
+KERNEL_SOURCES = ("fb_attn_tc.cu", "fb_attn_common.cuh", "fb_ptx.cuh", "fb_internal.h", "fb_api.cu")
 
 
 def kernel_source_hash():
