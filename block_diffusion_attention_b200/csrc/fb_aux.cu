@@ -14,6 +14,8 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <atomic>
+
 #include "fb_attn_common.cuh"
 #include "fb_internal.h"
 #include "fb_ptx.cuh"
@@ -573,23 +575,33 @@ cudaError_t launch_select_chunks(const fb_desc& d, const void* Q, const float* K
   // 16-byte alignment holds
   const size_t esz = d.dtype == FB_BF16 ? 2 : 4;
   const int rows = d.block_len * (d.num_q_heads / g.Hkv);
+  constexpr size_t BULK_SMEM_MAX = 220 * 1024;
   const size_t bulk_smem = sel_bulk_smem_bytes(rows, nch_total, esz);
   const size_t bulk_tx = (size_t)nch_total * SELB_D * 4 + (size_t)rows * SELB_D * esz;
-  if (g.D == SELB_D && bulk_smem <= 220 * 1024 && bulk_tx < (1u << 20) &&
+  if (g.D == SELB_D && bulk_smem <= BULK_SMEM_MAX && bulk_tx < (1u << 20) &&
       (reinterpret_cast<uintptr_t>(Q) & 15) == 0 && (reinterpret_cast<uintptr_t>(Kmean) & 15) == 0) {
-    if (d.dtype == FB_BF16) {
-      auto k = select_chunks_bulk_kernel<__nv_bfloat16>;
-      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bulk_smem);
-      if (e == cudaSuccess)
-        e = launch_pdl(k, grid, dim3(SEL_THREADS), bulk_smem, stream, g, d.prefix_lens, d.chunk_size, nch_total,
-                       d.block_len, d.num_q_heads, d.topk, static_cast<const __nv_bfloat16*>(Q), Kmean, idx, status);
-    } else {
-      auto k = select_chunks_bulk_kernel<float>;
-      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bulk_smem);
-      if (e == cudaSuccess)
-        e = launch_pdl(k, grid, dim3(SEL_THREADS), bulk_smem, stream, g, d.prefix_lens, d.chunk_size, nch_total,
-                       d.block_len, d.num_q_heads, d.topk, static_cast<const float*>(Q), Kmean, idx, status);
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    // the shared-memory limit of the bulk kernels, raised once per device
+    static std::atomic<bool> configured[64][2];
+    const int which = d.dtype == FB_BF16 ? 0 : 1;
+    void (*kb)(CacheGeom, const int32_t*, int, int, int, int, int, const __nv_bfloat16*, const float*, int32_t*,
+               int32_t*) = select_chunks_bulk_kernel<__nv_bfloat16>;
+    void (*kf)(CacheGeom, const int32_t*, int, int, int, int, int, const float*, const float*, int32_t*,
+               int32_t*) = select_chunks_bulk_kernel<float>;
+    if (dev >= 64 || !configured[dev][which].load(std::memory_order_acquire)) {
+      e = which == 0 ? cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BULK_SMEM_MAX)
+                     : cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BULK_SMEM_MAX);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) configured[dev][which].store(true, std::memory_order_release);
     }
+    if (which == 0)
+      e = launch_pdl(kb, grid, dim3(SEL_THREADS), bulk_smem, stream, g, d.prefix_lens, d.chunk_size, nch_total,
+                     d.block_len, d.num_q_heads, d.topk, static_cast<const __nv_bfloat16*>(Q), Kmean, idx, status);
+    else
+      e = launch_pdl(kf, grid, dim3(SEL_THREADS), bulk_smem, stream, g, d.prefix_lens, d.chunk_size, nch_total,
+                     d.block_len, d.num_q_heads, d.topk, static_cast<const float*>(Q), Kmean, idx, status);
     note_launch();
     return e != cudaSuccess ? e : cudaGetLastError();
   }
