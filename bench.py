@@ -557,6 +557,20 @@ def run_ours(args):
         torch.cuda.synchronize()
         res["pre_cold_ms"] = [a.elapsed_time(c) for a, c in cold]
         del flush
+    if not policy:
+        # The method's reuse error on these synthetic inputs (outside every
+        # timed region): per denoising step, the relative distance of the
+        # cached output from the uncached one, both from this library.
+        errs = []
+        for s_ in range(w.steps):
+            Q, Kb, Vb = dev_in[s_]
+            if s_ in w.refresh:
+                cached.select(Q)
+                cached.prefix(Q)
+            oc = cached.step(Q, Kb, Vb).float()
+            of = cached.full(Q, Kb, Vb).float()
+            errs.append(float((oc - of).norm() / of.norm()))
+        res["reuse_err"] = errs
     cached.check()
     del cached
 
@@ -759,6 +773,12 @@ def report(args, w0, w, world, res):
         "prefix_hbm_frac_l2_cold": (abytes / (cold_us * 1e-6) / 1e9 / hbm_peak) if cold_us else None,
         "roofline": roof,
         "clocks": res["clocks"],
+        "reuse_error": ({"per_denoise_step": res["reuse_err"], "refresh_steps": list(w.refresh),
+                         "definition": "||O_cached - O_uncached||_F / ||O_uncached||_F of one block, both outputs "
+                                       "from this library; refresh steps show bf16 rounding (plus, for top-k "
+                                       "workloads, the sparse selection's own error), reuse steps the method's "
+                                       "approximation under the synthetic per-step drift"}
+                        if "reuse_err" in res else None),
         "e2e": ({"value": tps(res["ms_e2e"]), "unit": "tokens/s", "h2d_bytes_per_step": res["h2d"],
                  "d2h_bytes_per_step": res["d2h"], "ms_per_step": res["ms_e2e"] / args.steps,
                  **({"h2d_ms_per_step_alone": res["h2d_ms"], "d2h_ms_per_step_alone": res["d2h_ms"],
