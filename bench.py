@@ -151,6 +151,18 @@ def prefix_flops(w, lens, residual=False):
     return 4.0 * w.num_q_heads * w.block_len * eff * w.head_dim
 
 
+def prefix_kernel_name(w):
+    """The kernel that runs the workload's prefix pass, as the library picks
+    it: fp32 on the CUDA cores; bf16 on the tensor cores with two 128-row
+    query tiles per CTA where a (b, kv head) unit has at least two
+    (S x G packed rows), else one."""
+    if w.dtype != "bf16":
+        return "prefix pass: attn_simt_kernel (fp32, CUDA cores)"
+    tiles = -(-(w.block_len * w.group) // 128)
+    kern = "attn_tc2_kernel<EPI_PARTIAL>" if tiles >= 2 else "attn_tc_kernel<EPI_PARTIAL>"
+    return f"prefix pass: {kern} (+ combine_kernel when the keys are split)"
+
+
 def measured_peaks():
     """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, source)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -746,7 +758,7 @@ def report(args, w0, w, world, res):
     traffic = None if args.residual else recorded_traffic(w.name)
     roof.update({"traffic": traffic,
                  "traffic_over_algorithmic": (traffic / abytes) if traffic else None,
-                 "kernel": "prefix pass: attn_tc_kernel<EPI_PARTIAL> (+ combine_kernel when split)",
+                 "kernel": prefix_kernel_name(w),
                  "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": pflops,
                  "intensity_flop_per_byte": intensity})
     ms_c = res["ms_cached"]
