@@ -393,7 +393,8 @@ __global__ void __launch_bounds__(SEL_THREADS)
     qbar[threadIdx.x] = ((a4[0] + a4[1]) + (a4[2] + a4[3])) / (float)rows;
   }
   __syncthreads();
-  // 3a. scores: eight lanes per chunk, each a quarter-stride of float4s
+  // 3a. scores: eight lanes per chunk (lane l8 takes every eighth float4 of
+  // the chunk's mean, starting at l8), four chunks per warp and pass
   {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int l8 = lane & 7;
