@@ -177,6 +177,20 @@ long long cta_units(const fb_desc& d) {
   return (long long)d.batch * d.num_kv_heads * (use_pairs(d) ? (rt + 1) / 2 : rt);
 }
 
+// Tail split of the two-tile kernel.  Unsplit, the grid's last wave can be
+// nearly empty: 760 tile pairs at the video shape are five full waves of 148
+// and one of 20, so a sixth of the pass runs on 20 SMs.  Where that last wave
+// holds at most half the SMs, its units can be split k ways over their keys
+// instead (k about SMs / tail units, at least 3 key tiles per split, at most
+// 32 splits), into slots the combine merges, while the other units keep one
+// CTA each.  tail_splits gives that k (0: no tail split).
+long long tail_splits(long long units, long long slots, long long est_tiles) {
+  const long long tail = units % slots;
+  if (units <= slots || tail == 0 || 2 * tail > slots) return 0;
+  const long long k = std::min<long long>(slots / tail, std::min<long long>(est_tiles / 3, 32));
+  return k >= 2 ? k : 0;
+}
+
 // Key-range splits of the prefix pass.  Cost model in key-tile times: every
 // wave of CTAs costs its longest split plus a fixed per-CTA overhead (set-up,
 // pipeline fill, epilogue ~ 3 tiles), and splitting adds a combine pass
@@ -206,6 +220,16 @@ int choose_splits(const fb_desc& d, long long est_tiles) {
       best = (int)ns;
     }
   }
+  // One split with the tail split (see tail_plan) where that is cheaper: the
+  // full waves of unsplit units, then the tail units' splits, then the combine.
+  if (use_pairs(d)) {
+    const long long k = tail_splits(units, slots, est_tiles);
+    if (k > 0) {
+      const double cost = (double)(units / slots) * ((double)est_tiles + 3.0) +
+                          (std::ceil((double)est_tiles / (double)k) + 3.0) + 2.0;
+      if (cost < best_cost - 1e-9) return 1;
+    }
+  }
   return best;
 }
 
@@ -225,6 +249,32 @@ size_t split_bytes(const fb_desc& d, int ns) {
   if (ns <= 1) return 0;
   const size_t rows = (size_t)d.batch * d.block_len * d.num_q_heads;
   return (size_t)ns * rows * (size_t)(d.head_dim + 1) * sizeof(float);
+}
+
+// The tail split of a pass planned with one split (choose_splits), where it
+// applies: two-tile units, no explicit split count.
+struct TailPlan {
+  int u0 = 0;     // first tail unit
+  int units = 0;  // tail units
+  int k = 0;      // splits per tail unit (0: no tail split)
+};
+
+TailPlan tail_plan(const fb_desc& d, int ns, long long est_tiles) {
+  TailPlan t;
+  if (ns != 1 || !use_pairs(d) || d.num_splits > 0) return t;
+  const long long units = cta_units(d);
+  const long long slots = device_sms();
+  const long long k = tail_splits(units, slots, est_tiles);
+  if (k == 0) return t;
+  t.u0 = (int)(units - units % slots);
+  t.units = (int)(units % slots);
+  t.k = (int)k;
+  return t;
+}
+
+// Slots of the tail splits: (tail unit, split, tile) x 128 rows x (D + 1) f32.
+size_t tail_bytes(const TailPlan& t) {
+  return (size_t)t.units * t.k * 2 * TC_BM * (TC_D + 1) * sizeof(float);
 }
 
 fb_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FB_OK : FB_ERR_LAUNCH; }
@@ -305,9 +355,12 @@ size_t fb_workspace_bytes(const fb_desc* d) {
   const int ns_pre = choose_splits(*d, prefix_tiles_estimate(*d));
   fb_desc dense = *d;
   dense.topk = 0;
-  const int ns_full = choose_splits(dense, prefix_tiles_estimate(dense) + (d->block_len + TC_BN - 1) / TC_BN);
+  const long long est_full = prefix_tiles_estimate(dense) + (d->block_len + TC_BN - 1) / TC_BN;
+  const int ns_full = choose_splits(dense, est_full);
   size_t need = split_bytes(*d, ns_pre);
+  need = std::max(need, tail_bytes(tail_plan(*d, ns_pre, prefix_tiles_estimate(*d))));
   need = std::max(need, split_bytes(*d, ns_full));
+  need = std::max(need, tail_bytes(tail_plan(dense, ns_full, est_full)));
   need = std::max(need, threshold_ws_bytes(*d));
   if (d->dtype == FB_BF16 && !use_pairs(*d)) {
     // the masked prefix pass's active-unit slots
@@ -381,6 +434,43 @@ fb_status prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const 
     c.n_rt = p.n_rt;
     return from_cuda(launch_combine(c, s));
   }
+  // the tail split where the workspace holds its slots (else the plain plan)
+  const TailPlan tp = pairs ? tail_plan(*d, ns, prefix_tiles_estimate(*d)) : TailPlan{};
+  if (tp.k > 0 && ws && ws_bytes >= tail_bytes(tp) && aligned16(ws)) {
+    const int slots = tp.units * tp.k * 2;
+    float* tail_o = static_cast<float*>(ws);
+    float* tail_l = tail_o + (size_t)slots * TC_BM * TC_D;
+    p.nsplit = 1;
+    p.tail_u0 = tp.u0;
+    p.tail_k = tp.k;
+    p.tail_o = tail_o;
+    p.tail_lse = tail_l;
+    p.out_o32 = O_pre;
+    p.out_lse = LSE_pre;
+    p.kv_stream_once = (p.n_rt <= 2);
+    CUtensorMap tm_out, tm_tail;
+    if (!pre_map(&tm_out, *d, O_pre, d->batch) || !slot_map(&tm_tail, *d, tail_o, slots)) return FB_ERR_LAUNCH;
+    cudaError_t e = launch_attn_tc2(p, m.q, m.kp, m.vp, m.kp, m.vp, tm_out, tm_tail, tp.u0 + tp.units * tp.k, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    CombineParams c;
+    std::memset(&c, 0, sizeof(c));
+    c.B = d->batch;
+    c.Hq = d->num_q_heads;
+    c.S = d->block_len;
+    c.D = d->head_dim;
+    c.part_o = tail_o;
+    c.part_lse = tail_l;
+    c.out_o32 = O_pre;
+    c.out_lse = LSE_pre;
+    c.G = p.G;
+    c.unit_mask = unit_mask;
+    c.tail_k = tp.k;
+    c.tail_u0 = tp.u0;
+    c.tail_units = tp.units;
+    c.npair = (p.n_rt + 1) / 2;
+    c.Hkv = d->num_kv_heads;
+    return from_cuda(launch_combine(c, s));
+  }
   p.nsplit = ns;
   float* part_o = O_pre;
   float* part_l = LSE_pre;
@@ -395,7 +485,7 @@ fb_status prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const 
   cudaError_t e;
   if (pairs) {
     p.kv_stream_once = (p.n_rt <= 2);  // one tile pair per unit: each K/V byte is read once
-    e = launch_attn_tc2(p, m.q, m.kp, m.vp, m.kp, m.vp, tm_out, (int)grid, s);
+    e = launch_attn_tc2(p, m.q, m.kp, m.vp, m.kp, m.vp, tm_out, tm_out, (int)grid, s);
   } else {
     e = launch_attn_tc(p, m.q, m.kp, m.vp, m.kp, m.vp, m.q, tm_out, (int)grid, s);
   }
@@ -494,7 +584,7 @@ fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const v
   const long long grid = cta_units(*d);
   if (use_pairs(*d)) {
     p.kv_stream_once = (p.n_rt <= 2);
-    return from_cuda(launch_attn_tc2(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_out, (int)grid, s));
+    return from_cuda(launch_attn_tc2(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_out, tm_out, (int)grid, s));
   }
   return from_cuda(launch_attn_tc(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_pre, tm_out, (int)grid, s));
 }
@@ -556,7 +646,8 @@ fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc,
                                       static_cast<const float*>(Vc), static_cast<const float*>(Kb),
                                       static_cast<const float*>(Vb), s));
   }
-  const int ns = choose_splits(dense, prefix_tiles_estimate(dense) + (d->block_len + TC_BN - 1) / TC_BN);
+  const long long est = prefix_tiles_estimate(dense) + (d->block_len + TC_BN - 1) / TC_BN;
+  const int ns = choose_splits(dense, est);
   const size_t need = split_bytes(dense, ns);
   if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return FB_ERR_WORKSPACE;
   Maps m;
@@ -572,7 +663,40 @@ fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc,
     p.out_lse = LSE_out;
     CUtensorMap tm_out;
     if (!q_map(&tm_out, dense, O)) return FB_ERR_LAUNCH;
-    if (pairs) return from_cuda(launch_attn_tc2(p, m.q, m.kp, m.vp, m.kb, m.vb, tm_out, (int)units, s));
+    // the tail split (see tail_plan) where the workspace holds its slots
+    const TailPlan tp = pairs ? tail_plan(dense, ns, est) : TailPlan{};
+    if (tp.k > 0 && ws && ws_bytes >= tail_bytes(tp) && aligned16(ws)) {
+      const int slots = tp.units * tp.k * 2;
+      float* tail_o = static_cast<float*>(ws);
+      float* tail_l = tail_o + (size_t)slots * TC_BM * TC_D;
+      p.tail_u0 = tp.u0;
+      p.tail_k = tp.k;
+      p.tail_o = tail_o;
+      p.tail_lse = tail_l;
+      CUtensorMap tm_tail;
+      if (!slot_map(&tm_tail, dense, tail_o, slots)) return FB_ERR_LAUNCH;
+      cudaError_t e = launch_attn_tc2(p, m.q, m.kp, m.vp, m.kb, m.vb, tm_out, tm_tail, tp.u0 + tp.units * tp.k, s);
+      if (e != cudaSuccess) return from_cuda(e);
+      CombineParams c;
+      std::memset(&c, 0, sizeof(c));
+      c.B = d->batch;
+      c.Hq = d->num_q_heads;
+      c.S = d->block_len;
+      c.D = d->head_dim;
+      c.part_o = tail_o;
+      c.part_lse = tail_l;
+      c.out_o = O;
+      c.out_bf16 = 1;
+      c.out_lse = LSE_out;
+      c.G = p.G;
+      c.tail_k = tp.k;
+      c.tail_u0 = tp.u0;
+      c.tail_units = tp.units;
+      c.npair = (p.n_rt + 1) / 2;
+      c.Hkv = d->num_kv_heads;
+      return from_cuda(launch_combine(c, s));
+    }
+    if (pairs) return from_cuda(launch_attn_tc2(p, m.q, m.kp, m.vp, m.kb, m.vb, tm_out, tm_out, (int)units, s));
     return from_cuda(launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, tm_out, (int)units, s));
   }
   p.epi = EPI_PARTIAL;
@@ -583,7 +707,7 @@ fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc,
   p.out_lse = part_l;
   CUtensorMap tm_out;
   if (!pre_map(&tm_out, dense, part_o, d->batch * ns)) return FB_ERR_LAUNCH;
-  cudaError_t e = pairs ? launch_attn_tc2(p, m.q, m.kp, m.vp, m.kb, m.vb, tm_out, (int)(units * ns), s)
+  cudaError_t e = pairs ? launch_attn_tc2(p, m.q, m.kp, m.vp, m.kb, m.vb, tm_out, tm_out, (int)(units * ns), s)
                         : launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, tm_out, (int)(units * ns), s);
   if (e != cudaSuccess) return from_cuda(e);
   CombineParams c;

@@ -153,6 +153,9 @@ __global__ void __launch_bounds__(WARPS * 32)
 #pragma unroll
     for (int k = 0; k < MAXD / 32; ++k) o[k] *= alpha;
     const int nk = min(32, ntot - base);
+    // (unrolled: the value rows' loads are in flight together; the sums keep
+    // their order)
+#pragma unroll 8
     for (int jj = 0; jj < nk; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, pz, jj);
       bool blk;

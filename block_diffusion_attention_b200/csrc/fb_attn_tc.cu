@@ -625,8 +625,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
 // Log-space merge of the split-key partials of one query row (the merge
 // equation applied across splits, in a fixed order).  One warp per row: lanes
-// read the splits' LSEs in parallel, the split weights go to shared memory,
-// then each lane accumulates four output columns over the splits.
+// read the splits' LSEs in parallel, then each lane accumulates four output
+// columns over the splits.  The partials come in one of three layouts: one
+// [B][S][Hq] set per split, the active-unit slots (CombineParams::dyn), or
+// the tail slots of the two-tile kernel (CombineParams::tail_k, only the
+// tail units' rows).
 constexpr int CMB_WARPS = 4;
 constexpr int CMB_INFLIGHT = 16;  // split loads in flight per lane (divides 32)
 static_assert(TC_MAX_SPLITS == 128, "combine holds four split weights per lane");
@@ -646,22 +649,51 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombinePa
   pdl_wait();
   pdl_launch_dependents();
   const int wi = threadIdx.x >> 5;
-  const long long row = (long long)blockIdx.x * CMB_WARPS + wi;
+  long long row = (long long)blockIdx.x * CMB_WARPS + wi;
   const int lane = threadIdx.x & 31;
   const long long nrows = (long long)c.B * c.S * c.Hq;
-  if (row >= nrows) return;
-  const int h = (int)(row % c.Hq);
-  const long long bt = row / c.Hq;
-  const int t = (int)(bt % c.S);
-  const int b = (int)(bt / c.S);
-  size_t so = (size_t)nrows * c.D;              // split stride of the partial O
-  size_t sl = (size_t)c.B * c.Hq * c.S;         // split stride of the partial LSE
+  int h, t, b;
+  const float* base;
+  const float* lbase;
+  size_t so, sl;  // split strides of the partial O and LSE
+  int nsplit;
+  if (c.tail_k > 0) {
+    // the tail units' rows (two tiles of 128 packed rows per unit) from the
+    // slots (tail unit, split, tile) of the two-tile kernel's tail splits
+    if (row >= (long long)c.tail_units * 2 * TC_BM) return;
+    const int ti = (int)(row / (2 * TC_BM));
+    const int rr = (int)(row % (2 * TC_BM));
+    long long u = (long long)c.tail_u0 + ti;
+    const int pair = (int)(u % c.npair);
+    u /= c.npair;
+    const int kvh = (int)(u % c.Hkv);
+    b = (int)(u / c.Hkv);
+    const int pr = pair * 2 * TC_BM + rr;  // packed query row of the unit
+    if (pr >= c.S * c.G) return;
+    t = pr / c.G;
+    h = kvh * c.G + pr % c.G;
+    row = ((long long)b * c.S + t) * c.Hq + h;
+    const size_t slot0 = (size_t)ti * c.tail_k * 2 + rr / TC_BM;
+    base = c.part_o + (slot0 * TC_BM + rr % TC_BM) * c.D;
+    lbase = c.part_lse + slot0 * TC_BM + rr % TC_BM;
+    so = (size_t)2 * TC_BM * c.D;
+    sl = 2 * TC_BM;
+    nsplit = c.tail_k;
+  } else {
+    if (row >= nrows) return;
+    h = (int)(row % c.Hq);
+    const long long bt = row / c.Hq;
+    t = (int)(bt % c.S);
+    b = (int)(bt / c.S);
+    base = c.part_o + row * c.D;
+    lbase = c.part_lse + ((size_t)b * c.Hq + h) * c.S + t;
+    so = (size_t)nrows * c.D;
+    sl = (size_t)c.B * c.Hq * c.S;
+    nsplit = c.nsplit;
+  }
   const size_t lrow = ((size_t)b * c.Hq + h) * c.S + t;
   const int unit = b * (c.Hq / c.G) + h / c.G;
   if (c.unit_mask && c.unit_mask[unit] == 0) return;  // unit not refreshed
-  int nsplit = c.nsplit;
-  const float* base = c.part_o + row * c.D;
-  const float* lbase = c.part_lse + lrow;
   if (c.dyn) {
     // active-unit slots: (rank of the unit, query tile, split) -> [128][D] rows
     const int na = active_count(c.unit_mask, c.B * (c.Hq / c.G));
@@ -815,7 +847,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, const CUtensorMap& tmQ, const CU
 }
 
 cudaError_t launch_combine(const CombineParams& c, cudaStream_t stream) {
-  const long long rows = (long long)c.B * c.S * c.Hq;
+  const long long rows = c.tail_k > 0 ? (long long)c.tail_units * 2 * TC_BM : (long long)c.B * c.S * c.Hq;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((rows + CMB_WARPS - 1) / CMB_WARPS));
   cfg.blockDim = dim3(CMB_WARPS * 32);

@@ -49,6 +49,11 @@
 // The epilogue of tile X stages its output in Q_X's region (every QK^T is
 // done once the last PV_X is).
 //
+// A prefix pass (or an uncached pass) whose last wave of CTAs is only partly
+// full may split the keys of those last units (AttnParams::tail_k): such a
+// CTA writes f32 partial rows to its tiles' slots through the second output
+// map, and the combine merges them.
+//
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // FB_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
 #include <cuda_bf16.h>
@@ -101,6 +106,7 @@ struct Work2 {
   int b, kvh, rtA, hasB, split, skip, j0, nt;
   int n0, n1, L;        // UnitTiles of the unit
   int list_in_smem;     // sparse chunk list copied to Shared2::clist
+  int tail;             // index of a tail split CTA (AttnParams::tail_k), else -1
   uint32_t tmem;        // tensor-memory base
 };
 constexpr uint32_t OFF_WORK2 = 160;  // inside the barrier area, after the barriers
@@ -135,6 +141,7 @@ __device__ __forceinline__ Work2 load_work2(uint8_t* smem) {
   Work2 r;
   r.b = w->b; r.kvh = w->kvh; r.rtA = w->rtA; r.hasB = w->hasB; r.split = w->split; r.skip = w->skip;
   r.j0 = w->j0; r.nt = w->nt; r.n0 = w->n0; r.n1 = w->n1; r.L = w->L; r.list_in_smem = w->list_in_smem;
+  r.tail = w->tail;
   r.tmem = w->tmem;
   return r;
 }
@@ -338,7 +345,8 @@ __device__ __forceinline__ void mma_role(const AttnParams& p) {
 // ------------------------------------------------------ softmax + epilogue
 // Warpgroup x (0: tile A, 1: tile B); thread r owns query row r (TMEM lane r).
 template <int EPI>
-__device__ __forceinline__ void softmax_role(const CUtensorMap* tmO, const AttnParams& p, int x) {
+__device__ __forceinline__ void softmax_role(const CUtensorMap* tmO, const CUtensorMap* tmT, const AttnParams& p,
+                                             int x) {
   constexpr int NC = BN;
   uint8_t* smem = smem_base2();
   const Shared2 sh = shared2(smem);
@@ -472,8 +480,9 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tmO, const AttnP
   const uint32_t st_row = smem_u32(stage) + r * 128;
   const int t0 = rt * (BM / p.G);
   const bool store = ok && t0 < p.S;  // rows of this tile exist
-  if (EPI == EPI_PARTIAL) {
+  if (EPI == EPI_PARTIAL || (EPI == EPI_NORM && w.tail >= 0)) {
     // the f32 tile (64 KB) in two rounds of 64 columns through the 32 KB stage
+    // (a tail split of the uncached pass writes its partial rows the same way)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       if (ok) {
@@ -493,14 +502,22 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tmO, const AttnP
       named_bar_sync(1 + x, 4 * 32);
       if (r == 0 && store && !*sh.abort_flag) {
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc)
-          tma_store_4d(tmO, stage + cc * (BM * 128), (2 * hf + cc) * 32, w.kvh * p.G, t0, w.split * p.B + w.b);
+        for (int cc = 0; cc < 2; ++cc) {
+          if (w.tail >= 0)  // a tail split: the tile's slot of tail_o
+            tma_store_4d(tmT, stage + cc * (BM * 128), (2 * hf + cc) * 32, 0, 0, 2 * w.tail + x);
+          else
+            tma_store_4d(tmO, stage + cc * (BM * 128), (2 * hf + cc) * 32, w.kvh * p.G, t0, w.split * p.B + w.b);
+        }
         tma_store_commit();
         tma_store_wait_read();
       }
       named_bar_sync(1 + x, 4 * 32);  // the stage may be written again
     }
-    if (row_ok) p.out_lse[(((size_t)w.split * p.B + w.b) * p.Hq + h) * p.S + tok] = lse2 * LN2;
+    if (w.tail >= 0) {
+      if (ok) p.tail_lse[(size_t)(2 * w.tail + x) * BM + r] = lse2 * LN2;  // slot layout: every row
+    } else if (row_ok) {
+      p.out_lse[(((size_t)w.split * p.B + w.b) * p.Hq + h) * p.S + tok] = lse2 * LN2;
+    }
   } else {
     const size_t orow = ((size_t)w.b * p.S + tok) * p.Hq + h;
     float wp = 0.f, wo = inv_l, inv_den = 1.f, lse_out2 = lse2;
@@ -560,7 +577,7 @@ __global__ void __launch_bounds__(THREADS2, 1)
     attn_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKp,
                     const __grid_constant__ CUtensorMap tmVp, const __grid_constant__ CUtensorMap tmKb,
                     const __grid_constant__ CUtensorMap tmVb, const __grid_constant__ CUtensorMap tmO,
-                    const AttnParams p) {
+                    const __grid_constant__ CUtensorMap tmT, const AttnParams p) {
   uint8_t* smem = smem_base2();
   const Shared2 sh = shared2(smem);
   const int warp = threadIdx.x >> 5;
@@ -593,13 +610,23 @@ __global__ void __launch_bounds__(THREADS2, 1)
     tma_prefetch_map(&tmKb);
     tma_prefetch_map(&tmVb);
     tma_prefetch_map(&tmO);
+    if (p.tail_k > 0) tma_prefetch_map(&tmT);
   }
   {
     // This CTA's (b, kv head, query-tile pair, key split) from its grid index.
     const int npair = (p.n_rt + 1) >> 1;
     unsigned bid = blockIdx.x;
-    const int split = (int)(bid % (unsigned)p.nsplit);
-    bid /= (unsigned)p.nsplit;
+    int split, nsplit = p.nsplit, tail = -1;
+    if (p.tail_k > 0 && bid >= (unsigned)p.tail_u0) {
+      // a key split of one of the last units (the tail wave)
+      tail = (int)(bid - (unsigned)p.tail_u0);
+      split = tail % p.tail_k;
+      nsplit = p.tail_k;
+      bid = (unsigned)p.tail_u0 + (unsigned)(tail / p.tail_k);
+    } else {
+      split = (int)(bid % (unsigned)p.nsplit);
+      bid /= (unsigned)p.nsplit;
+    }
     const int pair = (int)(bid % (unsigned)npair);
     bid /= (unsigned)npair;
     const int kvh = (int)(bid % (unsigned)p.Hkv);
@@ -629,14 +656,15 @@ __global__ void __launch_bounds__(THREADS2, 1)
       wk->split = split;
       wk->skip = skip;
       // split * ntot < 2^7 * 2^23: 32-bit arithmetic is exact
-      const int j0 = (int)(((unsigned)split * (unsigned)ntot) / (unsigned)p.nsplit);
-      const int j1 = (int)(((unsigned)(split + 1) * (unsigned)ntot) / (unsigned)p.nsplit);
+      const int j0 = (int)(((unsigned)split * (unsigned)ntot) / (unsigned)nsplit);
+      const int j1 = (int)(((unsigned)(split + 1) * (unsigned)ntot) / (unsigned)nsplit);
       wk->j0 = j0;
       wk->nt = j1 - j0;
       wk->n0 = u.n0;
       wk->n1 = u.n1;
       wk->L = u.L;
       wk->list_in_smem = list_in_smem;
+      wk->tail = tail;
       wk->tmem = *sh.tmem_slot;
     }
   }
@@ -655,7 +683,7 @@ __global__ void __launch_bounds__(THREADS2, 1)
     setmaxnreg_inc_softmax();
     const Work2 w = load_work2(smem);
     const int x = warp >> 2;  // 0: tile A, 1: tile B
-    if (!w.skip && (x == 0 || w.hasB)) softmax_role<EPI>(&tmO, p, x);
+    if (!w.skip && (x == 0 || w.hasB)) softmax_role<EPI>(&tmO, &tmT, p, x);
   }
 
   tc_fence_before_sync();
@@ -672,12 +700,14 @@ size_t tc2_smem_bytes() { return SMEM2_BYTES; }
 
 cudaError_t launch_attn_tc2(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
                             const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
-                            const CUtensorMap& tmO, int grid, cudaStream_t stream) {
+                            const CUtensorMap& tmO, const CUtensorMap& tmT, int grid, cudaStream_t stream) {
+  if (p.tail_k > 0 && p.epi == EPI_MERGE) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   int which;
-  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, AttnParams);
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+               AttnParams);
   if (p.epi == EPI_PARTIAL) {
     kern = attn_tc2_kernel<EPI_PARTIAL>;
     which = 0;
@@ -712,7 +742,7 @@ cudaError_t launch_attn_tc2(const AttnParams& p, const CUtensorMap& tmQ, const C
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tmQ, tmKp, tmVp, tmKb, tmVb, tmO, p);
+  e = cudaLaunchKernelEx(&cfg, kern, tmQ, tmKp, tmVp, tmKb, tmVb, tmO, tmT, p);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -47,6 +47,15 @@ struct AttnParams {
   // (active-unit split, EPI_PARTIAL only): CTA i writes its partial rows to
   // slot i of out_o32 ([grid][128][D]) and out_lse ([grid][128])
   int dyn;
+  // Two-tile kernel, EPI_PARTIAL or EPI_NORM with nsplit = 1: the units from tail_u0 on
+  // (the last, partial wave of CTAs) are split tail_k ways over their keys
+  // (tail_k = 0: no such split).  CTA tail_u0 + i is split i % tail_k of
+  // unit tail_u0 + i / tail_k; it writes its two tiles' partial rows to
+  // slots 2 i and 2 i + 1 of tail_o ([slots][128][D], through the kernel's
+  // second output map) and tail_lse ([slots][128]).
+  int tail_u0, tail_k;
+  float* tail_o;
+  float* tail_lse;
   KeySource src;
   // Test builds only (FB_TEST_HOOKS): 1 = every CTA's K producer leaves the
   // load of its second key tile out, so the pipeline wait for it runs out
@@ -67,6 +76,10 @@ struct CombineParams {
   const int32_t* unit_mask;  // [B, Hkv] or null: rows of units with 0 are left as they are
   int dyn;                // partials in the active-unit slot layout of AttnParams::dyn
   int grid, n_rt;         // (dyn) the attention launch's CTAs and query tiles per unit
+  // tail_k > 0: merge only the tail units' rows, from the slot layout of
+  // AttnParams::tail_o (tail_units units from tail_u0 on, npair tile pairs
+  // per (b, kv head), Hkv kv heads)
+  int tail_k, tail_u0, tail_units, npair, Hkv;
   const float* part_o;    // [nsplit][B][S][Hq][D]
   const float* part_lse;  // [nsplit][B][Hq][S]
   float* out_o32;         // f32 output (prefix pass) or null
@@ -208,9 +221,10 @@ cudaError_t launch_combine(const CombineParams& c, cudaStream_t stream);
 // Two 128-row query tiles per CTA (tiles 2i and 2i + 1 of a unit; the grid is
 // (b, kv head, tile pair, split) with the split fastest): for units of two or
 // more query tiles.  No active-unit split (AttnParams::dyn must be 0).
+// tmT: the tail slots' map (AttnParams::tail_o), or any map when tail_k = 0.
 cudaError_t launch_attn_tc2(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
                             const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
-                            const CUtensorMap& tmO, int grid, cudaStream_t stream);
+                            const CUtensorMap& tmO, const CUtensorMap& tmT, int grid, cudaStream_t stream);
 
 // CUDA-core (fp32) path.
 cudaError_t launch_attn_simt(const AttnParams& p, const float* Q, const float* Kp,

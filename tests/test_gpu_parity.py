@@ -92,6 +92,46 @@ def test_two_tile_kernel_paged_and_split(page_size, num_splits):
     gpu_cases.run_workload(w, page_size=page_size, num_splits=num_splits)
 
 
+@pytest.mark.parametrize("Hq,Hkv,S", [(80, 80, 256), (80, 40, 192)])
+def test_two_tile_prefix_pass_tail_split(Hq, Hkv, S):
+    # 160 units of two-tile CTAs on a GPU of 148 SMs: a last wave of 12, whose
+    # units the prefix pass splits over their keys (into slots the combine
+    # merges) while the first 148 write the cached pair directly.  G = 1 with
+    # one tile pair per unit, and G = 2 with three tiles (a pair and a lone
+    # ragged tile) per unit.
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    w = W["lm_gqa"].scaled(batch=2, num_q_heads=Hq, num_kv_heads=Hkv, block_len=S, prefix_len=1500, steps=2,
+                           blocks=1)
+    rt = -(-S * (Hq // Hkv) // 128)
+    units = w.batch * Hkv * ((rt + 1) // 2)
+    tail = units % sms
+    if not (units > sms and 0 < 2 * tail <= sms):
+        pytest.skip(f"{units} units on {sms} SMs leave no small last wave")
+    K, V, lens = synth.prefix_kv(w)
+    Kt, K64 = gpu_cases.tensors(w, K)
+    Vt, V64 = gpu_cases.tensors(w, V)
+    layer = gpu_cases.make_layer(w)
+    layer.load_prefix(Kt, Vt, lens)
+    k = min(sms // tail, -(-layer.desc.kv_capacity // 128) // 3, 32)
+    assert k >= 2
+    # A workspace that holds the tail slots only -- (tail unit, split, tile) x
+    # 128 rows x (D + 1) floats -- and not the f32 partials of a uniform key
+    # split: the call succeeds only on the one-split plan, which takes the
+    # tail split when its slots fit.
+    tail_bytes = tail * k * 2 * 128 * 129 * 4
+    ws = torch.empty(tail_bytes, dtype=torch.uint8, device="cuda")
+    Q, _, _ = synth.step_inputs(w, 0, 0)
+    Qt, Q64 = gpu_cases.tensors(w, Q)
+    fbl.fb_prefix_partial(layer.desc, Qt, layer.K, layer.V, None, layer.O_pre, layer.LSE_pre, ws, layer.status)
+    layer.check()
+    ref_o, ref_l = ora.prefix_partial(Q64, K64, V64, lens.astype(np.int64), w.softmax_scale, None, 0)
+    gpu_cases.compare("O_pre", layer.O_pre.cpu().numpy(), ref_o, w.dtype)
+    gpu_cases.compare("LSE_pre", layer.LSE_pre.cpu().numpy(), ref_l, w.dtype)
+    del layer, ws
+    # the whole cached schedule and the uncached pass at this shape
+    gpu_cases.run_workload(w)
+
+
 def test_block_step_kernel_choice_both_paths():
     # short blocks with few query rows run the warp-level MMA step kernel with
     # 16 rows per CTA; with more rows than one wave of those CTAs, the one
