@@ -137,9 +137,6 @@ __global__ void __launch_bounds__(WARPS * 32)
       const size_t off = simt_key_offset(p, u, b, kvh, i, blk);
       const float* kr = (blk ? Kb : Kp) + off;
       float acc = 0.f;
-      // (unrolled: eight of the row's loads in flight at a time; the sum
-      // keeps its order)
-#pragma unroll 8
       for (int d = 0; d < D; d += 4) {
         const float4 kv = *reinterpret_cast<const float4*>(kr + d);
         acc = fmaf(sq[warp][d], kv.x, acc);
@@ -156,9 +153,6 @@ __global__ void __launch_bounds__(WARPS * 32)
 #pragma unroll
     for (int k = 0; k < MAXD / 32; ++k) o[k] *= alpha;
     const int nk = min(32, ntot - base);
-    // (unrolled: the value rows' loads are in flight together; the sums keep
-    // their order)
-#pragma unroll 8
     for (int jj = 0; jj < nk; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, pz, jj);
       bool blk;
