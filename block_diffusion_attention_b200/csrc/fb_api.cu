@@ -182,12 +182,13 @@ long long cta_units(const fb_desc& d) {
 // and one of 20, so a sixth of the pass runs on 20 SMs.  Where that last wave
 // holds at most half the SMs, its units can be split k ways over their keys
 // instead (k about SMs / tail units, at least 3 key tiles per split, at most
-// 32 splits), into slots the combine merges, while the other units keep one
+// 31 splits, so that the combine holds them and the step's cached pair in
+// one warp), into slots the combine merges, while the other units keep one
 // CTA each.  tail_splits gives that k (0: no tail split).
 long long tail_splits(long long units, long long slots, long long est_tiles) {
   const long long tail = units % slots;
   if (units <= slots || tail == 0 || 2 * tail > slots) return 0;
-  const long long k = std::min<long long>(slots / tail, std::min<long long>(est_tiles / 3, 32));
+  const long long k = std::min<long long>(slots / tail, std::min<long long>(est_tiles / 3, 31));
   return k >= 2 ? k : 0;
 }
 
@@ -266,6 +267,26 @@ TailPlan tail_plan(const fb_desc& d, int ns, long long est_tiles) {
   const long long slots = device_sms();
   const long long k = tail_splits(units, slots, est_tiles);
   if (k == 0) return t;
+  t.u0 = (int)(units - units % slots);
+  t.units = (int)(units % slots);
+  t.k = (int)k;
+  return t;
+}
+
+// The tail split of the tensor-core step (two-tile units, S > 64): one CTA
+// per unit otherwise, so where its cost model (full waves, then the tail's
+// splits, then the combine) beats the plain grid.
+TailPlan step_tail_plan(const fb_desc& d) {
+  TailPlan t;
+  if (d.dtype != FB_BF16 || small_step_fits(d, device_sms()) || rows_step_fits(d) || !use_pairs(d)) return t;
+  const long long units = cta_units(d);
+  const long long slots = device_sms();
+  const long long est = (d.block_len + TC_BN - 1) / TC_BN;
+  const long long k = tail_splits(units, slots, est);
+  if (k == 0) return t;
+  const double plain = (double)((units + slots - 1) / slots) * ((double)est + 3.0);
+  const double split = (double)(units / slots) * ((double)est + 3.0) + (std::ceil((double)est / (double)k) + 3.0) + 2.0;
+  if (split >= plain) return t;
   t.u0 = (int)(units - units % slots);
   t.units = (int)(units % slots);
   t.k = (int)k;
@@ -361,6 +382,7 @@ size_t fb_workspace_bytes(const fb_desc* d) {
   need = std::max(need, tail_bytes(tail_plan(*d, ns_pre, prefix_tiles_estimate(*d))));
   need = std::max(need, split_bytes(*d, ns_full));
   need = std::max(need, tail_bytes(tail_plan(dense, ns_full, est_full)));
+  need = std::max(need, tail_bytes(step_tail_plan(*d)));
   need = std::max(need, threshold_ws_bytes(*d));
   if (d->dtype == FB_BF16 && !use_pairs(*d)) {
     // the masked prefix pass's active-unit slots
@@ -552,8 +574,8 @@ fb_status fb_threshold_refresh_mask(const fb_desc* d, void* K_prev, void* V_prev
 }
 
 fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const void* Vb,
-                        const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
-                        int32_t* dev_status, fb_stream_t stream) {
+                        const float* O_pre, const float* LSE_pre, void* O, float* LSE_out, void* ws,
+                        size_t ws_bytes, int32_t* dev_status, fb_stream_t stream) {
   fb_status st = check_desc(d);
   if (st != FB_OK) return st;
   if (!Q || !Kb || !Vb || !O_pre || !LSE_pre || !O) return FB_ERR_INVALID_ARG;
@@ -584,6 +606,42 @@ fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const v
   const long long grid = cta_units(*d);
   if (use_pairs(*d)) {
     p.kv_stream_once = (p.n_rt <= 2);
+    // the tail split (see tail_plan) where the workspace holds its slots:
+    // the combine merges the tail's key splits and the cached pair
+    const TailPlan tp = step_tail_plan(*d);
+    if (tp.k > 0 && ws && ws_bytes >= tail_bytes(tp) && aligned16(ws)) {
+      const int slots = tp.units * tp.k * 2;
+      float* tail_o = static_cast<float*>(ws);
+      float* tail_l = tail_o + (size_t)slots * TC_BM * TC_D;
+      p.tail_u0 = tp.u0;
+      p.tail_k = tp.k;
+      p.tail_o = tail_o;
+      p.tail_lse = tail_l;
+      CUtensorMap tm_tail;
+      if (!slot_map(&tm_tail, *d, tail_o, slots)) return FB_ERR_LAUNCH;
+      cudaError_t e = launch_attn_tc2(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_out, tm_tail, tp.u0 + tp.units * tp.k, s);
+      if (e != cudaSuccess) return from_cuda(e);
+      CombineParams c;
+      std::memset(&c, 0, sizeof(c));
+      c.B = d->batch;
+      c.Hq = d->num_q_heads;
+      c.S = d->block_len;
+      c.D = d->head_dim;
+      c.part_o = tail_o;
+      c.part_lse = tail_l;
+      c.out_o = O;
+      c.out_bf16 = 1;
+      c.out_lse = LSE_out;
+      c.G = p.G;
+      c.tail_k = tp.k;
+      c.tail_u0 = tp.u0;
+      c.tail_units = tp.units;
+      c.npair = (p.n_rt + 1) / 2;
+      c.Hkv = d->num_kv_heads;
+      c.pre_o = O_pre;
+      c.pre_lse = LSE_pre;
+      return from_cuda(launch_combine(c, s));
+    }
     return from_cuda(launch_attn_tc2(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_out, tm_out, (int)grid, s));
   }
   return from_cuda(launch_attn_tc(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_pre, tm_out, (int)grid, s));
@@ -591,7 +649,8 @@ fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const v
 
 fb_status fb_block_step_append(const fb_desc* d, const void* Q, const void* Kb, const void* Vb,
                                const float* O_pre, const float* LSE_pre, void* O, float* LSE_out, void* Kc,
-                               void* Vc, int32_t* lens_inout, int32_t* dev_status, fb_stream_t stream) {
+                               void* Vc, int32_t* lens_inout, void* ws, size_t ws_bytes, int32_t* dev_status,
+                               fb_stream_t stream) {
   fb_status st = check_desc(d);
   if (st != FB_OK) return st;
   if (!Q || !Kb || !Vb || !O_pre || !LSE_pre || !O || !Kc || !Vc) return FB_ERR_INVALID_ARG;
@@ -617,7 +676,7 @@ fb_status fb_block_step_append(const fb_desc* d, const void* Q, const void* Kb, 
     return from_cuda(launch_lens_advance(*d, lens_inout, s));
   }
   // other shapes: the step, then the append
-  st = fb_block_step(d, Q, Kb, Vb, O_pre, LSE_pre, O, LSE_out, dev_status, stream);
+  st = fb_block_step(d, Q, Kb, Vb, O_pre, LSE_pre, O, LSE_out, ws, ws_bytes, dev_status, stream);
   if (st != FB_OK) return st;
   return fb_kv_append(d, Kb, Vb, Kc, Vc, lens_inout, dev_status, stream);
 }

@@ -706,14 +706,23 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombinePa
     so = (size_t)TC_BM * c.D;
     sl = TC_BM;
   }
-  if (nsplit <= 32 && c.D == 4 * 32) {
-    // up to 32 splits: every load in flight at once -- lane l reads split l's
-    // LSE and the four output columns 4l..4l+3 of every split
-    const float lse_l = lane < nsplit ? lbase[lane * sl] : -CUDART_INF_F;
+  // the cached pair as one more partial (a tail split of the step: the
+  // merge equation over the splits and the pair at once)
+  const bool pre = c.tail_k > 0 && c.pre_o != nullptr;
+  if (pre || (nsplit <= 32 && c.D == 4 * 32)) {
+    // up to 32 partials: every load in flight at once -- lane l reads
+    // partial l's LSE and the four output columns 4l..4l+3 of every partial
+    const int nterm = nsplit + (pre ? 1 : 0);
+    float lse_l = lane < nsplit ? lbase[lane * sl] : -CUDART_INF_F;
+    if (pre && lane == nsplit) lse_l = c.pre_lse[lrow];
     float4 v[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (i < nsplit) v[i] = __ldg(reinterpret_cast<const float4*>(base + i * so + lane * 4));
+    for (int i = 0; i < 32; ++i) {
+      if (i < nsplit)
+        v[i] = __ldg(reinterpret_cast<const float4*>(base + i * so + lane * 4));
+      else if (pre && i == nsplit)
+        v[i] = __ldg(reinterpret_cast<const float4*>(c.pre_o + row * c.D + lane * 4));
+    }
     const float M = warp_max_f(lse_l);
     const bool empty = (M == -CUDART_INF_F);
     const float w_l = (empty || lse_l == -CUDART_INF_F) ? 0.f : expf(lse_l - M);
@@ -722,8 +731,8 @@ __global__ void __launch_bounds__(CMB_WARPS * 32) combine_kernel(const CombinePa
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float w = __shfl_sync(0xffffffffu, w_l, i);  // split order, as below
-      if (i < nsplit) {
+      const float w = __shfl_sync(0xffffffffu, w_l, i);  // partial order, as below
+      if (i < nterm) {
         acc.x = fmaf(w, v[i].x, acc.x);
         acc.y = fmaf(w, v[i].y, acc.y);
         acc.z = fmaf(w, v[i].z, acc.z);

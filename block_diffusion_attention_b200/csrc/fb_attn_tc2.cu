@@ -49,10 +49,10 @@
 // The epilogue of tile X stages its output in Q_X's region (every QK^T is
 // done once the last PV_X is).
 //
-// A prefix pass (or an uncached pass) whose last wave of CTAs is only partly
-// full may split the keys of those last units (AttnParams::tail_k): such a
-// CTA writes f32 partial rows to its tiles' slots through the second output
-// map, and the combine merges them.
+// A pass whose last wave of CTAs is only partly full may split the keys of
+// those last units (AttnParams::tail_k): such a CTA writes f32 partial rows
+// to its tiles' slots through the second output map, and the combine merges
+// them (for the step, together with the cached pair).
 //
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // FB_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
@@ -480,9 +480,10 @@ __device__ __forceinline__ void softmax_role(const CUtensorMap* tmO, const CUten
   const uint32_t st_row = smem_u32(stage) + r * 128;
   const int t0 = rt * (BM / p.G);
   const bool store = ok && t0 < p.S;  // rows of this tile exist
-  if (EPI == EPI_PARTIAL || (EPI == EPI_NORM && w.tail >= 0)) {
+  if (EPI == EPI_PARTIAL || w.tail >= 0) {
     // the f32 tile (64 KB) in two rounds of 64 columns through the 32 KB stage
-    // (a tail split of the uncached pass writes its partial rows the same way)
+    // (a tail split of the uncached pass or of the step writes its partial
+    // rows the same way; the combine does the rest)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       if (ok) {
@@ -701,7 +702,6 @@ size_t tc2_smem_bytes() { return SMEM2_BYTES; }
 cudaError_t launch_attn_tc2(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmKp,
                             const CUtensorMap& tmVp, const CUtensorMap& tmKb, const CUtensorMap& tmVb,
                             const CUtensorMap& tmO, const CUtensorMap& tmT, int grid, cudaStream_t stream) {
-  if (p.tail_k > 0 && p.epi == EPI_MERGE) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

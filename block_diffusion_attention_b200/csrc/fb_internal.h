@@ -47,7 +47,7 @@ struct AttnParams {
   // (active-unit split, EPI_PARTIAL only): CTA i writes its partial rows to
   // slot i of out_o32 ([grid][128][D]) and out_lse ([grid][128])
   int dyn;
-  // Two-tile kernel, EPI_PARTIAL or EPI_NORM with nsplit = 1: the units from tail_u0 on
+  // Two-tile kernel with nsplit = 1 (any epilogue): the units from tail_u0 on
   // (the last, partial wave of CTAs) are split tail_k ways over their keys
   // (tail_k = 0: no such split).  CTA tail_u0 + i is split i % tail_k of
   // unit tail_u0 + i / tail_k; it writes its two tiles' partial rows to
@@ -80,6 +80,10 @@ struct CombineParams {
   // AttnParams::tail_o (tail_units units from tail_u0 on, npair tile pairs
   // per (b, kv head), Hkv kv heads)
   int tail_k, tail_u0, tail_units, npair, Hkv;
+  // tail_k > 0 and not null: the cached pair joins the merge as one more
+  // partial (the step's merge equation); then tail_k < 32
+  const float* pre_o;     // [B][S][Hq][D]
+  const float* pre_lse;   // [B][Hq][S] natural log
   const float* part_o;    // [nsplit][B][S][Hq][D]
   const float* part_lse;  // [nsplit][B][Hq][S]
   float* out_o32;         // f32 output (prefix pass) or null

@@ -54,6 +54,10 @@ class fb_desc(ctypes.Structure):
 _lib = None
 
 
+# FB_ABI_VERSION of include/flashblock.h that the signatures below follow.
+ABI_VERSION = 2
+
+
 def load() -> ctypes.CDLL:
     """The loaded library (raises if it has not been built)."""
     global _lib
@@ -69,8 +73,8 @@ def load() -> ctypes.CDLL:
             "fb_workspace_bytes": (SZ, [D]),
             "fb_prefix_partial": (I32, [D, P, P, P, P, P, P, P, SZ, P, P]),
             "fb_prefix_partial_noalloc": (I32, [D, P, P, P, P, P, P, P, P]),
-            "fb_block_step": (I32, [D, P, P, P, P, P, P, P, P, P]),
-            "fb_block_step_append": (I32, [D, P, P, P, P, P, P, P, P, P, P, P, P]),
+            "fb_block_step": (I32, [D, P, P, P, P, P, P, P, P, SZ, P, P]),
+            "fb_block_step_append": (I32, [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
             "fb_full_reference_gpu": (I32, [D, P, P, P, P, P, P, P, P, SZ, P, P]),
             "fb_chunk_means": (I32, [D, P, I32, I32, P, P, P]),
             "fb_chunk_means_tail": (I32, [D, P, I32, P, P, P]),
@@ -89,6 +93,9 @@ def load() -> ctypes.CDLL:
             f = getattr(lib, name)
             f.restype = res
             f.argtypes = args
+        if lib.fb_abi_version() != ABI_VERSION:
+            raise RuntimeError(f"{LIB_PATH} has ABI version {lib.fb_abi_version()}, this binding needs "
+                               f"{ABI_VERSION}: rebuild it")
         _lib = lib
     return _lib
 
@@ -158,17 +165,17 @@ def fb_prefix_partial_noalloc(d, Q, Kcache, Vcache, chunk_idx, O_pre, LSE_pre, d
         _p(dev_status), _s(stream)))
 
 
-def fb_block_step(d, Q, Kblk, Vblk, O_pre, LSE_pre, O, LSE_out, dev_status, stream=None):
+def fb_block_step(d, Q, Kblk, Vblk, O_pre, LSE_pre, O, LSE_out, dev_status, stream=None, workspace=None):
     _ok("fb_block_step", load().fb_block_step(
         ctypes.byref(d), _p(Q), _p(Kblk), _p(Vblk), _p(O_pre), _p(LSE_pre), _p(O), _p(LSE_out),
-        _p(dev_status), _s(stream)))
+        _p(workspace), _nbytes(workspace), _p(dev_status), _s(stream)))
 
 
 def fb_block_step_append(d, Q, Kblk, Vblk, O_pre, LSE_pre, O, LSE_out, Kcache, Vcache, lens_inout, dev_status,
-                         stream=None):
+                         stream=None, workspace=None):
     _ok("fb_block_step_append", load().fb_block_step_append(
         ctypes.byref(d), _p(Q), _p(Kblk), _p(Vblk), _p(O_pre), _p(LSE_pre), _p(O), _p(LSE_out), _p(Kcache),
-        _p(Vcache), _p(lens_inout), _p(dev_status), _s(stream)))
+        _p(Vcache), _p(lens_inout), _p(workspace), _nbytes(workspace), _p(dev_status), _s(stream)))
 
 
 def fb_full_reference_gpu(d, Q, Kcache, Vcache, Kblk, Vblk, O, LSE_out, workspace, dev_status, stream=None):

@@ -199,7 +199,7 @@ class CachedBlockAttention:
         if self.residual:
             self._residual_merge(Q)
         fbl.fb_block_step(self.desc, Q, Kblk, Vblk, self.O_pre, self.LSE_pre, out,
-                          self.LSE if lse else None, self.status)
+                          self.LSE if lse else None, self.status, workspace=self.workspace)
         return out
 
     def step_append(self, Q, Kblk, Vblk, out: Optional[torch.Tensor] = None, lse: bool = False,
@@ -213,7 +213,7 @@ class CachedBlockAttention:
             self._residual_merge(Q)
         fbl.fb_block_step_append(self.desc, Q, Kblk, Vblk, self.O_pre, self.LSE_pre, out,
                                  self.LSE if lse else None, self.K, self.V, self.lens if advance else None,
-                                 self.status)
+                                 self.status, workspace=self.workspace)
         if advance and self.topk > 0:
             fbl.fb_chunk_means_tail(self.desc, self.K, self.S, self.Kmean, self.status)
         return out

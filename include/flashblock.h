@@ -53,7 +53,8 @@
 extern "C" {
 #endif
 
-#define FB_ABI_VERSION 1
+/* 2: fb_block_step and fb_block_step_append take an optional workspace. */
+#define FB_ABI_VERSION 2
 
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st* fb_stream_t;
@@ -95,7 +96,9 @@ int64_t fb_cache_rows(const fb_desc* d);
 
 /* Bytes of device workspace that fb_prefix_partial and fb_full_reference_gpu
  * need for this descriptor on the current device (split-key partials:
- * splits x B x S x Hq x (D + 1) float32).  0 means no workspace is needed. */
+ * splits x B x S x Hq x (D + 1) float32), and that lets fb_block_step split
+ * the keys of a nearly empty last wave of CTAs (see there).  0 means no
+ * workspace is needed. */
 size_t fb_workspace_bytes(const fb_desc* d);
 
 /* Block-external partial over the finalized prefix (the cached pair).
@@ -117,11 +120,16 @@ fb_status fb_prefix_partial(const fb_desc* d, const void* Q, const void* Kcache,
  * Q over the block's own keys (bidirectional, no mask) merged in the same
  * kernel with the cached (O_pre, LSE_pre) by the merge equation.
  * Q [B,S,Hq,D], Kblk/Vblk [B,S,Hkv,D] (dtype).  Writes O [B,S,Hq,D] (dtype)
- * and, when LSE_out is not NULL, the merged LSE [B,Hq,S] float32. */
+ * and, when LSE_out is not NULL, the merged LSE [B,Hq,S] float32.
+ * workspace: optional (NULL, or fewer than fb_workspace_bytes(d) bytes, is
+ * allowed).  With it, a long block (S > 64, bf16) whose one-CTA-per-unit grid
+ * ends in a nearly empty wave splits the keys of that wave's units and merges
+ * their partials with the cached pair in a second kernel (the same result up
+ * to rounding); without it every unit keeps one CTA. */
 fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kblk,
                         const void* Vblk, const float* O_pre, const float* LSE_pre,
-                        void* O, float* LSE_out, int32_t* dev_status,
-                        fb_stream_t stream);
+                        void* O, float* LSE_out, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, fb_stream_t stream);
 
 /* Uncached block diffusion (Technical Summary §1 Problem Statement): attention
  * of Q over [prefix rows j < L_b ; all S block rows] in one pass, no cached
@@ -247,8 +255,8 @@ fb_status fb_kv_append(const fb_desc* d, const void* Kblk, const void* Vblk,
  * and errors as for those two calls. */
 fb_status fb_block_step_append(const fb_desc* d, const void* Q, const void* Kblk, const void* Vblk,
                                const float* O_pre, const float* LSE_pre, void* O, float* LSE_out,
-                               void* Kcache, void* Vcache, int32_t* lens_inout, int32_t* dev_status,
-                               fb_stream_t stream);
+                               void* Kcache, void* Vcache, int32_t* lens_inout, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, fb_stream_t stream);
 
 /* Bytes of the static scratch array behind fb_prefix_partial_noalloc. */
 #define FB_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)

@@ -33,7 +33,7 @@ def test_test_hooks_only_in_the_test_library(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert fbl.fb_abi_version() == 1
+    assert fbl.fb_abi_version() == fbl.ABI_VERSION == 2
     for code, name in fbl.STATUS.items():
         assert fbl.fb_status_string(code) == name
     assert fbl.fb_status_string(99) == "FB_ERR_UNKNOWN"
@@ -78,7 +78,7 @@ def test_host_validation_codes(lib):
     d = _desc(kv_capacity=131072)
     assert fbl.fb_workspace_bytes(d) > 0
     assert _prefix(lib, d) == 4
-    blk = lib.fb_block_step(ctypes.byref(_desc()), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, None)
+    blk = lib.fb_block_step(ctypes.byref(_desc()), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 0, None, None)
     assert blk == 1
     assert lib.fb_chunk_means(ctypes.byref(_desc(chunk_size=256)), FAKE, 0, 999, FAKE, None, None) == 1
     assert lib.fb_select_chunks(ctypes.byref(_desc(chunk_size=256, topk=0)), FAKE, FAKE, FAKE, None, None) == 1

@@ -132,6 +132,39 @@ def test_two_tile_prefix_pass_tail_split(Hq, Hkv, S):
     gpu_cases.run_workload(w)
 
 
+def test_two_tile_step_tail_split():
+    # a long block (768 tokens, 52 heads, G = 1: three tile pairs per unit,
+    # 156 units) on a GPU of 148 SMs: the step's last wave holds 8 units,
+    # whose block keys are split 2 ways and merged with the cached pair by
+    # the combine (the prefix pass takes its own tail split here too)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    w = W["video"].scaled(batch=1, num_q_heads=52, num_kv_heads=52, block_len=768, prefix_len=300, steps=2,
+                          blocks=1)
+    units = 52 * 3
+    tail = units % sms
+    if not (units > sms and 0 < 2 * tail <= sms and sms // tail >= 2):
+        pytest.skip(f"{units} units on {sms} SMs leave no small last wave")
+    gpu_cases.run_workload(w)
+    # the split path ran: the same step without a workspace (one CTA per
+    # unit) agrees to rounding and differs in the tail rows
+    K, V, lens = synth.prefix_kv(w)
+    Kt, _ = gpu_cases.tensors(w, K)
+    Vt, _ = gpu_cases.tensors(w, V)
+    layer = gpu_cases.make_layer(w)
+    layer.load_prefix(Kt, Vt, lens)
+    Q, Kb, Vb = synth.step_inputs(w, 0, 0)
+    Qt, _ = gpu_cases.tensors(w, Q)
+    Kbt, _ = gpu_cases.tensors(w, Kb)
+    Vbt, _ = gpu_cases.tensors(w, Vb)
+    layer.refresh(Qt)
+    O_split = layer.step(Qt, Kbt, Vbt)
+    O_one = torch.empty_like(O_split)
+    fbl.fb_block_step(layer.desc, Qt, Kbt, Vbt, layer.O_pre, layer.LSE_pre, O_one, None, layer.status)
+    layer.check()
+    assert not torch.equal(O_split, O_one)
+    assert (O_split.float() - O_one.float()).abs().max().item() < 2e-2
+
+
 def test_block_step_kernel_choice_both_paths():
     # short blocks with few query rows run the warp-level MMA step kernel with
     # 16 rows per CTA; with more rows than one wave of those CTAs, the one
