@@ -338,6 +338,39 @@ bool slot_map(CUtensorMap* m, const fb_desc& d, const float* base, int slots) {
   return make_map(m, base, dims, str, box, true);
 }
 
+// The two-tile kernel with the tail split tp (its slots at the start of ws),
+// then the combine of the tail rows into the outputs (and, for the step, the
+// cached pair) that c names.
+fb_status run_tail_split(AttnParams p, const TailPlan& tp, const fb_desc& d, void* ws, const CUtensorMap& q,
+                         const CUtensorMap& kp, const CUtensorMap& vp, const CUtensorMap& kb,
+                         const CUtensorMap& vb, const CUtensorMap& tm_out, CombineParams c, cudaStream_t s) {
+  const int slots = tp.units * tp.k * 2;
+  float* tail_o = static_cast<float*>(ws);
+  float* tail_l = tail_o + (size_t)slots * TC_BM * TC_D;
+  p.nsplit = 1;
+  p.tail_u0 = tp.u0;
+  p.tail_k = tp.k;
+  p.tail_o = tail_o;
+  p.tail_lse = tail_l;
+  CUtensorMap tm_tail;
+  if (!slot_map(&tm_tail, d, tail_o, slots)) return FB_ERR_LAUNCH;
+  const cudaError_t e = launch_attn_tc2(p, q, kp, vp, kb, vb, tm_out, tm_tail, tp.u0 + tp.units * tp.k, s);
+  if (e != cudaSuccess) return from_cuda(e);
+  c.B = d.batch;
+  c.Hq = d.num_q_heads;
+  c.S = d.block_len;
+  c.D = d.head_dim;
+  c.G = p.G;
+  c.part_o = tail_o;
+  c.part_lse = tail_l;
+  c.tail_k = tp.k;
+  c.tail_u0 = tp.u0;
+  c.tail_units = tp.units;
+  c.npair = (p.n_rt + 1) / 2;
+  c.Hkv = d.num_kv_heads;
+  return from_cuda(launch_combine(c, s));
+}
+
 bool block_map(CUtensorMap* m, const fb_desc& d, const void* X) {
   const uint64_t D = d.head_dim, H = d.num_kv_heads, S = d.block_len, B = d.batch;
   const uint64_t dims[4] = {D, H, S, B};
@@ -459,39 +492,17 @@ fb_status prefix_partial(const fb_desc* d, const void* Q, const void* Kc, const 
   // the tail split where the workspace holds its slots (else the plain plan)
   const TailPlan tp = pairs ? tail_plan(*d, ns, prefix_tiles_estimate(*d)) : TailPlan{};
   if (tp.k > 0 && ws && ws_bytes >= tail_bytes(tp) && aligned16(ws)) {
-    const int slots = tp.units * tp.k * 2;
-    float* tail_o = static_cast<float*>(ws);
-    float* tail_l = tail_o + (size_t)slots * TC_BM * TC_D;
-    p.nsplit = 1;
-    p.tail_u0 = tp.u0;
-    p.tail_k = tp.k;
-    p.tail_o = tail_o;
-    p.tail_lse = tail_l;
     p.out_o32 = O_pre;
     p.out_lse = LSE_pre;
     p.kv_stream_once = (p.n_rt <= 2);
-    CUtensorMap tm_out, tm_tail;
-    if (!pre_map(&tm_out, *d, O_pre, d->batch) || !slot_map(&tm_tail, *d, tail_o, slots)) return FB_ERR_LAUNCH;
-    cudaError_t e = launch_attn_tc2(p, m.q, m.kp, m.vp, m.kp, m.vp, tm_out, tm_tail, tp.u0 + tp.units * tp.k, s);
-    if (e != cudaSuccess) return from_cuda(e);
+    CUtensorMap tm_out;
+    if (!pre_map(&tm_out, *d, O_pre, d->batch)) return FB_ERR_LAUNCH;
     CombineParams c;
     std::memset(&c, 0, sizeof(c));
-    c.B = d->batch;
-    c.Hq = d->num_q_heads;
-    c.S = d->block_len;
-    c.D = d->head_dim;
-    c.part_o = tail_o;
-    c.part_lse = tail_l;
     c.out_o32 = O_pre;
     c.out_lse = LSE_pre;
-    c.G = p.G;
     c.unit_mask = unit_mask;
-    c.tail_k = tp.k;
-    c.tail_u0 = tp.u0;
-    c.tail_units = tp.units;
-    c.npair = (p.n_rt + 1) / 2;
-    c.Hkv = d->num_kv_heads;
-    return from_cuda(launch_combine(c, s));
+    return run_tail_split(p, tp, *d, ws, m.q, m.kp, m.vp, m.kp, m.vp, tm_out, c, s);
   }
   p.nsplit = ns;
   float* part_o = O_pre;
@@ -610,37 +621,14 @@ fb_status fb_block_step(const fb_desc* d, const void* Q, const void* Kb, const v
     // the combine merges the tail's key splits and the cached pair
     const TailPlan tp = step_tail_plan(*d);
     if (tp.k > 0 && ws && ws_bytes >= tail_bytes(tp) && aligned16(ws)) {
-      const int slots = tp.units * tp.k * 2;
-      float* tail_o = static_cast<float*>(ws);
-      float* tail_l = tail_o + (size_t)slots * TC_BM * TC_D;
-      p.tail_u0 = tp.u0;
-      p.tail_k = tp.k;
-      p.tail_o = tail_o;
-      p.tail_lse = tail_l;
-      CUtensorMap tm_tail;
-      if (!slot_map(&tm_tail, *d, tail_o, slots)) return FB_ERR_LAUNCH;
-      cudaError_t e = launch_attn_tc2(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_out, tm_tail, tp.u0 + tp.units * tp.k, s);
-      if (e != cudaSuccess) return from_cuda(e);
       CombineParams c;
       std::memset(&c, 0, sizeof(c));
-      c.B = d->batch;
-      c.Hq = d->num_q_heads;
-      c.S = d->block_len;
-      c.D = d->head_dim;
-      c.part_o = tail_o;
-      c.part_lse = tail_l;
       c.out_o = O;
       c.out_bf16 = 1;
       c.out_lse = LSE_out;
-      c.G = p.G;
-      c.tail_k = tp.k;
-      c.tail_u0 = tp.u0;
-      c.tail_units = tp.units;
-      c.npair = (p.n_rt + 1) / 2;
-      c.Hkv = d->num_kv_heads;
       c.pre_o = O_pre;
       c.pre_lse = LSE_pre;
-      return from_cuda(launch_combine(c, s));
+      return run_tail_split(p, tp, *d, ws, m.q, m.kb, m.vb, m.kb, m.vb, tm_out, c, s);
     }
     return from_cuda(launch_attn_tc2(p, m.q, m.kb, m.vb, m.kb, m.vb, tm_out, tm_out, (int)grid, s));
   }
@@ -725,35 +713,12 @@ fb_status fb_full_reference_gpu(const fb_desc* d, const void* Q, const void* Kc,
     // the tail split (see tail_plan) where the workspace holds its slots
     const TailPlan tp = pairs ? tail_plan(dense, ns, est) : TailPlan{};
     if (tp.k > 0 && ws && ws_bytes >= tail_bytes(tp) && aligned16(ws)) {
-      const int slots = tp.units * tp.k * 2;
-      float* tail_o = static_cast<float*>(ws);
-      float* tail_l = tail_o + (size_t)slots * TC_BM * TC_D;
-      p.tail_u0 = tp.u0;
-      p.tail_k = tp.k;
-      p.tail_o = tail_o;
-      p.tail_lse = tail_l;
-      CUtensorMap tm_tail;
-      if (!slot_map(&tm_tail, dense, tail_o, slots)) return FB_ERR_LAUNCH;
-      cudaError_t e = launch_attn_tc2(p, m.q, m.kp, m.vp, m.kb, m.vb, tm_out, tm_tail, tp.u0 + tp.units * tp.k, s);
-      if (e != cudaSuccess) return from_cuda(e);
       CombineParams c;
       std::memset(&c, 0, sizeof(c));
-      c.B = d->batch;
-      c.Hq = d->num_q_heads;
-      c.S = d->block_len;
-      c.D = d->head_dim;
-      c.part_o = tail_o;
-      c.part_lse = tail_l;
       c.out_o = O;
       c.out_bf16 = 1;
       c.out_lse = LSE_out;
-      c.G = p.G;
-      c.tail_k = tp.k;
-      c.tail_u0 = tp.u0;
-      c.tail_units = tp.units;
-      c.npair = (p.n_rt + 1) / 2;
-      c.Hkv = d->num_kv_heads;
-      return from_cuda(launch_combine(c, s));
+      return run_tail_split(p, tp, dense, ws, m.q, m.kp, m.vp, m.kb, m.vb, tm_out, c, s);
     }
     if (pairs) return from_cuda(launch_attn_tc2(p, m.q, m.kp, m.vp, m.kb, m.vb, tm_out, tm_out, (int)units, s));
     return from_cuda(launch_attn_tc(p, m.q, m.kp, m.vp, m.kb, m.vb, m.q, tm_out, (int)units, s));
