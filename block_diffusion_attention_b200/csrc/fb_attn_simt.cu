@@ -2,13 +2,16 @@
 //
 // The fp32 path keeps float32 inputs exact to about 1e-6 (the tensor cores
 // have no fp32-input kind, and TF32 would not hold 1e-5).  One warp computes
-// one query row (b, t, h): lanes take 32 keys at a time, the row max and the
-// row sum come from warp shuffles, and each lane accumulates D/32 output
-// columns.  Key sources, epilogues and the merge are those of the tensor-core
+// one query row (b, t, h): lanes take 32 keys at a time (each lane copies its
+// key's K and V rows into shared memory with cp.async, all copies in flight
+// at once), the row max and the row sum come from warp shuffles, and each
+// lane accumulates D/32 output columns from the staged value rows.  Key sources, epilogues and the merge are those of the tensor-core
 // kernel (the partial, the merge equation and the uncached pass of the Core
 // Mechanism in "FlashBlock: Attention Caching for Efficient Long-Context
 // Block Diffusion", Technical Summary §2).
 #include <math_constants.h>
+
+#include <atomic>
 
 #include "fb_internal.h"
 #include "fb_ptx.cuh"
@@ -19,6 +22,9 @@ namespace {
 
 constexpr int MAXD = 128;
 constexpr int WARPS = 4;
+constexpr int VROW = MAXD + 4;  // floats per staged key or value row (16-byte aligned, banks staggered)
+// the key and the value rows of a chunk, per warp
+constexpr size_t SIMT_SMEM = (size_t)2 * WARPS * 32 * VROW * sizeof(float);
 
 struct SimtUnit {
   int n0;  // prefix keys
@@ -108,6 +114,7 @@ __global__ void __launch_bounds__(WARPS * 32)
   pdl_wait();
   pdl_launch_dependents();
   __shared__ float sq[WARPS][MAXD];
+  extern __shared__ __align__(16) float simt_sv[];  // values [WARPS][32 keys][VROW], then keys alike
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * WARPS + warp;
@@ -132,13 +139,24 @@ __global__ void __launch_bounds__(WARPS * 32)
   for (int base = 0; base < ntot; base += 32) {
     const int i = base + lane;
     float z = -CUDART_INF_F;
+    // this lane's key row (K and V share the layout): offset and tensor
+    size_t off = 0;
+    bool blk = false;
+    float* sv = simt_sv + ((size_t)warp * 32 + lane) * VROW;  // this lane's key's value row
+    float* sk = sv + (size_t)WARPS * 32 * VROW;                // and its key row
     if (i < ntot) {
-      bool blk;
-      const size_t off = simt_key_offset(p, u, b, kvh, i, blk);
-      const float* kr = (blk ? Kb : Kp) + off;
+      off = simt_key_offset(p, u, b, kvh, i, blk);
+      // the key and value rows go to shared memory with all their copies in
+      // flight at once (the value rows are read only after the dot products)
+      const float* krow = (blk ? Kb : Kp) + off;
+      const float* vrow = (blk ? Vb : Vp) + off;
+      for (int d = 0; d < D; d += 4) cp_async16(smem_u32(sk + d), krow + d, 16u);
+      for (int d = 0; d < D; d += 4) cp_async16(smem_u32(sv + d), vrow + d, 16u);
+      cp_async_commit();
+      cp_async_wait_all();  // (this lane's own rows: no other lane's copies needed)
       float acc = 0.f;
       for (int d = 0; d < D; d += 4) {
-        const float4 kv = *reinterpret_cast<const float4*>(kr + d);
+        const float4 kv = *reinterpret_cast<const float4*>(sk + d);
         acc = fmaf(sq[warp][d], kv.x, acc);
         acc = fmaf(sq[warp][d + 1], kv.y, acc);
         acc = fmaf(sq[warp][d + 2], kv.z, acc);
@@ -153,15 +171,17 @@ __global__ void __launch_bounds__(WARPS * 32)
 #pragma unroll
     for (int k = 0; k < MAXD / 32; ++k) o[k] *= alpha;
     const int nk = min(32, ntot - base);
+    // the chunk's value rows, staged by their lanes, from shared memory
+    __syncwarp();
+    const float* svw = simt_sv + (size_t)warp * 32 * VROW;
+#pragma unroll 8
     for (int jj = 0; jj < nk; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, pz, jj);
-      bool blk;
-      const size_t off = simt_key_offset(p, u, b, kvh, base + jj, blk);
-      const float* vr = (blk ? Vb : Vp) + off;
 #pragma unroll
       for (int k = 0; k < MAXD / 32; ++k)
-        if (k < nd) o[k] = fmaf(pj, vr[lane + 32 * k], o[k]);
+        if (k < nd) o[k] = fmaf(pj, svw[jj * VROW + lane + 32 * k], o[k]);
     }
+    __syncwarp();  // the rows may be written again by the next chunk
     m = m_new;
   }
 
@@ -209,7 +229,18 @@ cudaError_t launch_attn_simt(const AttnParams& p, const float* Q, const float* K
       p.epi == EPI_PARTIAL ? attn_simt_kernel<EPI_PARTIAL>
       : p.epi == EPI_MERGE ? attn_simt_kernel<EPI_MERGE>
                            : attn_simt_kernel<EPI_NORM>;
-  cudaError_t e = launch_pdl(kern, grid, dim3(WARPS * 32), 0, stream, p, Q, Kp, Vp, Kb, Vb);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  // (set once per device and kernel)
+  static std::atomic<bool> configured[64][3];
+  const int which = p.epi == EPI_PARTIAL ? 0 : p.epi == EPI_MERGE ? 1 : 2;
+  if (dev >= 64 || !configured[dev][which].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SIMT_SMEM);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) configured[dev][which].store(true, std::memory_order_release);
+  }
+  e = launch_pdl(kern, grid, dim3(WARPS * 32), SIMT_SMEM, stream, p, Q, Kp, Vp, Kb, Vb);
   note_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }
