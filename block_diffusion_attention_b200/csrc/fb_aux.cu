@@ -87,10 +87,10 @@ constexpr int SEL_THREADS = 512;
 constexpr int SEL_PART_FLOATS = SEL_THREADS * 8;  // row-group sums of the query mean (16-bit inputs)
 
 size_t sel_smem_bytes(int D, int nch_total) {
-  // row-group sums, qbar, every score (padded to 4), every key (padded to
-  // 2), one rank per chunk, warp totals
+  // row-group sums, qbar, every score (padded to 4; the ranks later take its
+  // place), every key (padded to 2), warp totals
   return (size_t)(SEL_PART_FLOATS + D + ((nch_total + 3) & ~3)) * sizeof(float) +
-         (size_t)((nch_total + 1) & ~1) * 8 + (size_t)nch_total * sizeof(int) + (SEL_THREADS / 32) * sizeof(int);
+         (size_t)((nch_total + 1) & ~1) * 8 + (SEL_THREADS / 32) * sizeof(int);
 }
 
 // Adds the eight bf16 or four f32 values of a 16-byte vector to acc.
@@ -126,8 +126,8 @@ __device__ __forceinline__ unsigned long long rank_key(float sc, int c) {
 
 // Steps 3b and 4 of the selection, from the scores of the nch valid chunks in
 // shared memory (key: nch 64-bit keys rounded up to an even count, rank: nch
-// ints and wsum: SEL_THREADS / 32 ints of shared memory); writes the unit's
-// topk list to out.
+// ints, which may take the scores' place, and wsum: SEL_THREADS / 32 ints of
+// shared memory); writes the unit's topk list to out.
 //   3b. rank of each chunk = the chunks that rank above it, counted by 1, 2
 //       or 4 lanes per chunk (as many as keep all chunks in one pass of the
 //       CTA where they can), two keys per shared-memory read; a chunk is
@@ -196,11 +196,11 @@ __global__ void __launch_bounds__(SEL_THREADS)
   const int D = g.D;
   float* rowsum = sm;                       // [rpi][D] row-group sums
   float* qbar = rowsum + SEL_PART_FLOATS;   // [D]
-  float* score = qbar + D;                  // [nch_total rounded up to 4]
+  float* score = qbar + D;                  // [nch_total rounded up to 4]; later the ranks
   unsigned long long* key =                 // [nch_total rounded up to 2], 16-byte aligned
       reinterpret_cast<unsigned long long*>(score + ((nch_total + 3) & ~3));
-  int* rank = reinterpret_cast<int*>(key + ((nch_total + 1) & ~1));  // [nch_total]
-  int* wsum = rank + nch_total;             // [warps]
+  int* rank = reinterpret_cast<int*>(score);  // (the scores are not read once the keys exist)
+  int* wsum = reinterpret_cast<int*>(key + ((nch_total + 1) & ~1));  // [warps]
   // 1. the first pass's chunk means, loaded before anything else (rows below
   // nch_total always exist, whatever the prefix length), in flight with the
   // query loads.  Lane q4 of a chunk's four takes the float4s q4, q4 + 4, ...
@@ -291,11 +291,11 @@ constexpr int SELB_GROUPS = 32;  // row groups of the column sums (at most)
 
 size_t sel_bulk_smem_bytes(int rows, int nch_total, size_t esz) {
   // barrier (16), chunk means, query rows, row-group sums, qbar, every
-  // score (padded to 4), every key (padded to 2), one rank per chunk, warp
-  // totals
+  // score (padded to 4; the ranks later take its place), every key (padded
+  // to 2), warp totals
   return 16 + (size_t)nch_total * SELB_D * 4 + (size_t)rows * SELB_D * esz +
          (size_t)(SELB_GROUPS * SELB_D + SELB_D + ((nch_total + 3) & ~3)) * sizeof(float) +
-         (size_t)((nch_total + 1) & ~1) * 8 + (size_t)nch_total * sizeof(int) + (SEL_THREADS / 32) * sizeof(int);
+         (size_t)((nch_total + 1) & ~1) * 8 + (SEL_THREADS / 32) * sizeof(int);
 }
 
 template <typename T>
@@ -314,11 +314,11 @@ __global__ void __launch_bounds__(SEL_THREADS)
   T* sq = reinterpret_cast<T*>(skm + (size_t)nch_total * D);  // [rows][D]
   float* part = reinterpret_cast<float*>(sq + (size_t)rows * D);  // [SELB_GROUPS][D]
   float* qbar = part + SELB_GROUPS * D;                       // [D]
-  float* score = qbar + D;                                    // [nch_total rounded up to 4]
+  float* score = qbar + D;                                    // [nch_total rounded up to 4]; later the ranks
   unsigned long long* key =                                   // [nch_total rounded up to 2]
       reinterpret_cast<unsigned long long*>(score + ((nch_total + 3) & ~3));
-  int* rank = reinterpret_cast<int*>(key + ((nch_total + 1) & ~1));  // [nch_total]
-  int* wsum = rank + nch_total;                               // [warps]
+  int* rank = reinterpret_cast<int*>(score);                  // (scores are not read once the keys exist)
+  int* wsum = reinterpret_cast<int*>(key + ((nch_total + 1) & ~1));  // [warps]
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
