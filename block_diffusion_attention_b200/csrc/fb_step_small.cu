@@ -288,18 +288,22 @@ __global__ void __launch_bounds__(SS_THREADS) block_step_small_kernel(const Smal
   }
 }
 
-// The same step for many query rows: a CTA takes 64 packed rows of one
-// (b, kv head), 16 per warp, and each warp runs its own rows over all 128
-// dims (no work repeated across warps).  K, V and Q reach shared memory by
-// cp.async (52 KB at 64 keys, so four CTAs share an SM and the grid runs in
-// about one wave where the tcgen05 kernel, one CTA per SM, needs several).
+// The same step for many query rows: a CTA takes 128 packed rows of one
+// (b, kv head), 16 per warp of eight, and each warp runs its own rows over
+// all 128 dims (no work repeated across warps).  K, V and Q reach shared
+// memory by cp.async (70 KB at 64 keys; two CTAs share an SM, so the batched
+// sparse step's 256 CTAs run in one wave, and each unit's K/V block is
+// brought in by two CTAs: 13.1 us against 13.9 us with 64 rows per CTA, four
+// CTAs per SM).
 // The cached O_pre entries are loaded at the start straight into the P V
 // accumulators: the merge is taken as one more online-softmax update,
 //     M* = max(m, L2_pre),  a = 2^(L2_pre - M*),  P' = 2^(s - M*),
 //     O = (a O_pre + P' V) / (a + sum P'),  L2 = M* + log2(a + sum P'),
 // which is the merge equation with both weights at most 1, so the O_pre
 // loads are in flight with those of K, V and Q.
-constexpr int SR_ROWS = 16 * SS_WARPS;  // packed query rows per CTA
+constexpr int SR_WARPS = 8;
+constexpr int SR_THREADS = SR_WARPS * 32;
+constexpr int SR_ROWS = 16 * SR_WARPS;  // packed query rows per CTA
 
 template <int SP>
 constexpr uint32_t rows_smem_bytes() {
@@ -307,7 +311,7 @@ constexpr uint32_t rows_smem_bytes() {
 }
 
 template <int SP>
-__global__ void __launch_bounds__(SS_THREADS, 4) block_step_rows_kernel(const SmallStepParams p) {
+__global__ void __launch_bounds__(SR_THREADS, 16 / SR_WARPS) block_step_rows_kernel(const SmallStepParams p) {
   static_assert(SP % 16 == 0 && SP <= SS_MAX_S, "padded key count");
   extern __shared__ __align__(16) uint8_t rows_smem[];
   uint8_t* sQ = rows_smem;                      // [SR_ROWS][272]
@@ -340,14 +344,14 @@ __global__ void __launch_bounds__(SS_THREADS, 4) block_step_rows_kernel(const Sm
   // zero-filled); the cached pair of this lane's entries into registers:
   // O_pre dims 8 j + 2 (lane % 4) + {0, 1} of the rows lane / 4 (entries 0,
   // 1 of accumulator j) and lane / 4 + 8 (entries 2, 3)
-  for (int i = threadIdx.x; i < SP * 16; i += SS_THREADS) {
+  for (int i = threadIdx.x; i < SP * 16; i += SR_THREADS) {
     const int k = i >> 4, c = i & 15;
     const bool ok = k < p.S;
     const size_t src = ok ? (((size_t)b * p.S + k) * p.Hkv + kvh) * SS_D + c * 8 : 0;
     cp_async16(smem_u32(sK + k * SS_ROW_BYTES + c * 16), p.Kb + src, ok ? 16u : 0u);
     cp_async16(smem_u32(sV + k * SS_ROW_BYTES + c * 16), p.Vb + src, ok ? 16u : 0u);
   }
-  for (int i = threadIdx.x; i < SR_ROWS * 16; i += SS_THREADS) {
+  for (int i = threadIdx.x; i < SR_ROWS * 16; i += SR_THREADS) {
     const int row = i >> 4, c = i & 15;
     const int pr = pr0 + row;
     const bool ok = pr < rows_unit;
@@ -375,7 +379,7 @@ __global__ void __launch_bounds__(SS_THREADS, 4) block_step_rows_kernel(const Sm
     // the last step of a block: this unit's K/V rows join the cache
     const int L = append_start(p, b);
     bool ok = true;
-    for (int i = threadIdx.x; L >= 0 && i < p.S * 16; i += SS_THREADS) {
+    for (int i = threadIdx.x; L >= 0 && i < p.S * 16; i += SR_THREADS) {
       const int k = i >> 4, c = i & 15;
       ok = append_chunk(p, p.Kc, b, kvh, L, k, c, *reinterpret_cast<const uint4*>(sK + k * SS_ROW_BYTES + c * 16)) &&
            append_chunk(p, p.Vc, b, kvh, L, k, c, *reinterpret_cast<const uint4*>(sV + k * SS_ROW_BYTES + c * 16)) &&
@@ -546,7 +550,7 @@ cudaError_t launch_rows(const SmallStepParams& p, dim3 grid, cudaStream_t stream
     if (e != cudaSuccess) return e;
     if (dev < 64) configured[dev].store(true, std::memory_order_release);
   }
-  return launch_pdl(block_step_rows_kernel<SP>, grid, dim3(SS_THREADS), rows_smem_bytes<SP>(), stream, p);
+  return launch_pdl(block_step_rows_kernel<SP>, grid, dim3(SR_THREADS), rows_smem_bytes<SP>(), stream, p);
 }
 }  // namespace
 

@@ -76,7 +76,7 @@ def test_wide_groups(B, L, S, G):
     # 32 and 64 query heads per kv head: a 128-row query tile holds 4 or 2
     # tokens of one group in the prefix pass; the step runs the 16-row MMA
     # kernel (the first two), the tcgen05 kernel (S > 64, ragged query tiles)
-    # and the 64-row MMA kernel (the last)
+    # and the 128-row MMA kernel (the last)
     w = W["lm_gqa"].scaled(batch=B, prefix_len=L, block_len=S, num_q_heads=2 * G, num_kv_heads=2, blocks=2,
                            steps=2)
     gpu_cases.run_workload(w)
@@ -168,7 +168,7 @@ def test_two_tile_step_tail_split():
 def test_block_step_kernel_choice_both_paths():
     # short blocks with few query rows run the warp-level MMA step kernel with
     # 16 rows per CTA; with more rows than one wave of those CTAs, the one
-    # with 64 rows per CTA (16 per warp) -- both against the oracle, the
+    # with 128 rows per CTA (16 per warp) -- both against the oracle, the
     # latter also with units whose row count leaves warps without rows (7
     # tokens x 4 heads = 28 rows) and with one-token blocks
     few = W["lm_gqa"].scaled(prefix_len=300, block_len=48, num_q_heads=16, num_kv_heads=2, blocks=1, steps=2)
@@ -328,7 +328,7 @@ def test_block_graph_advances_the_sequence(name, page_size):
                                                           (2, 0, 100, "lm_gqa"), (2, 0, 16, "tiny_fp32")])
 def test_step_append_equals_step_then_append(batch, page_size, block_len, wl):
     # the block's last step with its append fused into the step kernel (the
-    # 16-row kernel at batch 1, the 64-row kernel at batch 12; a 100-token
+    # 16-row kernel at batch 1, the 128-row kernel at batch 12; a 100-token
     # block and the fp32 path run the step and the append one after the
     # other): the same output, cache rows and lengths as fb_block_step then
     # fb_kv_append
