@@ -121,7 +121,8 @@ def workload_config(w, extra=None):
         "parallelism": "replicas",
         "l2": "KV cache larger than the 126 MB L2 at this workload; no flush" if kv_cache_bytes(w) > L2_BYTES else
               "KV cache fits in L2: the replayed blocks and prefix_gbs are L2-warm; prefix_pass_l2_cold_us times "
-              "the pass after a 256 MB scratch write",
+              "the pass after a 256 MB scratch read (L2 left holding clean lines), prefix_pass_l2_cold_dirty_us "
+              "after a 256 MB scratch write (dirty lines written back during the pass)",
     }
     if extra:
         cfg.update(extra)
@@ -564,24 +565,30 @@ def run_ours(args):
         del g_pre
     if not policy and kv_cache_bytes(w) < L2_BYTES:
         # The KV cache fits in L2, so the replayed blocks time the prefix pass
-        # L2-warm.  Cold figure: before each pass a 256 MB scratch buffer is
-        # written (evicting the cache from L2), then the pass is timed alone.
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        # L2-warm.  Cold figures, the pass timed alone after the cache has
+        # been evicted from L2 by (a) a read of a 256 MB scratch buffer: the
+        # L2 then holds clean lines, as after other layers' weight reads;
+        # (b) a write of it: the L2 then holds 126 MB of dirty lines, whose
+        # write-back to HBM runs during the pass and is charged to it.
+        flush = torch.zeros(256 << 20, dtype=torch.uint8, device="cuda")
+        total = torch.zeros((), dtype=torch.int64, device="cuda")
         Q0 = dev_in[0][0]
-        cold = []
-        for k in range(args.warmup + args.steps):
-            flush.fill_(k & 0xFF)
-            a = torch.cuda.Event(enable_timing=True)
-            c = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            cached.select(Q0)
-            cached.prefix(Q0)
-            c.record(stream)
-            if k >= args.warmup:
-                cold.append((a, c))
-        torch.cuda.synchronize()
-        res["pre_cold_ms"] = [a.elapsed_time(c) for a, c in cold]
-        del flush
+        for key, evict in (("pre_cold_ms", lambda k: torch.sum(flush, 0, dtype=torch.int64, out=total)),
+                           ("pre_cold_dirty_ms", lambda k: flush.fill_(k & 0xFF))):
+            cold = []
+            for k in range(args.warmup + args.steps):
+                evict(k)
+                a = torch.cuda.Event(enable_timing=True)
+                c = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                cached.select(Q0)
+                cached.prefix(Q0)
+                c.record(stream)
+                if k >= args.warmup:
+                    cold.append((a, c))
+            torch.cuda.synchronize()
+            res[key] = [a.elapsed_time(c) for a, c in cold]
+        del flush, total
     if not policy:
         # The method's reuse error on these synthetic inputs (outside every
         # timed region): per denoising step, the relative distance of the
@@ -735,6 +742,8 @@ def report(args, w0, w, world, res):
 
     pre_avg = sum(res["pre_ms"]) / len(res["pre_ms"])
     cold_us = (sum(res["pre_cold_ms"]) / len(res["pre_cold_ms"]) * 1e3) if res.get("pre_cold_ms") else None
+    cold_dirty_us = ((sum(res["pre_cold_dirty_ms"]) / len(res["pre_cold_dirty_ms"]) * 1e3)
+                     if res.get("pre_cold_dirty_ms") else None)
     blk_avg = sum(res["blk_ms"]) / len(res["blk_ms"])
     mid = [(a + b) / 2 for a, b in zip(res["lens0"], res["lens1"])]
     abytes = prefix_bytes(w, mid, args.residual)
@@ -796,6 +805,7 @@ def report(args, w0, w, world, res):
         "prefix_pass_l2_cold_us": cold_us,
         "prefix_gbs_l2_cold": (abytes / (cold_us * 1e-6) / 1e9) if cold_us else None,
         "prefix_hbm_frac_l2_cold": (abytes / (cold_us * 1e-6) / 1e9 / hbm_peak) if cold_us else None,
+        "prefix_pass_l2_cold_dirty_us": cold_dirty_us,
         "roofline": roof,
         "clocks": res["clocks"],
         "reuse_error": ({"per_denoise_step": res["reuse_err"], "refresh_steps": list(w.refresh),
