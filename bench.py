@@ -51,8 +51,8 @@ METRIC = "attention µs/denoise-step and tokens/s, cached vs uncached; prefix-pa
 # hash differs from the built sources is not reported: the kernel changed
 # since the counters were taken.
 NCU_TRAFFIC = {
-    # profiles/prefix_pass_long_ctx.md, capture b50_traffic_lc
-    "long_ctx": {"bytes": 537209344 + 3133184, "sources": "4694f290a6b0e554"},
+    # profiles/prefix_pass_long_ctx.md, capture b53_traffic_lc
+    "long_ctx": {"bytes": 537209088 + 2964736, "sources": "8db3988978716104"},
 }
 KERNEL_SOURCES = ("fb_attn_tc.cu", "fb_attn_common.cuh", "fb_ptx.cuh", "fb_internal.h", "fb_api.cu")
 

@@ -221,12 +221,15 @@ int choose_splits(const fb_desc& d, long long est_tiles) {
       best = (int)ns;
     }
   }
-  // The fewest splits whose cost is within 7 % of the best: the model counts
-  // work per SM, but a streaming pass gains nothing from more CTAs once HBM
-  // is saturated, and every split adds partials to combine (128K dense
-  // prefix, 8 kv heads: 17 splits 92.2 us, 18 splits 97.2 us, 16 splits
-  // 92.2-94.1 us, 15 splits 95.9-97.4 us).
-  for (long long ns = 1; ns < best; ++ns) {
+  // One-tile units (an HBM-streaming pass): the fewest splits whose cost is
+  // within 7 % of the best.  The model counts work per SM, but such a pass
+  // gains nothing from more CTAs once HBM is saturated, and every split adds
+  // partials to combine (128K dense prefix, 8 kv heads: 17 splits 92.2 us,
+  // 18 splits 97.2 us, 16 splits 92.2-94.1 us, 15 splits 95.9-97.4 us).
+  // Not for two-tile units, which are bound by the tensor pipe and the
+  // softmax: one wave of 128 unsplit CTAs on 148 SMs (uncached pass, 16
+  // sequences, 32K dense prefix) took 504 us against 457 us for 8 splits.
+  for (long long ns = 1; ns < best && !use_pairs(d); ++ns) {
     const long long waves = (units * ns + slots - 1) / slots;
     const double cost = (double)waves * (std::ceil((double)est_tiles / (double)ns) + 3.0) + (ns > 1 ? 2.0 : 0.0);
     if (cost <= 1.07 * best_cost) {
