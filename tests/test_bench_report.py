@@ -72,14 +72,17 @@ def test_recorded_traffic_needs_the_captured_sources(monkeypatch):
 
 def test_report_l2_cold_prefix_figure(capsys):
     # a workload whose KV cache fits in L2 reports the prefix pass after an
-    # L2 flush beside the warm figure
+    # L2 eviction (a scratch read; and a scratch write, dirty lines) beside
+    # the warm figure
     args = _args(workload="lm_gqa")
     w = synth.WORKLOADS["lm_gqa"].scaled(blocks=1)
     assert bench.kv_cache_bytes(w) < bench.L2_BYTES
-    bench.report(args, synth.WORKLOADS["lm_gqa"], w, 1, _res(w, pre_cold_ms=[0.02, 0.02]))
+    bench.report(args, synth.WORKLOADS["lm_gqa"], w, 1,
+                 _res(w, pre_cold_ms=[0.02, 0.02], pre_cold_dirty_ms=[0.024, 0.026]))
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["prefix_pass_l2_cold_us"] == pytest.approx(20.0)
     assert line["prefix_gbs_l2_cold"] == pytest.approx(bench.prefix_bytes(w, [w.prefix_len]) / 20e-6 / 1e9)
+    assert line["prefix_pass_l2_cold_dirty_us"] == pytest.approx(25.0)
     assert "L2" in line["config"]["l2"]
 
 
