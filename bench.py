@@ -731,6 +731,15 @@ def run_ours(args):
     return 0
 
 
+def e2e_bound(res, args):
+    """The longest of the three things an end-to-end block overlaps: its
+    compute (the device-timed cached block) and each copy direction timed
+    alone."""
+    parts = {"compute": res["ms_cached"] / args.steps, "host-to-device copies": res["h2d_ms"],
+             "device-to-host copies": res["d2h_ms"]}
+    return max(parts, key=parts.get)
+
+
 def report(args, w0, w, world, res):
     policy = args.policy
     tau = args.tau if args.tau is not None else max(1, w.block_len // 4)
@@ -818,7 +827,8 @@ def report(args, w0, w, world, res):
                  "d2h_bytes_per_step": res["d2h"], "ms_per_step": res["ms_e2e"] / args.steps,
                  **({"h2d_ms_per_step_alone": res["h2d_ms"], "d2h_ms_per_step_alone": res["d2h_ms"],
                      "h2d_gbs": res["h2d"] / (res["h2d_ms"] * 1e-3) / 1e9,
-                     "d2h_gbs": res["d2h"] / (res["d2h_ms"] * 1e-3) / 1e9} if "h2d_ms" in res else {}),
+                     "d2h_gbs": res["d2h"] / (res["d2h_ms"] * 1e-3) / 1e9,
+                     "bound_by": e2e_bound(res, args)} if "h2d_ms" in res else {}),
                  "copies": "pinned host buffers; each block's inputs in and outputs out on one stream per "
                            "direction, overlapping the neighbouring blocks' compute"}
                 if "ms_e2e" in res else None),

@@ -86,6 +86,17 @@ def test_report_l2_cold_prefix_figure(capsys):
     assert "L2" in line["config"]["l2"]
 
 
+@pytest.mark.parametrize("h2d_ms,d2h_ms,bound", [(0.1, 0.05, "compute"), (0.5, 0.05, "host-to-device copies"),
+                                                 (0.1, 0.3, "device-to-host copies")])
+def test_report_names_what_bounds_e2e(capsys, h2d_ms, d2h_ms, bound):
+    # a block's compute is 0.6 ms / 4 timed blocks = 0.15 ms
+    args = _args()
+    w = synth.WORKLOADS["long_ctx"].scaled(blocks=1)
+    bench.report(args, synth.WORKLOADS["long_ctx"], w, 1, _res(w, h2d_ms=h2d_ms, d2h_ms=d2h_ms))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["e2e"]["bound_by"] == bound
+
+
 def test_report_without_e2e_phase(capsys):
     args = _args(phases="cached")
     w = synth.WORKLOADS["long_ctx"].scaled(blocks=1)
